@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""bench.py -- the grouped NF4 W4A16 expert GEMM hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  moe_align (token->expert sort of topk_ids) -> grouped NF4 GEMM gate_up
+  (fused SwiGLU where the workload has it) -> grouped NF4 GEMM down,
+with sizes/expert_ids handed from the sort to the GEMMs on the device.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload olmoe|tiny|qwen3_30b_a3b|gpt_oss_120b|mixtral_8x22b]
+
+Prints ONE JSON line on rank 0. `value` is whole-job throughput (all ranks)
+of the metric: HBM GB/s for the decode workloads (algorithmic bytes: touched
+expert weights + absmax + x + y + sort I/O), TFLOP/s for the prefill workload
+(2*M*N*K per GEMM). With N > 1 every rank runs an independent replica (the
+decode path does not shard; weak scaling), the timed region is bracketed by a
+barrier + synchronize and its time is the max over ranks.
+
+Timing: CUDA events on the launching stream. Each step is a CUDA graph of the
+C-ABI calls (they are capture-safe: no host sync, no allocation). Weight
+stacks rotate over enough replicas that a step never finds its weights in
+L2. Per-kernel durations for the roofline come from external event nodes
+captured inside the step graphs (the last replay of each replica's graph).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "grouped NF4 GEMM: HBM GB/s & % roofline (decode); TFLOPS & % peak (prefill)"
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_STEPS = {"tiny": 20000, "olmoe": 20000, "qwen3_30b_a3b": 5000, "gpt_oss_120b": 500,
+                 "mixtral_8x22b": 100}
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def source_hash(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(kernel, workload, gemm):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        ent = d[kernel][f"{workload}.{gemm}"]
+        src = os.path.join(ROOT, "grouped_nf4_w4a16_b200", "csrc", ent["source"])
+        if source_hash(src) != ent["source_sha256"]:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class Clocks:
+    """nvidia-smi sampler (clocks and throttle reasons) around a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if ts < t0 or ts > t1:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _cuda_driver():
+    lib = ctypes.CDLL("libcuda.so.1")
+    lib.cuEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    lib.cuEventRecordWithFlags.restype = ctypes.c_int
+    return lib
+
+
+# ------------------------------------------------------------------ problem
+class Problem:
+    """Device-resident inputs for one workload (seeded, synthetic)."""
+
+    def __init__(self, name, seed=0, replicas=None, device="cuda"):
+        self.w = synth.WORKLOADS[name]
+        w = self.w
+        self.name = name
+        self.device = device
+        self.topk_np = synth.routing(w, seed)
+        self.U = int(np.unique(self.topk_np).size)
+        self.gemms = []
+        touched_bytes = 0
+        for g in w.gemms:
+            packed, absmax = synth.random_packed_stack(w.E, g.N, g.K, seed=seed, which=g.name)
+            x = synth.activations_bf16(w.M, g.K, seed=seed, which=g.name)
+            self.gemms.append(dict(g=g, packed_np=packed, absmax_np=absmax, x_np=x))
+            touched_bytes += self.U * g.N * g.K * 9 // 16
+        if replicas is None:
+            replicas = 1 if touched_bytes > 2 * L2_BYTES else 1 + -(-int(1.5 * L2_BYTES) // touched_bytes)
+        self.R = replicas
+        self.topk = torch.from_numpy(self.topk_np).to(device)
+        S = w.T * w.top_k
+        self.sorted_idx = torch.empty(S, dtype=torch.int32, device=device)
+        self.sizes = torch.empty(w.E, dtype=torch.int32, device=device)
+        self.expert_ids = torch.empty(w.E, dtype=torch.int32, device=device)
+        self.num_groups = torch.empty(1, dtype=torch.int32, device=device)
+        import grouped_nf4_w4a16_b200 as gnf4
+        self.gnf4 = gnf4
+        self.ws_align = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_MOE_ALIGN, S, E=w.E), device)
+        for d in self.gemms:
+            g = d["g"]
+            wd = torch.from_numpy(d["packed_np"]).to(device)
+            ad = torch.from_numpy(d["absmax_np"]).to(device)
+            d["W"] = [wd] + [wd.clone() for _ in range(self.R - 1)]
+            d["A"] = [ad] + [ad.clone() for _ in range(self.R - 1)]
+            d["x"] = torch.from_numpy(d["x_np"].view(np.int16)).to(device).view(torch.bfloat16)
+            n_out = g.N // 2 if g.swiglu else g.N
+            d["y"] = torch.empty((w.M, n_out), dtype=torch.bfloat16, device=device)
+            d["ws"] = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(
+                gnf4.GNF4_OP_GROUPED_GEMM, w.M, g.N, g.K, w.E, w.E), device)
+            d["epi"] = gnf4.GNF4_EPI_SWIGLU if g.swiglu else gnf4.GNF4_EPI_NONE
+        # algorithmic work per step
+        self.align_bytes = S * 4 + S * 4 + 2 * w.E * 4 + 4
+        for d in self.gemms:
+            g = d["g"]
+            n_out = g.N // 2 if g.swiglu else g.N
+            d["bytes"] = self.U * g.N * g.K * 9 // 16 + w.M * g.K * 2 + w.M * n_out * 2
+            d["flops"] = 2 * w.M * g.N * g.K
+        self.step_bytes = self.align_bytes + sum(d["bytes"] for d in self.gemms)
+        self.step_flops = sum(d["flops"] for d in self.gemms)
+        self.prefill = w.regime == "prefill"
+
+    def launch(self, r, events=None, drv=None, stream=None):
+        """Enqueue one step with weight replica r (optionally recording events)."""
+        gnf4 = self.gnf4
+
+        def ev(i):
+            if events is not None:
+                drv.cuEventRecordWithFlags(ctypes.c_void_p(events[i].cuda_event),
+                                           ctypes.c_void_p(stream.cuda_stream), 1)
+        ev(0)
+        gnf4.gnf4_moe_align(self.topk, self.w.E, sorted_idx=self.sorted_idx, sizes=self.sizes,
+                            expert_ids=self.expert_ids, num_groups=self.num_groups,
+                            workspace=self.ws_align)
+        ev(1)
+        for i, d in enumerate(self.gemms):
+            gnf4.gnf4_grouped_gemm(d["x"], d["W"][r], d["A"][r], self.sizes, self.expert_ids,
+                                   epilogue=d["epi"], y=d["y"], workspace=d["ws"])
+            ev(2 + i)
+
+    def describe(self):
+        w = self.w
+        return {
+            "workload": f"{w.name}: {w.description}",
+            "E": w.E, "top_k": w.top_k, "tokens": w.T, "rows": w.M,
+            "gemms": [f"{d['g'].name} K={d['g'].K} N={d['g'].N}" + (" +SwiGLU" if d['g'].swiglu else "")
+                      for d in self.gemms],
+            "touched_experts": self.U,
+            "weights": "uniform random NF4 codes, absmax U[0.04,0.06] (values do not affect timing)",
+            "l2": (f"{self.R} weight-stack replicas rotated per step "
+                   f"(touched bytes of the other replicas > L2)" if self.R > 1 else
+                   "touched weights per step > 2x L2 (no replica needed)"),
+            "graph": "each step is one CUDA graph of the C-ABI calls",
+        }
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    prob = Problem(args.workload, seed=0, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    drv = _cuda_driver()
+    nk = 1 + len(prob.gemms)
+    # one graph per weight replica, with external event nodes around each kernel
+    graphs, evs = [], []
+    with torch.cuda.stream(stream):
+        for r in range(prob.R):      # eager warm-up (sets kernel attributes, first-call work)
+            prob.launch(r)
+        torch.cuda.synchronize()
+        for r in range(prob.R):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                prob.launch(r, events=e, drv=drv, stream=stream)
+            graphs.append(g)
+            evs.append(e)
+    torch.cuda.synchronize()
+    launches_per_step = nk
+
+    clocks = Clocks(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % prob.R].replay()
+        # keep the GPU busy for ~0.5 s before timing so clocks settle
+        t_end = time.time() + 0.5
+        i = 0
+        while time.time() < t_end:
+            graphs[i % prob.R].replay()
+            i += 1
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            graphs[i % prob.R].replay()
+    stop.record(stream)
+    stop.synchronize()
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    # clock window: if the timed region was short, keep replaying the same
+    # steps for ~1 s so the sampler sees this workload under load
+    if t1 - t0 < 1.0:
+        with torch.cuda.stream(stream):
+            t_end = time.time() + 1.0
+            i = 0
+            while time.time() < t_end:
+                graphs[i % prob.R].replay()
+                i += 1
+        stream.synchronize()
+    t2 = time.time()
+    clk = clocks.stop(t0, t2)
+
+    # per-kernel durations: external event nodes of the last replay of each replica graph
+    per_kernel = [[] for _ in range(nk)]
+    for e in evs:
+        for k in range(nk):
+            per_kernel[k].append(e[k].elapsed_time(e[k + 1]))
+    kern_ms = [sum(v) / len(v) for v in per_kernel]
+
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end: host (pinned) inputs -> device, the C-ABI calls, results -> host
+    e2e = run_e2e(prob, stream, max(3, min(args.steps, 2000) // 10))
+    return prob, ms, kern_ms, clk, e2e, launches_per_step
+
+
+def run_e2e(prob, stream, steps):
+    gnf4 = prob.gnf4
+    dev = prob.topk.device
+    h_topk = torch.from_numpy(prob.topk_np).pin_memory()
+    h_x = [torch.from_numpy(d["x_np"].view(np.int16)).pin_memory() for d in prob.gemms]
+    h_y = [torch.empty(d["y"].shape, dtype=torch.int16).pin_memory() for d in prob.gemms]
+    d_topk = torch.empty_like(prob.topk)
+    d_x = [torch.empty(d["x"].shape, dtype=torch.int16, device=dev) for d in prob.gemms]
+    h2d = h_topk.numel() * 4 + sum(t.numel() * 2 for t in h_x)
+    d2h = sum(t.numel() * 2 for t in h_y)
+
+    def one(r):
+        d_topk.copy_(h_topk, non_blocking=True)
+        for a, b in zip(d_x, h_x):
+            a.copy_(b, non_blocking=True)
+        gnf4.gnf4_moe_align(d_topk, prob.w.E, sorted_idx=prob.sorted_idx, sizes=prob.sizes,
+                            expert_ids=prob.expert_ids, num_groups=prob.num_groups,
+                            workspace=prob.ws_align)
+        for i, d in enumerate(prob.gemms):
+            gnf4.gnf4_grouped_gemm(d_x[i].view(torch.bfloat16), d["W"][r], d["A"][r], prob.sizes,
+                                   prob.expert_ids, epilogue=d["epi"], y=d["y"],
+                                   workspace=d["ws"])
+            h_y[i].copy_(d["y"].view(torch.int16), non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            one(i % prob.R)
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            one(i % prob.R)
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h, steps
+
+
+# -------------------------------------------------------- oracle (CPU) arm
+def oracle_step_sample(prob, budget_s):
+    """Time the CPU oracle on a bounded sample of the step. Returns
+    (seconds per full step, description, threads)."""
+    import oracle
+    w = prob.w
+    nthreads = oracle.num_threads()
+    t_align = time.perf_counter()
+    _, sizes, experts, _ = oracle.moe_align(prob.topk_np, w.E)
+    t_align = time.perf_counter() - t_align
+    # rows per GEMM: all rows if a full step fits the budget, else a row sample
+    per_row = []
+    for d in prob.gemms:
+        rows = np.array([0, w.M - 1])
+        t = time.perf_counter()
+        oracle.grouped_gemm_f64(d["x_np"], d["packed_np"], d["absmax_np"], sizes, experts, rows=rows)
+        per_row.append((time.perf_counter() - t) / rows.size)
+    full_est = t_align + sum(per_row) * w.M
+    if full_est <= budget_s / 3:
+        n = 0
+        t = time.perf_counter()
+        while True:
+            oracle.moe_align(prob.topk_np, w.E)
+            for d in prob.gemms:
+                y = oracle.grouped_gemm_f64(d["x_np"], d["packed_np"], d["absmax_np"], sizes, experts)
+                if d["g"].swiglu:
+                    oracle.swiglu_f64(y)
+            n += 1
+            if time.perf_counter() - t >= budget_s:
+                break
+        sec = (time.perf_counter() - t) / n
+        return sec, f"{n} full steps (all {w.M} rows, every GEMM) in {sec * n:.1f} s", nthreads
+    # row sample: rows spread over the groups, time scaled by M / rows
+    k = max(nthreads, int(budget_s / max(sum(per_row), 1e-9)))
+    k = min(k, w.M)
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(w.M, size=k, replace=False))
+    t = time.perf_counter()
+    oracle.moe_align(prob.topk_np, w.E)
+    for d in prob.gemms:
+        oracle.grouped_gemm_f64(d["x_np"], d["packed_np"], d["absmax_np"], sizes, experts, rows=rows)
+    el = time.perf_counter() - t
+    sec = t_align + (el - t_align) * w.M / k
+    return sec, (f"{k} of {w.M} rows per GEMM (seeded sample) in {el:.1f} s; full-step time "
+                 f"extrapolated x{w.M / k:.1f} by rows"), nthreads
+
+
+def metric_value(prob, sec_per_step, n_ranks=1):
+    if prob.prefill:
+        return prob.step_flops * n_ranks / sec_per_step / 1e12, "TFLOP/s"
+    return prob.step_bytes * n_ranks / sec_per_step / 1e9, "GB/s"
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    prob = Problem(args.workload, seed=0, device="cuda" if torch.cuda.is_available() else "cpu") \
+        if torch.cuda.is_available() else None
+    if prob is None:
+        raise SystemExit("the reference arm builds its inputs with the same generator on the GPU box")
+    budget = max(3.0, min(60.0, 2.0 * (args.steps + args.warmup)))
+    sec, sample, threads = oracle_step_sample(prob, budget)
+    val, unit = metric_value(prob, sec)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": prob.describe(),
+        "cpu_baseline": {"value": val, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="olmoe", choices=list(synth.WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of CPU time for the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
+    if args.warmup is None:
+        args.warmup = max(3, args.steps // 20)
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            "nccl", device_id=torch.device("cuda", local_rank),
+            timeout=__import__("datetime").timedelta(seconds=120))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    import grouped_nf4_w4a16_b200 as gnf4
+    gnf4.load_library()    # fails loudly if the CUDA library is missing
+    prob, ms, kern_ms, clk, e2e, lps = run_ours(args, rank, world, local_rank)
+    sec = ms / 1e3 / args.steps
+    val, unit = metric_value(prob, sec, world)
+    pk = peaks()
+
+    # roofline of the dominant kernel: the gate_up grouped GEMM launch
+    d0 = prob.gemms[0]
+    k_ms = kern_ms[1]
+    kernel = "prefill_gemm" if prob.prefill else "decode_gemm_kernel"
+    if prob.prefill:
+        achieved = d0["flops"] / (k_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "traffic": traffic_for(kernel, prob.name, "gate_up")}
+    else:
+        achieved = d0["bytes"] / (k_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(kernel, prob.name, "gate_up")}
+    roof["kernel"] = f"{kernel} ({d0['g'].name} launch)"
+    roof["algorithmic_per_launch"] = d0["flops"] if prob.prefill else d0["bytes"]
+    roof["launch_ms"] = k_ms
+    roof["peak_source"] = f"{pk['source']} (MEASURED_PEAKS.json)" if pk["source"] == "measured" else "fallback"
+
+    kernels = {"moe_align": {"ms": kern_ms[0]}}
+    for i, d in enumerate(prob.gemms):
+        entry = {"ms": kern_ms[1 + i], "GB/s": d["bytes"] / (kern_ms[1 + i] / 1e3) / 1e9}
+        if prob.prefill:
+            entry["TFLOP/s"] = d["flops"] / (kern_ms[1 + i] / 1e3) / 1e12
+        kernels[d["g"].name] = entry
+
+    e2e_ms, h2d, d2h, e2e_steps = e2e
+    e2e_val, _ = metric_value(prob, e2e_ms / 1e3, world)
+    line = {
+        "metric": METRIC, "value": val, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": prob.describe(),
+        "roofline": roof,
+        "kernels": kernels,
+        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "eager C-ABI calls; pinned host inputs copied in and results copied out every step"},
+        "gpu_launches": lps * args.steps,
+        "clocks": clk,
+    }
+    line["config"]["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec_cpu, sample, threads = oracle_step_sample(prob, args.cpu_budget)
+        v, u = metric_value(prob, sec_cpu)
+        line["cpu_baseline"] = {"value": v, "unit": u, "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,33 @@
+"""grouped_nf4_w4a16_b200 -- grouped MoE expert GEMM on NF4-packed weights, B200.
+
+The compute lives in ``libgnf4.so`` (hand-written CUDA for sm_100a, C ABI in
+``include/gnf4.h``). This package is a thin ctypes binding with the same entry
+point names; it only marshals arguments (tensor -> pointer, current stream).
+There is no CPU or PyTorch fallback: without the built library every entry
+point raises.
+"""
+from .binding import (  # noqa: F401
+    Gnf4Error,
+    GNF4_OK,
+    GNF4_EPI_NONE,
+    GNF4_EPI_SWIGLU,
+    GNF4_MODE_AUTO,
+    GNF4_MODE_DECODE,
+    GNF4_MODE_PREFILL,
+    GNF4_OUT_F32,
+    GNF4_OUT_BF16,
+    GNF4_OP_MOE_ALIGN,
+    GNF4_OP_GROUPED_GEMM,
+    DEVERR_BITS,
+    EXPORTED_SYMBOLS,
+    library_path,
+    load_library,
+    gnf4_version,
+    gnf4_status_string,
+    gnf4_workspace_bytes,
+    gnf4_moe_align,
+    gnf4_grouped_gemm,
+    gnf4_dequant_debug,
+    gnf4_read_device_status,
+    make_workspace,
+)

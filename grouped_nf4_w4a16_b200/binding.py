@@ -1,0 +1,194 @@
+"""ctypes binding of libgnf4 (argument marshalling only; see include/gnf4.h).
+
+Every function here turns tensors into device pointers, picks the current CUDA
+stream and calls the C entry point of the same name; every step of the
+computation runs in the library's kernels. Tensors must already be on the
+GPU: the library refuses host memory (GNF4_ERR_HOST_POINTER) and this module
+never copies on the caller's behalf.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgnf4.so")
+
+GNF4_OK = 0
+_STATUS_NAMES = {
+    0: "GNF4_OK", 1: "GNF4_ERR_INVALID_ARGUMENT", 2: "GNF4_ERR_HOST_POINTER",
+    3: "GNF4_ERR_UNSUPPORTED_SHAPE", 4: "GNF4_ERR_WORKSPACE_TOO_SMALL", 5: "GNF4_ERR_CUDA",
+    6: "GNF4_ERR_DEVICE_METADATA", 7: "GNF4_ERR_TIMEOUT", 8: "GNF4_ERR_MISALIGNED",
+}
+GNF4_EPI_NONE, GNF4_EPI_SWIGLU = 0, 1
+GNF4_MODE_AUTO, GNF4_MODE_DECODE, GNF4_MODE_PREFILL = 0, 1, 2
+GNF4_OUT_F32, GNF4_OUT_BF16 = 0, 1
+GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM = 0, 1
+DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capacity": 0x10}
+
+# Every symbol include/gnf4.h declares.
+EXPORTED_SYMBOLS = (
+    "gnf4_moe_align", "gnf4_grouped_gemm", "gnf4_dequant_debug", "gnf4_workspace_bytes",
+    "gnf4_read_device_status", "gnf4_status_string", "gnf4_version",
+)
+
+_lib = None
+
+
+class Gnf4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libgnf4.so; raise if it is missing (there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"{_LIB_PATH} is missing: build it with `python -m grouped_nf4_w4a16_b200.build` "
+            "(this package has no CPU or PyTorch fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.gnf4_moe_align.argtypes = [P, i64, i32, i32, P, P, P, P, P, sz, P]
+    lib.gnf4_moe_align.restype = ctypes.c_int
+    lib.gnf4_grouped_gemm.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P,
+                                      P, sz, P]
+    lib.gnf4_grouped_gemm.restype = ctypes.c_int
+    lib.gnf4_dequant_debug.argtypes = [P, P, i64, i32, i32, i32, P, P]
+    lib.gnf4_dequant_debug.restype = ctypes.c_int
+    lib.gnf4_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
+    lib.gnf4_workspace_bytes.restype = sz
+    lib.gnf4_read_device_status.argtypes = [P, i32, ctypes.POINTER(ctypes.c_uint32), P]
+    lib.gnf4_read_device_status.restype = ctypes.c_int
+    lib.gnf4_status_string.argtypes = [ctypes.c_int]
+    lib.gnf4_status_string.restype = ctypes.c_char_p
+    lib.gnf4_version.argtypes = []
+    lib.gnf4_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(st: int, where: str):
+    if st != GNF4_OK:
+        raise Gnf4Error(st, where)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gnf4_version() -> int:
+    return int(load_library().gnf4_version())
+
+
+def gnf4_status_string(status: int) -> str:
+    return load_library().gnf4_status_string(int(status)).decode()
+
+
+def gnf4_workspace_bytes(op: int, M: int, N: int = 1, K: int = 64, E: int = 1, G: int = 1) -> int:
+    return int(load_library().gnf4_workspace_bytes(op, M, N, K, E, G))
+
+
+def make_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled byte buffer usable as a workspace (zero it once, reuse it)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def gnf4_moe_align(topk_ids: torch.Tensor, E: int, *, sorted_idx=None, sizes=None,
+                   expert_ids=None, num_groups=None, workspace=None, stream=None):
+    """-> (sorted_idx [T*k], sizes [E], expert_ids [E], num_groups [1]) int32 device tensors."""
+    _need(topk_ids, "topk_ids", torch.int32)
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    sorted_idx = sorted_idx if sorted_idx is not None else torch.empty(T * k, dtype=torch.int32, device=dev)
+    sizes = sizes if sizes is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    expert_ids = expert_ids if expert_ids is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    num_groups = num_groups if num_groups is not None else torch.empty(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = make_workspace(gnf4_workspace_bytes(GNF4_OP_MOE_ALIGN, T * k, E=E), dev)
+    st = load_library().gnf4_moe_align(
+        _ptr(topk_ids), T, k, E, _ptr(sorted_idx), _ptr(sizes), _ptr(expert_ids), _ptr(num_groups),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "gnf4_moe_align")
+    return sorted_idx, sizes, expert_ids, num_groups
+
+
+def gnf4_grouped_gemm(x: torch.Tensor, w: torch.Tensor, absmax: torch.Tensor, sizes: torch.Tensor,
+                      expert_ids: torch.Tensor, *, epilogue: int = GNF4_EPI_NONE,
+                      mode: int = GNF4_MODE_AUTO, y: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, blocksize: int = 64,
+                      stream=None) -> torch.Tensor:
+    """y = grouped NF4 GEMM of x [M,K] bf16 with w [E,N,K/2] uint8 / absmax [E,N,K/64] fp32."""
+    _need(x, "x", torch.bfloat16)
+    _need(w, "w", torch.uint8)
+    _need(absmax, "absmax", torch.float32)
+    _need(sizes, "sizes", torch.int32)
+    _need(expert_ids, "expert_ids", torch.int32)
+    M, K = x.shape
+    E, N, Kh = w.shape
+    if Kh * 2 != K:
+        raise ValueError(f"w has K/2={Kh} but x has K={K}")
+    G = sizes.numel()
+    n_out = N // 2 if epilogue == GNF4_EPI_SWIGLU else N
+    if y is None:
+        y = torch.empty((M, n_out), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(y, "y", torch.bfloat16)
+    if workspace is None:
+        workspace = make_workspace(gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G), x.device)
+    st = load_library().gnf4_grouped_gemm(
+        _ptr(x), _ptr(w), _ptr(absmax), _ptr(sizes), _ptr(expert_ids), G, M, N, K, E, blocksize,
+        epilogue, mode, _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "gnf4_grouped_gemm")
+    return y
+
+
+def gnf4_dequant_debug(w: torch.Tensor, absmax: torch.Tensor, out_dtype: int = GNF4_OUT_F32, *,
+                       out: Optional[torch.Tensor] = None, blocksize: int = 64,
+                       stream=None) -> torch.Tensor:
+    """NF4[code] * absmax for every element: fp32 (or bf16) [..., K]."""
+    _need(w, "w", torch.uint8)
+    _need(absmax, "absmax", torch.float32)
+    K = w.shape[-1] * 2
+    rows = w.numel() // w.shape[-1] if w.numel() else 0
+    dt = torch.bfloat16 if out_dtype == GNF4_OUT_BF16 else torch.float32
+    if out is None:
+        out = torch.empty(tuple(w.shape[:-1]) + (K,), dtype=dt, device=w.device)
+    st = load_library().gnf4_dequant_debug(_ptr(w), _ptr(absmax), rows, K, blocksize, out_dtype,
+                                           _ptr(out), _stream(stream))
+    _check(st, "gnf4_dequant_debug")
+    return out
+
+
+def gnf4_read_device_status(workspace: torch.Tensor, clear: bool = True,
+                            stream=None) -> Tuple[int, int]:
+    """Synchronise and read the workspace error word -> (status, GNF4_DEVERR bits)."""
+    bits = ctypes.c_uint32(0)
+    st = load_library().gnf4_read_device_status(_ptr(workspace), 1 if clear else 0,
+                                                ctypes.byref(bits), _stream(stream))
+    return int(st), int(bits.value)

@@ -1,0 +1,189 @@
+// api.cu -- the extern "C" entry points of libgnf4 (see include/gnf4.h).
+//
+// Host-side argument checks (synchronous, before any launch), mode choice and
+// kernel launches on the caller's stream. No allocation, no synchronisation
+// (except gnf4_read_device_status), no host fallback: the package page
+// "grouped-nf4-gemm" ("Do not use this when") states that nothing falls back
+// silently on the CPU and host tensors are refused with an error.
+#include <climits>
+#include <cstring>
+
+#include "launch.h"
+
+namespace gnf4 {
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+namespace {
+
+bool is_device_pointer(const void *p) {
+  cudaPointerAttributes attr;
+  std::memset(&attr, 0, sizeof(attr));
+  const cudaError_t err = cudaPointerGetAttributes(&attr, p);
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();   // clear the sticky error of a bad query
+    return false;
+  }
+  return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+gnf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GNF4_OK : GNF4_ERR_CUDA; }
+
+// Mean rows per possible group above which the tensor-core kernel is used.
+constexpr int64_t kPrefillMeanRows = 64;
+
+}  // namespace
+}  // namespace gnf4
+
+using namespace gnf4;
+
+extern "C" {
+
+int32_t gnf4_version(void) { return GNF4_VERSION; }
+
+const char *gnf4_status_string(gnf4_status s) {
+  switch (s) {
+    case GNF4_OK: return "GNF4_OK";
+    case GNF4_ERR_INVALID_ARGUMENT: return "GNF4_ERR_INVALID_ARGUMENT";
+    case GNF4_ERR_HOST_POINTER: return "GNF4_ERR_HOST_POINTER (a pointer is not device memory; there is no host path)";
+    case GNF4_ERR_UNSUPPORTED_SHAPE: return "GNF4_ERR_UNSUPPORTED_SHAPE";
+    case GNF4_ERR_WORKSPACE_TOO_SMALL: return "GNF4_ERR_WORKSPACE_TOO_SMALL";
+    case GNF4_ERR_CUDA: return "GNF4_ERR_CUDA";
+    case GNF4_ERR_DEVICE_METADATA: return "GNF4_ERR_DEVICE_METADATA";
+    case GNF4_ERR_TIMEOUT: return "GNF4_ERR_TIMEOUT";
+    case GNF4_ERR_MISALIGNED: return "GNF4_ERR_MISALIGNED";
+  }
+  return "GNF4_ERR_UNKNOWN";
+}
+
+size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t E, int32_t G) {
+  (void)E;
+  if (op == GNF4_OP_MOE_ALIGN) return kWsHeaderBytes;
+  if (op != GNF4_OP_GROUPED_GEMM || M < 0 || N < 1 || K < 1 || G < 1) return 0;
+  const size_t d = decode_workspace_bytes(M, N, K, G, 1);
+  const size_t d2 = decode_workspace_bytes(M, N, K, G, 0);
+  const size_t p = prefill_workspace_bytes(M, N, K, G, 0);
+  const size_t p2 = prefill_workspace_bytes(M, N, K, G, 1);
+  size_t r = d > d2 ? d : d2;
+  if (p > r) r = p;
+  if (p2 > r) r = p2;
+  return r;
+}
+
+gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t top_k, int32_t E,
+                           int32_t *sorted_idx, int32_t *sizes, int32_t *expert_ids,
+                           int32_t *num_groups, void *workspace, size_t ws_bytes,
+                           gnf4_stream_t stream) {
+  if (T < 0 || top_k < 1 || E < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if ((T > 0 && (!topk_ids || !sorted_idx)) || !sizes || !expert_ids || !num_groups || !workspace)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (E > GNF4_MAX_EXPERTS || T * static_cast<int64_t>(top_k) >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < kWsHeaderBytes) return GNF4_ERR_WORKSPACE_TOO_SMALL;
+  const bool need_ids = T > 0;
+  if ((need_ids && (!is_device_pointer(topk_ids) || !is_device_pointer(sorted_idx))) ||
+      !is_device_pointer(sizes) || !is_device_pointer(expert_ids) ||
+      !is_device_pointer(num_groups) || !is_device_pointer(workspace))
+    return GNF4_ERR_HOST_POINTER;
+  if ((need_ids && (!aligned(topk_ids, 4) || !aligned(sorted_idx, 4))) || !aligned(sizes, 4) ||
+      !aligned(expert_ids, 4) || !aligned(num_groups, 4) || !aligned(workspace, 16))
+    return GNF4_ERR_MISALIGNED;
+  const int32_t S = static_cast<int32_t>(T * top_k);
+  return from_cuda(launch_moe_align(topk_ids, S, E, sorted_idx, sizes, expert_ids, num_groups,
+                                    static_cast<WsHeader *>(workspace),
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *absmax,
+                              const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                              int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                              int32_t epilogue, int32_t mode, uint16_t *y, void *workspace,
+                              size_t ws_bytes, gnf4_stream_t stream) {
+  if (!x || !w || !absmax || !sizes || !expert_ids || !y || !workspace)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (epilogue != GNF4_EPI_NONE && epilogue != GNF4_EPI_SWIGLU) return GNF4_ERR_INVALID_ARGUMENT;
+  if (mode != GNF4_MODE_AUTO && mode != GNF4_MODE_DECODE && mode != GNF4_MODE_PREFILL)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return GNF4_OK;
+  if (!is_device_pointer(x) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
+      !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(y) ||
+      !is_device_pointer(workspace))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(x, 32) || !aligned(w, 32) || !aligned(y, 32) || !aligned(workspace, 32) ||
+      !aligned(absmax, 4) || !aligned(sizes, 4) || !aligned(expert_ids, 4))
+    return GNF4_ERR_MISALIGNED;
+  if (ws_bytes < gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G))
+    return GNF4_ERR_WORKSPACE_TOO_SMALL;
+
+  GemmArgs a;
+  a.x = x; a.w = w; a.absmax = absmax; a.sizes = sizes; a.expert_ids = expert_ids;
+  a.G = G; a.M = M; a.N = N; a.K = K; a.E = E; a.swiglu = (epilogue == GNF4_EPI_SWIGLU);
+  a.y = y; a.workspace = workspace; a.ws_bytes = ws_bytes;
+
+  int32_t use = mode;
+  if (use == GNF4_MODE_AUTO) {
+    const int64_t groups = G < E ? G : E;
+    use = (M > kPrefillMeanRows * groups) ? GNF4_MODE_PREFILL : GNF4_MODE_DECODE;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use == GNF4_MODE_PREFILL) {
+    const cudaError_t e = launch_prefill_gemm(a, s);
+    if (e == cudaErrorNotSupported) return GNF4_ERR_UNSUPPORTED_SHAPE;
+    return from_cuda(e);
+  }
+  return from_cuda(launch_decode_gemm(a, s));
+}
+
+gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,
+                               int32_t blocksize, int32_t out_dtype, void *out,
+                               gnf4_stream_t stream) {
+  if (!w || !absmax || !out) return GNF4_ERR_INVALID_ARGUMENT;
+  if (rows < 0 || K < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (out_dtype != GNF4_OUT_F32 && out_dtype != GNF4_OUT_BF16) return GNF4_ERR_INVALID_ARGUMENT;
+  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return GNF4_OK;
+  if (!is_device_pointer(w) || !is_device_pointer(absmax) || !is_device_pointer(out))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(w, 16) || !aligned(out, 16) || !aligned(absmax, 4)) return GNF4_ERR_MISALIGNED;
+  return from_cuda(launch_dequant(w, absmax, rows, K, out_dtype == GNF4_OUT_BF16 ? 1 : 0, out,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uint32_t *error_bits,
+                                    gnf4_stream_t stream) {
+  if (!workspace) return GNF4_ERR_INVALID_ARGUMENT;
+  if (!is_device_pointer(workspace)) return GNF4_ERR_HOST_POINTER;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && clear) {
+    e = cudaMemsetAsync(workspace, 0, sizeof(h), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return GNF4_ERR_CUDA;
+  if (error_bits) *error_bits = h[0];
+  if (h[0] & (GNF4_DEVERR_SIZES | GNF4_DEVERR_EXPERT | GNF4_DEVERR_TOPK | GNF4_DEVERR_CAPACITY))
+    return GNF4_ERR_DEVICE_METADATA;
+  if (h[0] & GNF4_DEVERR_TIMEOUT) return GNF4_ERR_TIMEOUT;
+  return GNF4_OK;
+}
+
+}  // extern "C"

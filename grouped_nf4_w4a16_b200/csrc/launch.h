@@ -1,0 +1,51 @@
+// launch.h -- internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace gnf4 {
+
+// Grouped GEMM problem as seen by the kernels (all pointers device memory).
+struct GemmArgs {
+  const uint16_t *x;        // bf16 [M][K]
+  const uint8_t *w;         // [E][N][K/2]
+  const float *absmax;      // [E][N][K/64]
+  const int32_t *sizes;     // [G]
+  const int32_t *expert_ids;// [G]
+  int32_t G;
+  int64_t M;
+  int32_t N;
+  int32_t K;
+  int32_t E;
+  int32_t swiglu;           // 0 / 1
+  uint16_t *y;              // bf16 [M][N] or [M][N/2]
+  void *workspace;
+  size_t ws_bytes;
+};
+
+// ---- moe_align (moe_align.cu)
+size_t moe_align_smem_bytes(int32_t E);
+cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t *sorted_idx,
+                             int32_t *sizes, int32_t *expert_ids, int32_t *num_groups,
+                             WsHeader *hdr, cudaStream_t stream);
+
+// ---- dequant_debug (dequant.cu)
+cudaError_t launch_dequant(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,
+                           int out_bf16, void *out, cudaStream_t stream);
+
+// ---- decode-regime grouped GEMM (decode_gemm.cu)
+size_t decode_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu);
+cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream);
+
+// ---- prefill-regime grouped GEMM (prefill_gemm.cu)
+size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu);
+cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace gnf4

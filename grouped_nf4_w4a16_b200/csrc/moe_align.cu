@@ -1,0 +1,144 @@
+// moe_align.cu -- stable counting sort of token->expert slots (one CTA).
+//
+// Passage: "grouped-nf4-gemm -- single-launch W4A16 GEMM over fused NF4 MoE
+// expert stacks", opening section: (sizes, expert_ids) are supplied after the
+// usual token->expert sort. The sort fixed here (gnf4.h documents it):
+// groups = non-empty experts in ascending id, slots ascending within a group.
+//
+// Design: a single 1024-thread CTA, everything in shared memory, one launch.
+//   1. each warp owns a contiguous segment of the S = T*top_k slots and builds
+//      its own per-expert histogram (shared-memory atomics);
+//   2. per expert, an exclusive scan over the 32 warp histograms gives each
+//      warp its starting rank inside the expert's group;
+//   3. a block scan over experts gives each expert's first output position and
+//      each non-empty expert its group index;
+//   4. each warp walks its segment 32 slots at a time; lanes holding the same
+//      expert find each other with __match_any_sync and take consecutive
+//      positions in lane order, so the output is stable without atomics.
+// The decode-regime problems this serves have at most a few thousand slots;
+// the kernel is latency-bound (a few microseconds).
+#include "launch.h"
+
+namespace gnf4 {
+namespace {
+
+constexpr int kAlignThreads = 1024;
+constexpr int kAlignWarps = kAlignThreads / 32;
+
+__global__ void __launch_bounds__(kAlignThreads, 1)
+    moe_align_kernel(const int32_t *__restrict__ topk, int32_t S, int32_t E,
+                     int32_t *__restrict__ sorted_idx, int32_t *__restrict__ sizes,
+                     int32_t *__restrict__ expert_ids, int32_t *__restrict__ num_groups,
+                     WsHeader *hdr) {
+  extern __shared__ int32_t sm[];
+  int32_t *hist = sm;                        // [kAlignWarps][E]
+  int32_t *start = hist + kAlignWarps * E;   // [E] first output position of each expert
+  __shared__ int32_t warp_sum_v[kAlignWarps];
+  __shared__ int32_t warp_sum_f[kAlignWarps];
+  __shared__ int32_t s_valid, s_groups;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) hist[i] = 0;
+  __syncthreads();
+
+  const int seg = (S + kAlignWarps - 1) / kAlignWarps;
+  const int beg = min(S, warp * seg), end = min(S, beg + seg);
+
+  // 1. per-warp histograms
+  for (int s = beg + lane; s < end; s += 32) {
+    const int e = topk[s];
+    if (e >= 0 && e < E) {
+      atomicAdd(&hist[warp * E + e], 1);
+    } else {
+      report_error(hdr, GNF4_DEVERR_TOPK, static_cast<uint32_t>(s));
+    }
+  }
+  __syncthreads();
+
+  // 2. per expert: exclusive scan over warps (E <= 1024: one expert per thread)
+  int tot = 0;
+  if (tid < E) {
+    for (int w = 0; w < kAlignWarps; ++w) {
+      const int c = hist[w * E + tid];
+      hist[w * E + tid] = tot;
+      tot += c;
+    }
+  }
+  const int flag = (tid < E && tot > 0) ? 1 : 0;
+
+  // 3. block exclusive scans over experts of counts (v) and non-empty flags (f)
+  int v = tot, f = flag;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, v, o);
+    const int b = __shfl_up_sync(0xffffffffu, f, o);
+    if (lane >= o) { v += a; f += b; }
+  }
+  if (lane == 31) { warp_sum_v[warp] = v; warp_sum_f[warp] = f; }
+  __syncthreads();
+  if (warp == 0) {
+    const int a0 = warp_sum_v[lane], b0 = warp_sum_f[lane];
+    int a = a0, b = b0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ua = __shfl_up_sync(0xffffffffu, a, o);
+      const int ub = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) { a += ua; b += ub; }
+    }
+    warp_sum_v[lane] = a - a0;
+    warp_sum_f[lane] = b - b0;
+    if (lane == 31) { s_valid = a; s_groups = b; }
+  }
+  __syncthreads();
+  const int excl_v = v - tot + warp_sum_v[warp];
+  const int excl_f = f - flag + warp_sum_f[warp];
+  if (tid < E) {
+    start[tid] = excl_v;
+    if (flag) { sizes[excl_f] = tot; expert_ids[excl_f] = tid; }
+  }
+  __syncthreads();
+  const int ngroups = s_groups;
+  for (int g = ngroups + tid; g < E; g += kAlignThreads) { sizes[g] = 0; expert_ids[g] = -1; }
+  if (tid == 0) *num_groups = ngroups;
+
+  // 4. stable scatter, 32 slots per warp step
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = beg; base < end; base += 32) {
+    const int s = base + lane;
+    const int e = (s < end) ? topk[s] : -1;
+    const bool ok = (s < end) && e >= 0 && e < E;
+    const int key = ok ? e : -1 - lane;   // invalid lanes never match each other
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(peers & lt_mask);
+    const int cur = ok ? hist[warp * E + e] : 0;
+    __syncwarp();
+    if (ok) {
+      sorted_idx[start[e] + cur + rank] = s;
+      if (rank == 0) hist[warp * E + e] = cur + __popc(peers);
+    }
+    __syncwarp();
+  }
+  // slots with an invalid id are left out; pad the tail of the permutation
+  for (int i = s_valid + tid; i < S; i += kAlignThreads) sorted_idx[i] = -1;
+}
+
+}  // namespace
+
+size_t moe_align_smem_bytes(int32_t E) {
+  return static_cast<size_t>(kAlignWarps + 1) * static_cast<size_t>(E) * sizeof(int32_t);
+}
+
+cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t *sorted_idx,
+                             int32_t *sizes, int32_t *expert_ids, int32_t *num_groups,
+                             WsHeader *hdr, cudaStream_t stream) {
+  const size_t smem = moe_align_smem_bytes(E);
+  cudaError_t err = cudaFuncSetAttribute(moe_align_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  moe_align_kernel<<<1, kAlignThreads, smem, stream>>>(topk, S, E, sorted_idx, sizes, expert_ids,
+                                                       num_groups, hdr);
+  return cudaGetLastError();
+}
+
+}  // namespace gnf4

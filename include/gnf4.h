@@ -1,0 +1,209 @@
+/*
+ * gnf4.h -- C ABI of libgnf4: the grouped MoE expert GEMM computed directly on
+ * NF4-packed weights, for NVIDIA B200 (sm_100a).
+ *
+ * Source of the operation: "grouped-nf4-gemm -- single-launch W4A16 GEMM over
+ * fused NF4 MoE expert stacks" (PyPI README of grouped_nf4_gemm 0.1.0), opening
+ * section: one launch over all active experts; LUT decode of 4-bit NF4 codes,
+ * blockwise fp32 absmax, fp32 accumulation, bf16 epilogue; no per-expert
+ * dequantise-then-matmul and no bf16 weight copy; inputs in the bitsandbytes
+ * gemm_4bit layout, [E, N, K/2] uint8 plus fp32 blockwise absmax, with
+ * (sizes, expert_ids) supplied after the token->expert sort. The package page
+ * "grouped-nf4-gemm" ("Do not use this when") adds that nothing falls back
+ * silently: host tensors are refused with an error.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Plain pointers and sizes only. The caller owns all memory: inputs,
+ *    outputs and the workspace. The library allocates nothing.
+ *  - All work is enqueued asynchronously on `stream` (NULL = legacy default
+ *    stream). No entry point synchronises the stream or copies to the host,
+ *    except gnf4_read_device_status, which exists to do exactly that.
+ *  - Host-side checks run first and synchronously; on failure nothing is
+ *    launched and a status != GNF4_OK is returned. Pointers that are not
+ *    device memory (host or unregistered) give GNF4_ERR_HOST_POINTER.
+ *  - Data that only the device knows (sizes, expert_ids, topk_ids) is checked
+ *    on the device. A violation sets a bit in the workspace's error word (see
+ *    GNF4_DEVERR_*) and the kernel skips the affected work; it never traps.
+ *    Read the word with gnf4_read_device_status.
+ *  - Every device-side wait is bounded; a wait that runs out sets
+ *    GNF4_DEVERR_TIMEOUT and the kernel returns.
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *
+ * Weight layout (NF4, bitsandbytes gemm_4bit conventions):
+ *    w[e][n][j]        uint8, j < K/2: element k=2j in the HIGH nibble (bits
+ *                      7..4), element k=2j+1 in the LOW nibble (bits 3..0).
+ *    absmax[e][n][b]   fp32, b < K/64: scale of elements k in [64b, 64b+64).
+ *    value(e,n,k)      = NF4[code] * absmax[e][n][k/64], NF4 = the 16-entry
+ *                        normal-float table of QLoRA/bitsandbytes.
+ */
+#ifndef GNF4_H
+#define GNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GNF4_VERSION 100 /* 1.0.0 */
+
+/* Exported entry points (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define GNF4_API __attribute__((visibility("default")))
+#else
+#define GNF4_API
+#endif
+
+/* A CUDA stream handle (identical to cudaStream_t). */
+typedef struct CUstream_st *gnf4_stream_t;
+
+typedef enum {
+    GNF4_OK = 0,
+    GNF4_ERR_INVALID_ARGUMENT = 1,    /* null pointer, bad enum, negative size */
+    GNF4_ERR_HOST_POINTER = 2,        /* a pointer is not device memory */
+    GNF4_ERR_UNSUPPORTED_SHAPE = 3,   /* K % 64, blocksize != 64, odd N with SwiGLU, limits */
+    GNF4_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < gnf4_workspace_bytes(...) */
+    GNF4_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
+    GNF4_ERR_DEVICE_METADATA = 6,     /* (read_device_status) device data was invalid */
+    GNF4_ERR_TIMEOUT = 7,             /* (read_device_status) a bounded device wait ran out */
+    GNF4_ERR_MISALIGNED = 8           /* a pointer breaks the alignment rule below */
+} gnf4_status;
+
+typedef enum { GNF4_EPI_NONE = 0, GNF4_EPI_SWIGLU = 1 } gnf4_epilogue;
+typedef enum { GNF4_MODE_AUTO = 0, GNF4_MODE_DECODE = 1, GNF4_MODE_PREFILL = 2 } gnf4_mode;
+typedef enum { GNF4_OUT_F32 = 0, GNF4_OUT_BF16 = 1 } gnf4_out_dtype;
+typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1 } gnf4_op;
+
+/* Bits of the device error word (gnf4_read_device_status). */
+#define GNF4_DEVERR_SIZES 0x1u      /* a size < 0, or sum(sizes) != M */
+#define GNF4_DEVERR_EXPERT 0x2u     /* expert_ids[g] outside [0, E) on a non-empty group */
+#define GNF4_DEVERR_TOPK 0x4u       /* a topk id outside [0, E) */
+#define GNF4_DEVERR_TIMEOUT 0x8u    /* a bounded wait ran out */
+#define GNF4_DEVERR_CAPACITY 0x10u  /* work exceeded what the workspace was sized for */
+
+/* Limits. */
+#define GNF4_MAX_EXPERTS 1024       /* E (and G) */
+#define GNF4_BLOCKSIZE 64           /* the only absmax block size */
+
+/*
+ * gnf4_moe_align -- the token->expert sort that produces (sizes, expert_ids).
+ *
+ * Passage: README opening section, "(sizes, expert_ids) supplied after the
+ * usual token->expert sort". The pages do not define the sort further; this
+ * library fixes it as a stable counting sort:
+ *   - slots are the flat indices s = t*top_k + j of topk_ids[T][top_k];
+ *   - groups are the experts that received at least one slot, in ascending
+ *     expert id; sizes[g] = slot count, expert_ids[g] = expert id, for
+ *     g < *num_groups; entries g >= *num_groups are sizes=0, expert_ids=-1;
+ *   - sorted_idx lists the slots group by group, ascending s within a group;
+ *     the caller gathers x_sorted[i] = hidden[sorted_idx[i] / top_k].
+ * Arrays sizes/expert_ids have E entries so they feed gnf4_grouped_gemm with
+ * G = E and no host synchronisation. Duplicate experts within a token count
+ * twice. A topk id outside [0, E) sets GNF4_DEVERR_TOPK; such slots are left
+ * out of every group and sorted_idx is padded with -1 at its tail.
+ *
+ *   topk_ids    device int32 [T*top_k], row-major [T][top_k] (may be NULL if T == 0)
+ *   T >= 0, 1 <= top_k, 1 <= E <= GNF4_MAX_EXPERTS, T*top_k < 2^31
+ *   sorted_idx  device int32 [T*top_k]    (written; may be NULL if T == 0)
+ *   sizes       device int32 [E]          (written)
+ *   expert_ids  device int32 [E]          (written)
+ *   num_groups  device int32 [1]          (written)
+ *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_MOE_ALIGN, ...) bytes,
+ *               zero-filled once by the caller before its first use.
+ * One kernel launch.
+ */
+GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t top_k, int32_t E,
+                           int32_t *sorted_idx, int32_t *sizes, int32_t *expert_ids,
+                           int32_t *num_groups, void *workspace, size_t ws_bytes,
+                           gnf4_stream_t stream);
+
+/*
+ * gnf4_grouped_gemm -- y = x . W^T per group, on NF4-packed W, one launch.
+ *
+ * Passage: README opening section (the whole operation, quoted in substance
+ * at the top of this file); "The claim" (fp32 accumulation, more accurate than
+ * materialising bf16 weights). Rows of x are already sorted by group: group g
+ * owns rows [sum(sizes[0..g)), sum(sizes[0..g])) and multiplies expert
+ * expert_ids[g]. For every row m of group g and column n:
+ *     acc[m][n] = sum_k x[m][k] * NF4[code(e,n,k)] * absmax[e][n][k/64]   (fp32)
+ *     epilogue NONE:   y[m][n] = bf16_rne(acc[m][n]),            y is [M][N]
+ *     epilogue SWIGLU: y[m][j] = bf16_rne(silu(acc[m][j]) * acc[m][j+N/2]),
+ *                      j < N/2, silu(g) = g/(1+exp(-g)),          y is [M][N/2]
+ * No bf16 (or other) copy of the weights is written anywhere.
+ *
+ *   x           device bf16 [M][K] (uint16 bit patterns), row stride K
+ *   w           device uint8 [E][N][K/2]
+ *   absmax      device fp32 [E][N][K/64]
+ *   sizes       device int32 [G]; sizes[g] >= 0, sum == M (checked on device)
+ *   expert_ids  device int32 [G]; in [0, E) where sizes[g] > 0, else ignored
+ *   1 <= G <= GNF4_MAX_EXPERTS; M >= 0 (M == 0: returns GNF4_OK, no launch)
+ *   N >= 1 (even for SWIGLU); K >= 64, K % 64 == 0; 1 <= E <= GNF4_MAX_EXPERTS
+ *   blocksize   must be 64
+ *   epilogue    gnf4_epilogue
+ *   mode        gnf4_mode: AUTO picks DECODE when the mean rows per possible
+ *               group, M / min(G, E), is at most 64, else PREFILL. Both
+ *               modes accept any group sizes; the mode only selects the kernel.
+ *   y           device bf16 [M][N] or [M][N/2]; fully overwritten; must not
+ *               overlap x, w, absmax or the workspace.
+ *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G)
+ *               bytes, zero-filled once by the caller before its first use;
+ *               the kernels leave its counters at zero again when they finish.
+ *               Two calls that may run concurrently need separate workspaces.
+ * Alignment: x, w, y and the workspace 32-byte aligned; absmax 4-byte aligned.
+ * On a device-side metadata error no output is written.
+ */
+GNF4_API gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *absmax,
+                              const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                              int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                              int32_t epilogue, int32_t mode, uint16_t *y, void *workspace,
+                              size_t ws_bytes, gnf4_stream_t stream);
+
+/*
+ * gnf4_dequant_debug -- materialise NF4[code] * absmax for inspection/tests.
+ *
+ * Off the hot path (the GEMM never calls it). It is this library's analogue of
+ * the package's pure-torch reference decode ("grouped-nf4-gemm" package page,
+ * "Owns": pack and pure-torch reference operations). Each element is one IEEE
+ * fp32 multiply NF4[code] * absmax; with GNF4_OUT_BF16 that product is rounded
+ * once to bf16 (round to nearest even).
+ *
+ *   w       device uint8 [rows][K/2]   (rows = E*N for a whole stack)
+ *   absmax  device fp32 [rows][K/64]
+ *   rows >= 0, K >= 64, K % 64 == 0, blocksize == 64
+ *   out     device fp32 or bf16 [rows][K]
+ * Alignment: w and out 16-byte aligned.
+ */
+GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,
+                               int32_t blocksize, int32_t out_dtype, void *out,
+                               gnf4_stream_t stream);
+
+/*
+ * gnf4_workspace_bytes -- workspace size for an op and problem size (no GPU
+ * work; queries the current device's SM count once). For GNF4_OP_MOE_ALIGN
+ * only E matters; for GNF4_OP_GROUPED_GEMM the size covers every mode.
+ */
+GNF4_API size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t E, int32_t G);
+
+/*
+ * gnf4_read_device_status -- synchronise `stream`, read the device error word
+ * from `workspace` into *error_bits (GNF4_DEVERR_* bits; may be NULL) and,
+ * if clear != 0, reset it to zero. Returns GNF4_ERR_DEVICE_METADATA if any
+ * metadata bit is set, GNF4_ERR_TIMEOUT if only the timeout bit is set,
+ * GNF4_ERR_CUDA on a CUDA failure, else GNF4_OK. Not for the hot path.
+ */
+GNF4_API gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uint32_t *error_bits,
+                                    gnf4_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+GNF4_API const char *gnf4_status_string(gnf4_status status);
+
+/* GNF4_VERSION of the loaded library. */
+GNF4_API int32_t gnf4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GNF4_H */

@@ -1,0 +1,90 @@
+"""C ABI of libgnf4 on the CPU: the library loads, exports every symbol that
+include/gnf4.h declares, and its host-side argument checks return the
+documented status codes before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import grouped_nf4_w4a16_b200 as gnf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gnf4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gnf4_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(gnf4.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = gnf4.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    raw = ctypes.CDLL(gnf4.library_path())
+    for name in declared_functions():
+        assert ctypes.cast(getattr(raw, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings():
+    assert gnf4.gnf4_version() == 100
+    assert gnf4.gnf4_status_string(0) == "GNF4_OK"
+    assert "HOST_POINTER" in gnf4.gnf4_status_string(2)
+    assert gnf4.gnf4_status_string(99) == "GNF4_ERR_UNKNOWN"
+
+
+def test_workspace_sizes_are_positive_and_monotone():
+    a = gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_MOE_ALIGN, 16, E=4)
+    assert a >= 256
+    s1 = gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_GEMM, 16, 128, 256, 4, 4)
+    s2 = gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_GEMM, 256, 5760, 2880, 128, 128)
+    assert 256 < s1 <= s2
+    assert gnf4.gnf4_workspace_bytes(7, 16, 128, 256, 4, 4) == 0
+
+
+def _gemm(lib, **kw):
+    args = dict(x=1, w=1, absmax=1, sizes=1, expert_ids=1, G=4, M=16, N=128, K=256, E=4,
+                blocksize=64, epi=0, mode=0, y=1, ws=1, ws_bytes=1 << 20, stream=None)
+    args.update(kw)
+    return lib.gnf4_grouped_gemm(args["x"], args["w"], args["absmax"], args["sizes"],
+                                 args["expert_ids"], args["G"], args["M"], args["N"], args["K"],
+                                 args["E"], args["blocksize"], args["epi"], args["mode"], args["y"],
+                                 args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), 1), (dict(y=None), 1), (dict(ws=None), 1),
+    (dict(M=-1), 1), (dict(N=0), 1), (dict(E=0), 1), (dict(G=0), 1),
+    (dict(epi=5), 1), (dict(mode=9), 1),
+    (dict(blocksize=32), 3), (dict(K=96), 3), (dict(E=2000), 3), (dict(G=2000), 3),
+    (dict(epi=1, N=127), 3),
+    (dict(M=0), 0),
+])
+def test_grouped_gemm_host_checks(kw, status):
+    assert _gemm(gnf4.load_library(), **kw) == status
+
+
+def test_moe_align_and_dequant_host_checks():
+    lib = gnf4.load_library()
+    assert lib.gnf4_moe_align(None, 8, 2, 4, 1, 1, 1, 1, 1, 256, None) == 1
+    assert lib.gnf4_moe_align(1, 8, 0, 4, 1, 1, 1, 1, 1, 256, None) == 1
+    assert lib.gnf4_moe_align(1, 8, 2, 4096, 1, 1, 1, 1, 1, 256, None) == 3
+    assert lib.gnf4_moe_align(1, 8, 2, 4, 1, 1, 1, 1, 1, 16, None) == 4
+    assert lib.gnf4_dequant_debug(None, 1, 4, 64, 64, 0, 1, None) == 1
+    assert lib.gnf4_dequant_debug(1, 1, 4, 96, 64, 0, 1, None) == 3
+    assert lib.gnf4_dequant_debug(1, 1, 4, 64, 64, 7, 1, None) == 1
+    assert lib.gnf4_dequant_debug(1, 1, 0, 64, 64, 0, 1, None) == 0
+
+
+def test_host_buffers_are_refused():
+    # Host memory is refused with GNF4_ERR_HOST_POINTER (no host path exists).
+    buf = (ctypes.c_uint8 * (1 << 16))()
+    p = ctypes.addressof(buf)
+    assert _gemm(gnf4.load_library(), x=p, w=p, absmax=p, sizes=p, expert_ids=p, y=p, ws=p) == 2
+    assert gnf4.load_library().gnf4_dequant_debug(p, p, 4, 64, 64, 0, p, None) == 2
