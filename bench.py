@@ -141,7 +141,30 @@ def _cuda_driver():
     lib = ctypes.CDLL("libcuda.so.1")
     lib.cuEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
     lib.cuEventRecordWithFlags.restype = ctypes.c_int
+    lib.cuEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p,
+                                       ctypes.c_void_p]
+    lib.cuEventElapsedTime.restype = ctypes.c_int
+    lib.cuEventCreate.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
+    lib.cuEventCreate.restype = ctypes.c_int
     return lib
+
+
+def _new_event(drv):
+    """A timing-enabled CUevent created through the driver API."""
+    ev = ctypes.c_void_p(0)
+    st = drv.cuEventCreate(ctypes.byref(ev), 0)
+    if st != 0:
+        raise RuntimeError(f"cuEventCreate failed with CUresult {st}")
+    return ev
+
+
+def _elapsed_ms(drv, a, b):
+    """Elapsed time between two events recorded by external graph nodes."""
+    out = ctypes.c_float(0.0)
+    st = drv.cuEventElapsedTime(ctypes.byref(out), a, b)
+    if st != 0:
+        raise RuntimeError(f"cuEventElapsedTime failed with CUresult {st}")
+    return float(out.value)
 
 
 # ------------------------------------------------------------------ problem
@@ -203,8 +226,10 @@ class Problem:
 
         def ev(i):
             if events is not None:
-                drv.cuEventRecordWithFlags(ctypes.c_void_p(events[i].cuda_event),
-                                           ctypes.c_void_p(stream.cuda_stream), 1)
+                # CU_EVENT_RECORD_EXTERNAL: a real timestamp node inside the graph
+                st = drv.cuEventRecordWithFlags(events[i], ctypes.c_void_p(stream.cuda_stream), 1)
+                if st != 0:
+                    raise RuntimeError(f"cuEventRecordWithFlags failed with CUresult {st}")
         ev(0)
         gnf4.gnf4_moe_align(self.topk, self.w.E, sorted_idx=self.sorted_idx, sizes=self.sizes,
                             expert_ids=self.expert_ids, num_groups=self.num_groups,
@@ -246,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
             prob.launch(r)
         torch.cuda.synchronize()
         for r in range(prob.R):
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
+            e = [_new_event(drv) for _ in range(nk + 1)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 prob.launch(r, events=e, drv=drv, stream=stream)
@@ -301,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
     per_kernel = [[] for _ in range(nk)]
     for e in evs:
         for k in range(nk):
-            per_kernel[k].append(e[k].elapsed_time(e[k + 1]))
+            per_kernel[k].append(_elapsed_ms(drv, e[k], e[k + 1]))
     kern_ms = [sum(v) / len(v) for v in per_kernel]
 
     if world > 1:

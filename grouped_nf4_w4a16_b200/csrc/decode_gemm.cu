@@ -2,65 +2,81 @@
 //
 // Passage: "grouped-nf4-gemm -- single-launch W4A16 GEMM over fused NF4 MoE
 // expert stacks", opening section (one launch for all active experts, LUT
-// decode to fp32 in registers, blockwise fp32 absmax, fp32 accumulation, bf16
+// decode of the packed codes, blockwise fp32 absmax, fp32 accumulation, bf16
 // epilogue, no bf16 weight copy) and "Status / roadmap" (split-K for starved
 // grids). At a handful of rows per expert this GEMM streams every touched
 // weight byte exactly once and is bound by HBM bandwidth.
 //
 // Work decomposition
-//   tile   = (row chunk, column tile): up to kMT activation rows of one group
+//   tile   = (row chunk, column tile): up to 8 activation rows of one group
 //            times 256 weight rows of that group's expert (with SwiGLU: 128
 //            gate rows j..j+127 and the matching 128 up rows N/2+j.., so the
-//            epilogue can pair them inside the CTA).
+//            epilogue pairs them in registers).
 //   unit   = one 64-element absmax block of K for a whole tile.
-//   Stream-K: the tiles' units are laid end to end and every CTA (one per SM)
-//   takes an equal contiguous range. A tile covered by one CTA is finished in
+//   Stream-K: the tiles' units are laid end to end and every CTA takes an
+//   equal contiguous range. A tile covered by one CTA is finished in
 //   registers; a tile split between CTAs is finished by whichever contributor
 //   arrives last (per-tile counter in the workspace), which sums the fp32
 //   partials in CTA order, so the result does not depend on arrival order.
 //   The tile list is derived on the device from (sizes, expert_ids): the
 //   host never learns which experts are active (no sync, graph-capturable).
 //
-// Inside a CTA (8 consumer warps + 1 producer warp)
-//   consumer thread t owns weight row t of the tile. It streams its row with
-//   32-byte loads straight from HBM into registers (one absmax block per
-//   load), one step ahead of use. Each byte (two codes) is decoded with ONE
-//   shared-memory load from a 256-entry table of fp32 pairs
-//   (NF4[hi], NF4[lo]), replicated per lane so the warp never hits a bank
-//   conflict; the byte-to-address step is a single byte permute. The pair
-//   multiplies the matching x pair with a packed fp32x2 FMA. After each block
-//   the fp32 partial is scaled by that block's absmax and accumulated.
-//   producer warp: converts the tile's activation rows for the next steps
-//   from bf16 to fp32 into a shared ring (mbarrier handshake); consumers read
-//   them as warp-wide broadcasts.
+// Inside a CTA (8 warps, two CTAs per SM)
+//   Warp w owns 32 of the tile's weight rows as four groups of 8 (row group
+//   rg). A step covers 2 blocks; for each block, lane (g = lane/4, q = lane%4)
+//   loads 8 packed bytes of row g of each group (one 8-byte load per row; the
+//   four lanes of a row cover its 32 bytes, so every load instruction reads
+//   whole 32-byte sectors) and the block's absmax, one step ahead of use.
+//   Decode: each byte (two codes) is ONE 8-byte shared-memory load from a
+//   256-entry table, replicated per lane so the warp never hits a bank
+//   conflict and addressed by a single byte permute. The entry holds
+//   (NF4[hi], NF4[lo]) as a bf16 pair plus the bf16 pair of their
+//   remainders, so hi + lo equals the fp32 code value to within 2^-18
+//   relative. The two 32-bit halves of the entry feed an m16n8k16 bf16
+//   tensor-core MMA directly as adjacent A-fragment registers: A rows 0-7
+//   carry the hi parts of the group's 8 weight rows and A rows 8-15 the lo
+//   parts of the same rows, so C rows g and g+8 are the hi and lo partial
+//   sums of weight row g and their sum is the exact-weight dot product. The
+//   multiply-accumulate over a block's 64 elements for all 8 activation rows
+//   is then four MMAs per 8x64 weights instead of one FMA per weight per
+//   row: the CUDA cores only decode (one permute and one shared load per two
+//   weights). The contraction index inside a block is permuted identically
+//   for weights and activations so that each lane's weight bytes are
+//   contiguous; each lane reads its bf16 activation fragment (16 contiguous
+//   values of one row) straight from global memory, where it stays cached in
+//   L1 for the whole CTA. The block's fp32 result is scaled by absmax(weight
+//   row, block) and added to an fp32 accumulator.
 #include "launch.h"
 
 namespace gnf4 {
 namespace {
 
-constexpr int kRows = 256;            // weight rows per tile = consumer threads
-constexpr int kConsumers = kRows;
-constexpr int kThreads = kConsumers + 32;
-constexpr int kMT = 8;                // activation rows per tile (row chunk)
-constexpr int kStepBlocks = 4;        // 64-element blocks per step (256 k)
-constexpr int kStepK = kStepBlocks * 64;
-constexpr int kStages = 3;            // activation ring depth
+constexpr int kThreads = 256;         // 8 warps
+constexpr int kCtasPerSm = 2;
+constexpr int kRows = 256;            // weight rows per tile: 8 warps x 2 slices x 16
+constexpr int kMT = 8;                // activation rows per tile = MMA N
+constexpr int kStepBlocks = 2;        // 64-element blocks per step
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
+constexpr int kPartialFloats = 8 * kThreads;   // 8 accumulators per thread
 
 // Dynamic shared memory layout (bytes).
-constexpr int kLutBytes = 256 * 32 * 8;                       // [byte][lane] float2
-constexpr int kXsOff = kLutBytes;
-constexpr int kXsBytes = kStages * kMT * kStepK * 4;
-constexpr int kChunkStartOff = kXsOff + kXsBytes;             // int[kMaxG + 1]
+constexpr int kLutOff = 0;                                    // uint2 [256 bytes][32 lanes]
+constexpr int kLutBytes = 256 * 32 * 8;
+constexpr int kChunkStartOff = kLutOff + kLutBytes;           // int[kMaxG + 1]
 constexpr int kRowOffOff = kChunkStartOff + (kMaxG + 4) * 4;  // int[kMaxG]
 constexpr int kGSizeOff = kRowOffOff + kMaxG * 4;             // int[kMaxG]
 constexpr int kGExpOff = kGSizeOff + kMaxG * 4;               // int[kMaxG]
-constexpr int kExOff = kGExpOff + kMaxG * 4;                  // float[kMT][128]
-constexpr int kBarOff = kExOff + kMT * 128 * 4;               // uint64[2*kStages]
-constexpr int kMiscOff = kBarOff + 2 * kStages * 8;           // int[16]
+constexpr int kMiscOff = kGExpOff + kMaxG * 4;                // int[16]
 constexpr int kSmemBytes = kMiscOff + 16 * 4;
 
-constexpr int64_t kTimeoutNs = 2000000000LL;   // 2 s per wait, then give up
+// Named barrier of the split-tile protocol (all kThreads threads take part).
+constexpr uint32_t kBarPartial = 1;
+
+// Blocks in a step: at most kStepBlocks, never past the row end or range end.
+__device__ __forceinline__ int step_blocks(int64_t left_in_row, int64_t left_in_range) {
+  const int64_t n = left_in_row < left_in_range ? left_in_row : left_in_range;
+  return static_cast<int>(n < kStepBlocks ? n : kStepBlocks);
+}
 
 struct Sched {
   int32_t G, N, K, E, swiglu;
@@ -70,150 +86,159 @@ struct Sched {
   int64_t lo, hi;    // this CTA's unit range
 };
 
-struct Tile {
+// Tile-level facts (identical in every thread).
+struct TileGroup {
   int64_t row0;      // first activation row
   int32_t mrows;     // activation rows (1..kMT)
   int32_t j;         // column tile
-  int64_t wrow;      // this thread's global weight row (e*N + n)
-  int32_t col;       // output column of this thread (or -1 if not an output column)
-  bool valid;        // this thread's weight row exists
+  int32_t e;         // expert
 };
 
-// Blocks in a step: at most kStepBlocks, never past the row end or range end.
-__device__ __forceinline__ int step_blocks(int64_t left_in_row, int64_t left_in_range) {
-  int64_t n = left_in_row < left_in_range ? left_in_row : left_in_range;
-  return static_cast<int>(n < kStepBlocks ? n : kStepBlocks);
-}
+// This thread's view of a tile: weight row wrow0 + RowOffsets::dr[rg] for
+// row group rg (row g of the group), its activation row (row0 + g, or -1 if
+// the tile has no row g), and which row groups exist.
+struct ThreadTile {
+  int64_t wrow0;
+  int64_t xrow;
+  int32_t col0;       // output column of row group 0
+  uint32_t vmask;     // bit rg: that weight row exists
+};
 
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
+// Row offsets of the four row groups from row group 0 (uniform per launch).
+struct RowOffsets {
+  int32_t dr[4];      // weight rows
+  int32_t dc[4];      // output columns (-1: not an output row)
+};
 
-// Bounded wait; after the first timeout in this CTA every later wait gives
-// up at once, so a broken pipeline ends quickly instead of hanging.
-__device__ __forceinline__ void wait_or_flag(uint64_t *bar, uint32_t parity, int *timed_out,
-                                             WsHeader *hdr) {
-  if (mbar_try_wait(bar, parity)) return;
-  if (*reinterpret_cast<volatile int *>(timed_out)) return;
-  const uint64_t t0 = global_timer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return;
-    if (global_timer() - t0 > static_cast<uint64_t>(kTimeoutNs)) {
-      *reinterpret_cast<volatile int *>(timed_out) = 1;
-      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
-      return;
+__device__ __forceinline__ RowOffsets make_offsets(int32_t N, int32_t swiglu) {
+  RowOffsets o;
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg) {
+    if (swiglu) {   // rg 0,1: gate rows; rg 2,3: the up rows of the same columns
+      o.dr[rg] = 8 * (rg & 1) + (rg < 2 ? 0 : N / 2);
+      o.dc[rg] = rg < 2 ? 8 * rg : -1;
+    } else {
+      o.dr[rg] = 8 * rg;
+      o.dc[rg] = 8 * rg;
     }
   }
+  return o;
 }
 
-__device__ __forceinline__ Tile tile_info(int64_t T, const Sched &s, const int *chunk_start,
-                                          const int *row_off, const int *gsize, const int *gexp,
-                                          int t) {
-  Tile ti;
+__device__ __forceinline__ TileGroup tile_group(int64_t T, const Sched &s, const int *chunk_start,
+                                                const int *row_off, const int *gsize,
+                                                const int *gexp) {
+  TileGroup tg;
   const int64_t c = T / s.NT;
-  ti.j = static_cast<int32_t>(T - c * s.NT);
-  // group g with chunk_start[g] <= c < chunk_start[g+1]
+  tg.j = static_cast<int32_t>(T - c * s.NT);
   int lo = 0, hi = s.G;   // invariant: chunk_start[lo] <= c < chunk_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (chunk_start[mid] <= c) lo = mid; else hi = mid;
   }
-  const int g = lo;
-  const int32_t local = static_cast<int32_t>(c - chunk_start[g]);
-  ti.row0 = static_cast<int64_t>(row_off[g]) + static_cast<int64_t>(local) * kMT;
-  ti.mrows = min(kMT, gsize[g] - local * kMT);
-  const int e = gexp[g];
-  int n;
+  const int32_t local = static_cast<int32_t>(c - chunk_start[lo]);
+  tg.row0 = static_cast<int64_t>(row_off[lo]) + static_cast<int64_t>(local) * kMT;
+  tg.mrows = min(kMT, gsize[lo] - local * kMT);
+  tg.e = gexp[lo];
+  return tg;
+}
+
+__device__ __forceinline__ ThreadTile thread_tile(const TileGroup &tg, const Sched &s, int warp,
+                                                  int g) {
+  ThreadTile r;
+  const int n0 = s.swiglu ? tg.j * 128 + warp * 16 + g : tg.j * kRows + warp * 32 + g;
+  const int lim = s.swiglu ? s.N / 2 : s.N;   // columns at or past lim are padding
+  uint32_t m;
   if (s.swiglu) {
-    const int h = s.N / 2;
-    const int jj = ti.j * 128 + (t & 127);
-    ti.valid = jj < h;
-    n = (t < 128) ? jj : h + jj;
-    ti.col = (t < 128 && ti.valid) ? jj : -1;
+    m = (n0 < lim ? 5u : 0u) | (n0 + 8 < lim ? 10u : 0u);   // rg 0/2 share n0, rg 1/3 n0+8
   } else {
-    n = ti.j * kRows + t;
-    ti.valid = n < s.N;
-    ti.col = ti.valid ? n : -1;
+    m = (n0 < lim ? 1u : 0u) | (n0 + 8 < lim ? 2u : 0u) | (n0 + 16 < lim ? 4u : 0u) |
+        (n0 + 24 < lim ? 8u : 0u);
   }
-  ti.wrow = static_cast<int64_t>(e) * s.N + (ti.valid ? n : 0);
-  return ti;
+  r.vmask = m;
+  r.col0 = n0;
+  r.wrow0 = static_cast<int64_t>(tg.e) * s.N + n0;
+  r.xrow = g < tg.mrows ? tg.row0 + g : -1;
+  return r;
 }
 
-// Load this thread's weight bytes and scales for blocks [kb0, kb0+nblk).
-__device__ __forceinline__ void load_step(const uint8_t *__restrict__ w,
-                                          const float *__restrict__ absmax, const Tile &ti,
-                                          const Sched &s, int kb0, int nblk,
-                                          uint32_t (&wq)[kStepBlocks][8], float (&aq)[kStepBlocks]) {
-  const uint8_t *wr = w + ti.wrow * static_cast<int64_t>(s.K / 2);
-  const float *ar = absmax + ti.wrow * static_cast<int64_t>(s.KB);
+// 8 packed bytes (16 codes) of a row; streamed, no L1 allocation.
+__device__ __forceinline__ uint2 ldg64_stream(const void *p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+struct StepW {
+  uint2 w[kStepBlocks][4];    // [block][row group]: this lane's 8 bytes
+  float a[kStepBlocks][4];    // [block][row group]: absmax
+};
+
+__device__ __forceinline__ void load_step(const ThreadTile &tt, const RowOffsets &ro,
+                                          const uint8_t *__restrict__ w,
+                                          const float *__restrict__ absmax, int64_t row_bytes,
+                                          int KB, int kb0, int nblk, int q, StepW &d) {
 #pragma unroll
-  for (int b = 0; b < kStepBlocks; ++b) {
-    if (ti.valid && b < nblk) {
-      ldg256_stream(wr + static_cast<int64_t>(kb0 + b) * 32, wq[b]);
-      aq[b] = __ldg(ar + kb0 + b);
-    } else {
+  for (int rg = 0; rg < 4; ++rg) {
+    const int64_t row = tt.wrow0 + ro.dr[rg];
+    const bool ok = (tt.vmask >> rg) & 1u;
+    const uint8_t *wp = w + row * row_bytes + kb0 * 32 + 8 * q;
+    const float *ap = absmax + row * KB + kb0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) wq[b][i] = 0x77777777u;   // codes 7 = 0.0
-      aq[b] = 0.0f;
+    for (int b = 0; b < kStepBlocks; ++b) {
+      const bool on = ok && b < nblk;
+      d.w[b][rg] = on ? ldg64_stream(wp + b * 32) : make_uint2(0x77777777u, 0x77777777u);
+      d.a[b][rg] = on ? __ldg(ap + b) : 0.0f;
     }
   }
 }
 
-// acc[m] += sum over the step's blocks of absmax_b * sum_k x[m,k] * NF4[code_k]
-template <int MR>
-__device__ __forceinline__ void compute_step(const uint32_t (&wq)[kStepBlocks][8],
-                                             const float (&aq)[kStepBlocks], int nblk,
-                                             const float *__restrict__ xs, const char *lut,
-                                             uint32_t lane8, float (&acc)[kMT]) {
-#pragma unroll
-  for (int b = 0; b < kStepBlocks; ++b) {
-    if (b < nblk) {
-      float2 part[MR];
-#pragma unroll
-      for (int m = 0; m < MR; ++m) part[m] = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t word = wq[b][q];
-        float2 wv[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          // byte p of the word -> (byte << 8) | lane*8 : offset of this lane's copy
-          const uint32_t off = __byte_perm(word, lane8, 0x5504u | (p << 4));
-          wv[p] = *reinterpret_cast<const float2 *>(lut + off);
-        }
-#pragma unroll
-        for (int m = 0; m < MR; ++m) {
-          const float4 *xp = reinterpret_cast<const float4 *>(xs + m * kStepK + b * 64 + q * 8);
-          const float4 xa = xp[0], xb = xp[1];
-          part[m] = __ffma2_rn(wv[0], make_float2(xa.x, xa.y), part[m]);
-          part[m] = __ffma2_rn(wv[1], make_float2(xa.z, xa.w), part[m]);
-          part[m] = __ffma2_rn(wv[2], make_float2(xb.x, xb.y), part[m]);
-          part[m] = __ffma2_rn(wv[3], make_float2(xb.z, xb.w), part[m]);
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < MR; ++m) acc[m] = fmaf(aq[b], part[m].x + part[m].y, acc[m]);
-    }
-  }
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void compute_dispatch(int mrows, const uint32_t (&wq)[kStepBlocks][8],
-                                                 const float (&aq)[kStepBlocks], int nblk,
-                                                 const float *xs, const char *lut, uint32_t lane8,
-                                                 float (&acc)[kMT]) {
-  switch (mrows) {
-    case 1: compute_step<1>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 2: compute_step<2>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 3: compute_step<3>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 4: compute_step<4>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 5: compute_step<5>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 6: compute_step<6>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    case 7: compute_step<7>(wq, aq, nblk, xs, lut, lane8, acc); break;
-    default: compute_step<8>(wq, aq, nblk, xs, lut, lane8, acc); break;
+// (hi pair, lo pair) of byte p of `word`, from this lane's table slot.
+__device__ __forceinline__ uint2 lut_pair(const char *lut, uint32_t word, uint32_t lane8,
+                                          uint32_t p) {
+  const uint32_t off = __byte_perm(word, lane8, 0x5504u | (p << 4));   // byte*256 + lane*8
+  return *reinterpret_cast<const uint2 *>(lut + off);
+}
+
+// acc[rg][i] += absmax * (64-element block dot product) for activation row 2q+i.
+// b: block within the step.
+__device__ __forceinline__ void compute_block(const StepW &d, int b, const ThreadTile &tt,
+                                              const uint16_t *__restrict__ x, int64_t K, int kb,
+                                              int q, int lane, const char *lut, uint32_t lane8,
+                                              float (&acc)[4][2]) {
+  // activation fragment: 16 bf16 of row g at k = 16q..16q+15 of this block
+  uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
+  if (tt.xrow >= 0) {
+    const uint4 *xp = reinterpret_cast<const uint4 *>(x + tt.xrow * K + kb * 64 + 16 * q);
+    xa = __ldg(xp);
+    xb = __ldg(xp + 1);
+  }
+  const uint32_t xr[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg) {
+    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      const uint32_t word = st < 2 ? d.w[b][rg].x : d.w[b][rg].y;
+      const uint32_t p = (st & 1) * 2;
+      const uint2 e0 = lut_pair(lut, word, lane8, p);       // k = 16q+4st+{0,1}
+      const uint2 e1 = lut_pair(lut, word, lane8, p + 1);   // k = 16q+4st+{2,3}
+      mma_bf16(c, e0.x, e0.y, e1.x, e1.y, xr[2 * st], xr[2 * st + 1]);
+    }
+    const float a = d.a[b][rg];
+    acc[rg][0] = fmaf(c[0] + c[2], a, acc[rg][0]);
+    acc[rg][1] = fmaf(c[1] + c[3], a, acc[rg][1]);
   }
 }
 
@@ -227,39 +252,41 @@ __device__ __forceinline__ int64_t cta_of(int64_t units, int64_t u, int64_t P) {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
-// Epilogue for finished accumulators (one activation row set of the tile).
-__device__ __forceinline__ void write_tile(const float (&v)[kMT], const Tile &ti, const Sched &s,
-                                           uint16_t *__restrict__ y, float *ex, int t) {
-  if (!s.swiglu) {
-    if (ti.col >= 0) {
+__device__ __forceinline__ void store_bf16(uint16_t *p, float v) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  *p = *reinterpret_cast<const uint16_t *>(&b);
+}
+
+// Epilogue: acc[rg][i] is weight row group rg, activation row 2q + i.
+__device__ __forceinline__ void write_tile(const float (&v)[4][2], const TileGroup &tg,
+                                           const ThreadTile &tt, const RowOffsets &ro,
+                                           const Sched &s, uint16_t *__restrict__ y, int q) {
 #pragma unroll
-      for (int m = 0; m < kMT; ++m)
-        if (m < ti.mrows) {
-          const __nv_bfloat16 b = __float2bfloat16_rn(v[m]);
-          y[(ti.row0 + m) * s.N + ti.col] = *reinterpret_cast<const uint16_t *>(&b);
-        }
-    }
-  } else {
-    if (t >= 128) {
+  for (int i = 0; i < 2; ++i) {
+    const int m = 2 * q + i;
+    if (m >= tg.mrows) continue;
+    if (!s.swiglu) {
 #pragma unroll
-      for (int m = 0; m < kMT; ++m) ex[m * 128 + (t - 128)] = v[m];
-    }
-    named_barrier(2, kConsumers);
-    if (ti.col >= 0) {
-      const int h = s.N / 2;
+      for (int rg = 0; rg < 4; ++rg)
+        if ((tt.vmask >> rg) & 1u)
+          store_bf16(y + (tg.row0 + m) * s.N + tt.col0 + ro.dc[rg], v[rg][i]);
+    } else {
 #pragma unroll
-      for (int m = 0; m < kMT; ++m)
-        if (m < ti.mrows) {
-          const float r = silu(v[m]) * ex[m * 128 + t];
-          const __nv_bfloat16 b = __float2bfloat16_rn(r);
-          y[(ti.row0 + m) * h + ti.col] = *reinterpret_cast<const uint16_t *>(&b);
-        }
+      for (int rg = 0; rg < 2; ++rg)
+        if ((tt.vmask >> rg) & 1u)
+          store_bf16(y + (tg.row0 + m) * (s.N / 2) + tt.col0 + ro.dc[rg],
+                     silu(v[rg][i]) * v[rg + 2][i]);
     }
-    named_barrier(2, kConsumers);
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// bf16 (hi, lo) split of an fp32 value: hi = RNE(v), lo = RNE(v - hi).
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+  hi = __float2bfloat16_rn(v);
+  lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_gemm_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ w,
                        const float *__restrict__ absmax, const int32_t *__restrict__ sizes,
                        const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
@@ -267,51 +294,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                        WsHeader *hdr, int32_t *__restrict__ tile_cnt, int64_t tile_cap,
                        float *__restrict__ partials) {
   extern __shared__ __align__(1024) char smem[];
-  float *xs = reinterpret_cast<float *>(smem + kXsOff);
   int *chunk_start = reinterpret_cast<int *>(smem + kChunkStartOff);
   int *row_off = reinterpret_cast<int *>(smem + kRowOffOff);
   int *gsize = reinterpret_cast<int *>(smem + kGSizeOff);
   int *gexp = reinterpret_cast<int *>(smem + kGExpOff);
-  float *ex = reinterpret_cast<float *>(smem + kExOff);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + kBarOff);
-  uint64_t *empty_bar = full_bar + kStages;
-  int *misc = reinterpret_cast<int *>(smem + kMiscOff);
-  // misc[0]: error bits, misc[1]: timed out, misc[2]: last-arriver flag,
-  // misc[3]: warp sums scratch base not used, misc[4..]: scan scratch
+  int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [2] last-arriver flag
 
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+  const int g = lane >> 2, q = lane & 3;
 
-  // ---- 1. decode table: entry (byte b, lane l) = (NF4[b >> 4], NF4[b & 15])
-  for (int i = tid; i < 256 * 32; i += kThreads) {
+  // ---- 1. decode table: entry byte b, lane slot l = {bf16x2 hi, bf16x2 lo}
+  //      of the pair (NF4[b >> 4], NF4[b & 15]) (low half = even k = high nibble).
+  for (int i = t; i < 256 * 32; i += kThreads) {
     const int b = i >> 5;
-    reinterpret_cast<float2 *>(smem)[i] = make_float2(nf4_value(b >> 4), nf4_value(b & 15));
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(nf4_value(b >> 4), h0, l0);
+    split_bf16(nf4_value(b & 15), h1, l1);
+    __nv_bfloat162 hp, lp;
+    hp.x = h0; hp.y = h1;
+    lp.x = l0; lp.y = l1;
+    uint2 e;
+    e.x = *reinterpret_cast<const uint32_t *>(&hp);
+    e.y = *reinterpret_cast<const uint32_t *>(&lp);
+    reinterpret_cast<uint2 *>(smem + kLutOff)[i] = e;
   }
-  if (tid == 0) {
-    misc[0] = 0;
-    misc[1] = 0;
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full_bar[i], 32);
-      mbar_init(&empty_bar[i], kConsumers / 32);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
+  if (t == 0) misc[0] = 0;
   __syncthreads();
 
-  // ---- 2. group table from (sizes, expert_ids), validated on the device
-  // Each thread takes a contiguous run of groups; two-level exclusive scan of
-  // the row counts and the row-chunk counts.
+  // ---- 2. group table from (sizes, expert_ids), validated on the device.
   __shared__ int s_wsum[2][kThreads / 32];
   const int per = (G + kThreads - 1) / kThreads;
-  const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
+  const int g0 = min(G, t * per), g1 = min(G, g0 + per);
   int my_rows = 0, my_chunks = 0, bad = 0;
-  for (int g = g0; g < g1; ++g) {
-    const int sz = sizes[g];
-    const int e = expert_ids[g];
+  for (int gi = g0; gi < g1; ++gi) {
+    const int sz = sizes[gi];
+    const int e = expert_ids[gi];
     if (sz < 0) bad |= GNF4_DEVERR_SIZES;
     if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
-    gsize[g] = sz;
-    gexp[g] = e;
+    gsize[gi] = sz;
+    gexp[gi] = e;
     my_rows += max(sz, 0);
     my_chunks += sz > 0 ? (sz + kMT - 1) / kMT : 0;
   }
@@ -333,16 +355,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   {
     int r = wr + vr - my_rows, c = wc + vc - my_chunks;
-    for (int g = g0; g < g1; ++g) {
-      row_off[g] = r;
-      chunk_start[g] = c;
-      const int sz = max(gsize[g], 0);
+    for (int gi = g0; gi < g1; ++gi) {
+      row_off[gi] = r;
+      chunk_start[gi] = c;
+      const int sz = max(gsize[gi], 0);
       r += sz;
       c += sz > 0 ? (sz + kMT - 1) / kMT : 0;
     }
-    if (tid == 0) chunk_start[G] = tot_c;
+    if (t == 0) chunk_start[G] = tot_c;
   }
-  if (tid == 0 && static_cast<int64_t>(tot_r) != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
+  if (t == 0 && static_cast<int64_t>(tot_r) != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
   __syncthreads();
 
   Sched s;
@@ -353,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int errbits = misc[0];
   if (errbits == 0 && tiles > tile_cap) errbits = GNF4_DEVERR_CAPACITY;
   if (errbits) {
-    if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
+    if (blockIdx.x == 0 && t == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
     return;
   }
   s.units = tiles * s.KB;
@@ -362,132 +384,100 @@ __global__ void __launch_bounds__(kThreads, 1)
   s.hi = cta_lo(s.units, blockIdx.x + 1, P);
   if (s.lo >= s.hi) return;
 
-  int *timed_out = &misc[1];
-
-  if (warp == kConsumers / 32) {
-    // ---------------------------------------------------------- producer
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t curT = -1;
-    Tile ti{};
-    for (int64_t u = s.lo; u < s.hi;) {
-      const int64_t T = u / s.KB;
-      const int kb0 = static_cast<int>(u - T * s.KB);
-      const int nblk = static_cast<int>(step_blocks(s.KB - kb0, s.hi - u));
-      if (T != curT) { ti = tile_info(T, s, chunk_start, row_off, gsize, gexp, 0); curT = T; }
-      wait_or_flag(&empty_bar[stage], phase ^ 1u, timed_out, hdr);
-      float *dst = xs + stage * kMT * kStepK;
-      const int k = kb0 * 64 + lane * 8;
-      const bool in = lane * 8 < nblk * 64;
-      for (int m = 0; m < ti.mrows; ++m) {
-        float4 lo4 = make_float4(0.f, 0.f, 0.f, 0.f), hi4 = lo4;
-        if (in) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(x + (ti.row0 + m) * K + k);
-          lo4 = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
-                            __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
-          hi4 = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
-                            __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
-        }
-        float4 *d = reinterpret_cast<float4 *>(dst + m * kStepK + lane * 8);
-        d[0] = lo4;
-        d[1] = hi4;
-      }
-      mbar_arrive(&full_bar[stage]);
-      if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      u += nblk;
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int t = tid;
   const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
-  const char *lut = smem;
-  float acc[kMT];
+  const char *lut = smem + kLutOff;
+  const RowOffsets ro = make_offsets(N, swiglu);
+  const int64_t row_bytes = K / 2;
+
+  float acc[4][2];
 #pragma unroll
-  for (int m = 0; m < kMT; ++m) acc[m] = 0.0f;
+  for (int rg = 0; rg < 4; ++rg) acc[rg][0] = acc[rg][1] = 0.0f;
 
-  int stage = 0;
-  uint32_t phase = 0;
+  // ---- 4. main loop: steps of up to kStepBlocks blocks, never crossing a tile
+  int64_t T = s.lo / s.KB;
+  int kb0 = static_cast<int>(s.lo - T * s.KB);
   int64_t u = s.lo;
-  int64_t T = u / s.KB;
-  int kb0 = static_cast<int>(u - T * s.KB);
-  int nblk = static_cast<int>(step_blocks(s.KB - kb0, s.hi - u));
-  Tile ti = tile_info(T, s, chunk_start, row_off, gsize, gexp, t);
-  uint32_t wq[kStepBlocks][8];
-  float aq[kStepBlocks];
-  load_step(w, absmax, ti, s, kb0, nblk, wq, aq);
+  TileGroup tg = tile_group(T, s, chunk_start, row_off, gsize, gexp);
+  ThreadTile tt = thread_tile(tg, s, warp, g);
+  int nblk = step_blocks(s.KB - kb0, s.hi - u);
+  StepW cur;
+  load_step(tt, ro, w, absmax, row_bytes, s.KB, kb0, nblk, q, cur);
 
-  while (u < s.hi) {
+  while (true) {
     // issue the next step's loads before consuming this one
     const int64_t un = u + nblk;
     const bool has_next = un < s.hi;
+    const bool tile_end = (kb0 + nblk == s.KB) || !has_next;
     int64_t Tn = T;
-    int kbn = 0, nbn = 0;
-    Tile tn = ti;
-    uint32_t wn[kStepBlocks][8];
-    float an[kStepBlocks];
+    int kbn = kb0 + nblk;
+    TileGroup tgn = tg;
+    ThreadTile ttn = tt;
+    int nbn = 0;
+    StepW nxt;
     if (has_next) {
-      Tn = un / s.KB;
-      kbn = static_cast<int>(un - Tn * s.KB);
-      nbn = static_cast<int>(step_blocks(s.KB - kbn, s.hi - un));
-      if (Tn != T) tn = tile_info(Tn, s, chunk_start, row_off, gsize, gexp, t);
-      load_step(w, absmax, tn, s, kbn, nbn, wn, an);
+      if (kbn == s.KB) {
+        kbn = 0;
+        Tn = T + 1;
+        tgn = tile_group(Tn, s, chunk_start, row_off, gsize, gexp);
+        ttn = thread_tile(tgn, s, warp, g);
+      }
+      nbn = step_blocks(s.KB - kbn, s.hi - un);
+      load_step(ttn, ro, w, absmax, row_bytes, s.KB, kbn, nbn, q, nxt);
     }
 
-    wait_or_flag(&full_bar[stage], phase, timed_out, hdr);
-    compute_dispatch(ti.mrows, wq, aq, nblk, xs + stage * kMT * kStepK, lut, lane8, acc);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[stage]);
-    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+#pragma unroll
+    for (int b = 0; b < kStepBlocks; ++b)
+      if (b < nblk) compute_block(cur, b, tt, x, s.K, kb0 + b, q, lane, lut, lane8, acc);
 
-    const bool tile_end = (un == (T + 1) * s.KB) || !has_next;
     if (tile_end) {
       const bool whole = (T * s.KB >= s.lo) && ((T + 1) * s.KB <= s.hi);
       if (whole) {
-        write_tile(acc, ti, s, y, ex, t);
+        write_tile(acc, tg, tt, ro, s, y, q);
       } else {
         // split tile: publish the partial, the last contributor finishes it
-        const int64_t P2 = P;
         const int slot = (T == s.lo / s.KB) ? 0 : 1;
-        float *mine = partials + (static_cast<int64_t>(blockIdx.x) * 2 + slot) * (kMT * kRows);
+        float *mine = partials + (static_cast<int64_t>(blockIdx.x) * 2 + slot) * kPartialFloats;
 #pragma unroll
-        for (int m = 0; m < kMT; ++m) mine[m * kRows + t] = acc[m];
+        for (int rg = 0; rg < 4; ++rg)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) mine[(rg * 2 + i) * kThreads + t] = acc[rg][i];
         __threadfence();
-        named_barrier(1, kConsumers);
+        named_barrier(kBarPartial, kThreads);
         if (t == 0) {
           // contributors: the CTAs with a non-empty range inside [c0, c1]
-          const int64_t c0 = cta_of(s.units, T * s.KB, P2);
-          const int64_t c1 = cta_of(s.units, (T + 1) * s.KB - 1, P2);
+          const int64_t c0 = cta_of(s.units, T * s.KB, P);
+          const int64_t c1 = cta_of(s.units, (T + 1) * s.KB - 1, P);
           int ncontrib = 0;
           for (int64_t c = c0; c <= c1; ++c)
-            ncontrib += cta_lo(s.units, c, P2) < cta_lo(s.units, c + 1, P2) ? 1 : 0;
+            ncontrib += cta_lo(s.units, c, P) < cta_lo(s.units, c + 1, P) ? 1 : 0;
           const int old = atomicAdd(&tile_cnt[T], 1);
           misc[2] = (old == ncontrib - 1) ? 1 : 0;
         }
-        named_barrier(1, kConsumers);
+        named_barrier(kBarPartial, kThreads);
         if (misc[2]) {
           __threadfence();
-          const int64_t c0 = cta_of(s.units, T * s.KB, P2);
-          const int64_t c1 = cta_of(s.units, (T + 1) * s.KB - 1, P2);
-          float sum[kMT];
+          const int64_t c0 = cta_of(s.units, T * s.KB, P);
+          const int64_t c1 = cta_of(s.units, (T + 1) * s.KB - 1, P);
+          float sum[4][2];
 #pragma unroll
-          for (int m = 0; m < kMT; ++m) sum[m] = 0.0f;
+          for (int rg = 0; rg < 4; ++rg) sum[rg][0] = sum[rg][1] = 0.0f;
           for (int64_t c = c0; c <= c1; ++c) {
-            const int64_t lo_c = cta_lo(s.units, c, P2);
-            if (lo_c >= cta_lo(s.units, c + 1, P2)) continue;   // empty range: no partial
-            const int sl = (T == lo_c / s.KB) ? 0 : 1;
-            const float *src = partials + (c * 2 + sl) * (kMT * kRows);
+            const int64_t lo_c = cta_lo(s.units, c, P);
+            if (lo_c >= cta_lo(s.units, c + 1, P)) continue;   // empty range: no partial
+            const int sl_c = (T == lo_c / s.KB) ? 0 : 1;
+            const float *src = partials + (c * 2 + sl_c) * kPartialFloats;
 #pragma unroll
-            for (int m = 0; m < kMT; ++m) sum[m] += __ldcg(src + m * kRows + t);
+            for (int rg = 0; rg < 4; ++rg)
+#pragma unroll
+              for (int i = 0; i < 2; ++i) sum[rg][i] += __ldcg(src + (rg * 2 + i) * kThreads + t);
           }
-          write_tile(sum, ti, s, y, ex, t);
+          write_tile(sum, tg, tt, ro, s, y, q);
           if (t == 0) tile_cnt[T] = 0;
         }
-        named_barrier(1, kConsumers);   // misc[2] is reused by the next split tile
+        named_barrier(kBarPartial, kThreads);   // misc[2] is reused by the next split tile
       }
 #pragma unroll
-      for (int m = 0; m < kMT; ++m) acc[m] = 0.0f;
+      for (int rg = 0; rg < 4; ++rg) acc[rg][0] = acc[rg][1] = 0.0f;
     }
 
     if (!has_next) break;
@@ -495,32 +485,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     T = Tn;
     kb0 = kbn;
     nblk = nbn;
-    ti = tn;
-#pragma unroll
-    for (int b = 0; b < kStepBlocks; ++b) {
-      aq[b] = an[b];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) wq[b][i] = wn[b][i];
-    }
+    tg = tgn;
+    tt = ttn;
+    cur = nxt;
   }
+}
+
+int decode_grid() { return device_sm_count() * kCtasPerSm; }
+
+int64_t decode_tile_cap(int64_t M, int32_t N, int32_t G, int32_t swiglu) {
+  const int64_t nt = swiglu ? (N / 2 + 127) / 128 : (N + kRows - 1) / kRows;
+  const int64_t groups = G < M ? G : M;
+  return (M / kMT + groups) * nt;
 }
 
 }  // namespace
 
 size_t decode_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu) {
   (void)K;
-  const int64_t nt = swiglu ? (N / 2 + 127) / 128 : (N + kRows - 1) / kRows;
-  const int64_t groups = G < M ? G : M;
-  const int64_t tile_cap = (M / kMT + groups) * nt;
+  const int64_t tile_cap = decode_tile_cap(M, N, G, swiglu);
   const size_t cnt_bytes = ((static_cast<size_t>(tile_cap) * 4 + 255) / 256) * 256;
-  const size_t part_bytes = static_cast<size_t>(device_sm_count()) * 2 * kMT * kRows * 4;
+  const size_t part_bytes = static_cast<size_t>(decode_grid()) * 2 * kPartialFloats * 4;
   return kWsHeaderBytes + cnt_bytes + part_bytes;
 }
 
 cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
-  const int64_t nt = a.swiglu ? (a.N / 2 + 127) / 128 : (a.N + kRows - 1) / kRows;
-  const int64_t groups = a.G < a.M ? a.G : a.M;
-  const int64_t tile_cap = (a.M / kMT + groups) * nt;
+  const int64_t tile_cap = decode_tile_cap(a.M, a.N, a.G, a.swiglu);
   const size_t cnt_bytes = ((static_cast<size_t>(tile_cap) * 4 + 255) / 256) * 256;
   char *ws = static_cast<char *>(a.workspace);
   WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
@@ -530,14 +520,13 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
     cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    configured[dev] = true;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  const int grid = device_sm_count();
-  decode_gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+  decode_gemm_kernel<<<decode_grid(), kThreads, kSmemBytes, stream>>>(
       a.x, a.w, a.absmax, a.sizes, a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.swiglu, a.y, hdr, cnt,
       tile_cap, partials);
   return cudaGetLastError();

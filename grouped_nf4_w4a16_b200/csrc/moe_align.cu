@@ -5,7 +5,8 @@
 // usual token->expert sort. The sort fixed here (gnf4.h documents it):
 // groups = non-empty experts in ascending id, slots ascending within a group.
 //
-// Design: a single 1024-thread CTA, everything in shared memory, one launch.
+// Design: a single CTA (8 warps up to 4096 slots, else 32), everything in
+// shared memory, one launch.
 //   1. each warp owns a contiguous segment of the S = T*top_k slots and builds
 //      its own per-expert histogram (shared-memory atomics);
 //   2. per expert, an exclusive scan over the 32 warp histograms gives each
@@ -22,26 +23,26 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kAlignThreads = 1024;
-constexpr int kAlignWarps = kAlignThreads / 32;
-
-__global__ void __launch_bounds__(kAlignThreads, 1)
+// NW warps; each warp owns a contiguous segment of the slots.
+template <int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
     moe_align_kernel(const int32_t *__restrict__ topk, int32_t S, int32_t E,
                      int32_t *__restrict__ sorted_idx, int32_t *__restrict__ sizes,
                      int32_t *__restrict__ expert_ids, int32_t *__restrict__ num_groups,
                      WsHeader *hdr) {
+  constexpr int NT = NW * 32;
   extern __shared__ int32_t sm[];
-  int32_t *hist = sm;                        // [kAlignWarps][E]
-  int32_t *start = hist + kAlignWarps * E;   // [E] first output position of each expert
-  __shared__ int32_t warp_sum_v[kAlignWarps];
-  __shared__ int32_t warp_sum_f[kAlignWarps];
+  int32_t *hist = sm;                 // [NW][E]
+  int32_t *start = hist + NW * E;     // [E] first output position of each expert
+  __shared__ int32_t warp_sum_v[NW];
+  __shared__ int32_t warp_sum_f[NW];
   __shared__ int32_t s_valid, s_groups;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) hist[i] = 0;
+  for (int i = tid; i < NW * E; i += NT) hist[i] = 0;
   __syncthreads();
 
-  const int seg = (S + kAlignWarps - 1) / kAlignWarps;
+  const int seg = (S + NW - 1) / NW;
   const int beg = min(S, warp * seg), end = min(S, beg + seg);
 
   // 1. per-warp histograms
@@ -55,19 +56,25 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   }
   __syncthreads();
 
-  // 2. per expert: exclusive scan over warps (E <= 1024: one expert per thread)
-  int tot = 0;
-  if (tid < E) {
-    for (int w = 0; w < kAlignWarps; ++w) {
-      const int c = hist[w * E + tid];
-      hist[w * E + tid] = tot;
+  // 2. per expert: exclusive scan over the warps' histograms. Thread tid owns
+  //    the contiguous experts [e0, e1); its local sums feed the block scan.
+  const int per = (E + NT - 1) / NT;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int my_v = 0, my_f = 0;
+  for (int e = e0; e < e1; ++e) {
+    int tot = 0;
+    for (int w = 0; w < NW; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = tot;
       tot += c;
     }
+    start[e] = tot;            // count for now; turned into a position below
+    my_v += tot;
+    my_f += tot > 0 ? 1 : 0;
   }
-  const int flag = (tid < E && tot > 0) ? 1 : 0;
 
-  // 3. block exclusive scans over experts of counts (v) and non-empty flags (f)
-  int v = tot, f = flag;
+  // 3. block exclusive scans of counts (v) and non-empty flags (f) over experts
+  int v = my_v, f = my_f;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int a = __shfl_up_sync(0xffffffffu, v, o);
@@ -77,7 +84,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   if (lane == 31) { warp_sum_v[warp] = v; warp_sum_f[warp] = f; }
   __syncthreads();
   if (warp == 0) {
-    const int a0 = warp_sum_v[lane], b0 = warp_sum_f[lane];
+    const int a0 = lane < NW ? warp_sum_v[lane] : 0, b0 = lane < NW ? warp_sum_f[lane] : 0;
     int a = a0, b = b0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -85,20 +92,23 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
       const int ub = __shfl_up_sync(0xffffffffu, b, o);
       if (lane >= o) { a += ua; b += ub; }
     }
-    warp_sum_v[lane] = a - a0;
-    warp_sum_f[lane] = b - b0;
+    if (lane < NW) { warp_sum_v[lane] = a - a0; warp_sum_f[lane] = b - b0; }
     if (lane == 31) { s_valid = a; s_groups = b; }
   }
   __syncthreads();
-  const int excl_v = v - tot + warp_sum_v[warp];
-  const int excl_f = f - flag + warp_sum_f[warp];
-  if (tid < E) {
-    start[tid] = excl_v;
-    if (flag) { sizes[excl_f] = tot; expert_ids[excl_f] = tid; }
+  {
+    int pos = v - my_v + warp_sum_v[warp];
+    int grp = f - my_f + warp_sum_f[warp];
+    for (int e = e0; e < e1; ++e) {
+      const int cnt = start[e];
+      start[e] = pos;
+      if (cnt > 0) { sizes[grp] = cnt; expert_ids[grp] = e; ++grp; }
+      pos += cnt;
+    }
   }
   __syncthreads();
   const int ngroups = s_groups;
-  for (int g = ngroups + tid; g < E; g += kAlignThreads) { sizes[g] = 0; expert_ids[g] = -1; }
+  for (int g = ngroups + tid; g < E; g += NT) { sizes[g] = 0; expert_ids[g] = -1; }
   if (tid == 0) *num_groups = ngroups;
 
   // 4. stable scatter, 32 slots per warp step
@@ -119,25 +129,46 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     __syncwarp();
   }
   // slots with an invalid id are left out; pad the tail of the permutation
-  for (int i = s_valid + tid; i < S; i += kAlignThreads) sorted_idx[i] = -1;
+  for (int i = s_valid + tid; i < S; i += NT) sorted_idx[i] = -1;
 }
+
+constexpr int kSmallWarps = 8;    // up to kSmallSlots slots
+constexpr int kLargeWarps = 32;
+constexpr int kSmallSlots = 4096;
 
 }  // namespace
 
 size_t moe_align_smem_bytes(int32_t E) {
-  return static_cast<size_t>(kAlignWarps + 1) * static_cast<size_t>(E) * sizeof(int32_t);
+  return static_cast<size_t>(kLargeWarps + 1) * static_cast<size_t>(E) * sizeof(int32_t);
 }
 
 cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t *sorted_idx,
                              int32_t *sizes, int32_t *expert_ids, int32_t *num_groups,
                              WsHeader *hdr, cudaStream_t stream) {
-  const size_t smem = moe_align_smem_bytes(E);
-  cudaError_t err = cudaFuncSetAttribute(moe_align_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  moe_align_kernel<<<1, kAlignThreads, smem, stream>>>(topk, S, E, sorted_idx, sizes, expert_ids,
-                                                       num_groups, hdr);
+  // Opt in once per device to the largest table the kernels can need, so
+  // that later calls (including ones under stream capture) set no attributes.
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    const int big = static_cast<int>(moe_align_smem_bytes(GNF4_MAX_EXPERTS));
+    cudaError_t err = cudaFuncSetAttribute(moe_align_kernel<kSmallWarps>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(moe_align_kernel<kLargeWarps>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
+  }
+  if (S <= kSmallSlots) {
+    const size_t smem = static_cast<size_t>(kSmallWarps + 1) * E * sizeof(int32_t);
+    moe_align_kernel<kSmallWarps><<<1, kSmallWarps * 32, smem, stream>>>(
+        topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
+  } else {
+    const size_t smem = static_cast<size_t>(kLargeWarps + 1) * E * sizeof(int32_t);
+    moe_align_kernel<kLargeWarps><<<1, kLargeWarps * 32, smem, stream>>>(
+        topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
+  }
   return cudaGetLastError();
 }
 
