@@ -27,6 +27,8 @@ from .binding import (  # noqa: F401
     gnf4_workspace_bytes,
     gnf4_moe_align,
     gnf4_grouped_gemm,
+    gnf4_grouped_gemm_noalloc,
+    GNF4_NOALLOC_SCRATCH_BYTES,
     gnf4_dequant_debug,
     gnf4_read_device_status,
     make_workspace,

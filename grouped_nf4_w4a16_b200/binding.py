@@ -22,7 +22,9 @@ _STATUS_NAMES = {
     0: "GNF4_OK", 1: "GNF4_ERR_INVALID_ARGUMENT", 2: "GNF4_ERR_HOST_POINTER",
     3: "GNF4_ERR_UNSUPPORTED_SHAPE", 4: "GNF4_ERR_WORKSPACE_TOO_SMALL", 5: "GNF4_ERR_CUDA",
     6: "GNF4_ERR_DEVICE_METADATA", 7: "GNF4_ERR_TIMEOUT", 8: "GNF4_ERR_MISALIGNED",
+    9: "GNF4_ERR_SCRATCH_LIMIT",
 }
+GNF4_NOALLOC_SCRATCH_BYTES = 8 << 20
 GNF4_EPI_NONE, GNF4_EPI_SWIGLU = 0, 1
 GNF4_MODE_AUTO, GNF4_MODE_DECODE, GNF4_MODE_PREFILL = 0, 1, 2
 GNF4_OUT_F32, GNF4_OUT_BF16 = 0, 1
@@ -33,6 +35,7 @@ DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capaci
 EXPORTED_SYMBOLS = (
     "gnf4_moe_align", "gnf4_grouped_gemm", "gnf4_dequant_debug", "gnf4_workspace_bytes",
     "gnf4_read_device_status", "gnf4_status_string", "gnf4_version",
+    "gnf4_grouped_gemm_noalloc",
 )
 
 _lib = None
@@ -64,6 +67,9 @@ def load_library():
     lib.gnf4_grouped_gemm.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P,
                                       P, sz, P]
     lib.gnf4_grouped_gemm.restype = ctypes.c_int
+    lib.gnf4_grouped_gemm_noalloc.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32,
+                                              P, P]
+    lib.gnf4_grouped_gemm_noalloc.restype = ctypes.c_int
     lib.gnf4_dequant_debug.argtypes = [P, P, i64, i32, i32, i32, P, P]
     lib.gnf4_dequant_debug.restype = ctypes.c_int
     lib.gnf4_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
@@ -165,6 +171,38 @@ def gnf4_grouped_gemm(x: torch.Tensor, w: torch.Tensor, absmax: torch.Tensor, si
         _ptr(x), _ptr(w), _ptr(absmax), _ptr(sizes), _ptr(expert_ids), G, M, N, K, E, blocksize,
         epilogue, mode, _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "gnf4_grouped_gemm")
+    return y
+
+
+def gnf4_grouped_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, absmax: torch.Tensor,
+                              sizes: torch.Tensor, expert_ids: torch.Tensor, *,
+                              epilogue: int = GNF4_EPI_NONE, y: Optional[torch.Tensor] = None,
+                              blocksize: int = 64, stream=None) -> torch.Tensor:
+    """The decode grouped GEMM without a workspace argument.
+
+    For callers that must not allocate device memory: the library uses its own
+    fixed scratch array (GNF4_NOALLOC_SCRATCH_BYTES per GPU). Calls must not
+    overlap on the GPU; problems larger than the scratch raise
+    GNF4_ERR_SCRATCH_LIMIT. Pass `y` to avoid the output allocation here.
+    """
+    _need(x, "x", torch.bfloat16)
+    _need(w, "w", torch.uint8)
+    _need(absmax, "absmax", torch.float32)
+    _need(sizes, "sizes", torch.int32)
+    _need(expert_ids, "expert_ids", torch.int32)
+    M, K = x.shape
+    E, N, Kh = w.shape
+    if Kh * 2 != K:
+        raise ValueError(f"w has K/2={Kh} but x has K={K}")
+    n_out = N // 2 if epilogue == GNF4_EPI_SWIGLU else N
+    if y is None:
+        y = torch.empty((M, n_out), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(y, "y", torch.bfloat16)
+    st = load_library().gnf4_grouped_gemm_noalloc(
+        _ptr(x), _ptr(w), _ptr(absmax), _ptr(sizes), _ptr(expert_ids), sizes.numel(), M, N, K, E,
+        blocksize, epilogue, _ptr(y), _stream(stream))
+    _check(st, "gnf4_grouped_gemm_noalloc")
     return y
 
 

@@ -65,6 +65,9 @@ const char *gnf4_status_string(gnf4_status s) {
     case GNF4_ERR_DEVICE_METADATA: return "GNF4_ERR_DEVICE_METADATA";
     case GNF4_ERR_TIMEOUT: return "GNF4_ERR_TIMEOUT";
     case GNF4_ERR_MISALIGNED: return "GNF4_ERR_MISALIGNED";
+    case GNF4_ERR_SCRATCH_LIMIT:
+      return "GNF4_ERR_SCRATCH_LIMIT (problem needs more than the fixed scratch of "
+             "gnf4_grouped_gemm_noalloc; use gnf4_grouped_gemm with a workspace)";
   }
   return "GNF4_ERR_UNKNOWN";
 }

@@ -509,6 +509,11 @@ size_t decode_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_
   return kWsHeaderBytes + cnt_bytes + part_bytes;
 }
 
+size_t decode_zero_prefix_bytes(int64_t M, int32_t N, int32_t G, int32_t swiglu) {
+  const int64_t tile_cap = decode_tile_cap(M, N, G, swiglu);
+  return kWsHeaderBytes + ((static_cast<size_t>(tile_cap) * 4 + 255) / 256) * 256;
+}
+
 cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   const int64_t tile_cap = decode_tile_cap(a.M, a.N, a.G, a.swiglu);
   const size_t cnt_bytes = ((static_cast<size_t>(tile_cap) * 4 + 255) / 256) * 256;

@@ -39,6 +39,9 @@ cudaError_t launch_dequant(const uint8_t *w, const float *absmax, int64_t rows, 
 
 // ---- decode-regime grouped GEMM (decode_gemm.cu)
 size_t decode_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu);
+// Leading bytes of a decode workspace that must be zero before a launch
+// (header and split-tile counters; the partial sums behind them need not be).
+size_t decode_zero_prefix_bytes(int64_t M, int32_t N, int32_t G, int32_t swiglu);
 cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream);
 
 // ---- prefill-regime grouped GEMM (prefill_gemm.cu)

@@ -1,0 +1,83 @@
+// noalloc.cu -- gnf4_grouped_gemm_noalloc: the decode grouped GEMM for callers
+// that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc at all: a plugin running inside a host
+// application that owns every byte of device memory through its own
+// pre-planned pool, or a latency-critical path that cannot pay for the
+// implicit synchronisation an allocation may bring. gnf4_grouped_gemm needs a
+// caller-provided workspace (split-tile counters and partial sums of the
+// decode kernel); this entry point instead uses a scratch array compiled into
+// the library, so the caller passes only inputs and outputs.
+//
+// The array is reserved on every GPU that loads the library, for the life of
+// the process. In host code its name only denotes a host-side stand-in, not a
+// device address, so the address handed to the kernel is looked up once per
+// device with cudaGetSymbolAddress (with that device current).
+#include <mutex>
+
+#include "launch.h"
+
+namespace gnf4 {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GNF4_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_lock;
+void *g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device, looked up on the
+// first call for that device.
+cudaError_t scratch_address(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> guard(g_scratch_lock);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace gnf4
+
+using namespace gnf4;
+
+extern "C" gnf4_status gnf4_grouped_gemm_noalloc(const uint16_t *x, const uint8_t *w,
+                                                 const float *absmax, const int32_t *sizes,
+                                                 const int32_t *expert_ids, int32_t G, int64_t M,
+                                                 int32_t N, int32_t K, int32_t E,
+                                                 int32_t blocksize, int32_t epilogue, uint16_t *y,
+                                                 gnf4_stream_t stream) {
+  // Shape checks that decide how much scratch the call needs; every other
+  // check is made by gnf4_grouped_gemm below, unchanged.
+  if (!x || !w || !absmax || !sizes || !expert_ids || !y) return GNF4_ERR_INVALID_ARGUMENT;
+  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (epilogue != GNF4_EPI_NONE && epilogue != GNF4_EPI_SWIGLU) return GNF4_ERR_INVALID_ARGUMENT;
+  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return GNF4_OK;
+
+  const size_t need = gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G);
+  if (need == 0 || need > GNF4_NOALLOC_SCRATCH_BYTES) return GNF4_ERR_SCRATCH_LIMIT;
+
+  void *scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return GNF4_ERR_CUDA;
+
+  // The array still holds the previous call's contents: the error word and
+  // the split-tile counters must start at zero.
+  const size_t clear =
+      decode_zero_prefix_bytes(M, N, G, epilogue == GNF4_EPI_SWIGLU ? 1 : 0);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, clear, s) != cudaSuccess) return GNF4_ERR_CUDA;
+
+  return gnf4_grouped_gemm(x, w, absmax, sizes, expert_ids, G, M, N, K, E, blocksize, epilogue,
+                           GNF4_MODE_DECODE, y, scratch, GNF4_NOALLOC_SCRATCH_BYTES, stream);
+}

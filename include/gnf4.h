@@ -68,7 +68,9 @@ typedef enum {
     GNF4_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
     GNF4_ERR_DEVICE_METADATA = 6,     /* (read_device_status) device data was invalid */
     GNF4_ERR_TIMEOUT = 7,             /* (read_device_status) a bounded device wait ran out */
-    GNF4_ERR_MISALIGNED = 8           /* a pointer breaks the alignment rule below */
+    GNF4_ERR_MISALIGNED = 8,          /* a pointer breaks the alignment rule below */
+    GNF4_ERR_SCRATCH_LIMIT = 9        /* problem needs more than the fixed scratch of
+                                         gnf4_grouped_gemm_noalloc */
 } gnf4_status;
 
 typedef enum { GNF4_EPI_NONE = 0, GNF4_EPI_SWIGLU = 1 } gnf4_epilogue;
@@ -195,6 +197,46 @@ GNF4_API size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K
  */
 GNF4_API gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uint32_t *error_bits,
                                     gnf4_stream_t stream);
+
+/*
+ * gnf4_grouped_gemm_noalloc -- gnf4_grouped_gemm (decode kernel) with no
+ * caller-provided workspace.
+ *
+ * No counterpart in the grouped-nf4-gemm pages: this entry point exists for
+ * callers that must not allocate device memory themselves, for example a
+ * plugin inside a host application that hands out all device memory from its
+ * own pre-planned pool and forbids further cudaMalloc calls, or a
+ * latency-critical path that cannot afford the implicit synchronisation an
+ * allocation may cause.
+ *
+ * It computes exactly what gnf4_grouped_gemm computes with mode =
+ * GNF4_MODE_DECODE (same arguments, minus workspace and mode), using a
+ * scratch area that lives inside the library: a fixed device array of
+ * GNF4_NOALLOC_SCRATCH_BYTES bytes, reserved on every GPU that loads the
+ * library for as long as the process runs. Nothing is allocated or freed.
+ *  - The first call on a device looks up that array's device address (one
+ *    runtime query, once per device, with that device current). Make that
+ *    first call before starting any stream capture on the device.
+ *  - Problems whose scratch need (gnf4_workspace_bytes for the same sizes)
+ *    exceeds GNF4_NOALLOC_SCRATCH_BYTES are refused with
+ *    GNF4_ERR_SCRATCH_LIMIT before anything is launched.
+ *  - All calls share the one array and it keeps the previous call's
+ *    contents; each call first clears the part that must start at zero (an
+ *    asynchronous memset on `stream`). Calls whose GPU work can overlap (on
+ *    different streams, or from different threads) race on the array and
+ *    give wrong results: serialise them.
+ *  - Device-side metadata errors leave y unwritten, as in gnf4_grouped_gemm,
+ *    but the error word stays inside the library's array; use
+ *    gnf4_grouped_gemm with a workspace when the error word is needed.
+ */
+#define GNF4_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB per device */
+
+GNF4_API gnf4_status gnf4_grouped_gemm_noalloc(const uint16_t *x, const uint8_t *w,
+                                               const float *absmax, const int32_t *sizes,
+                                               const int32_t *expert_ids, int32_t G, int64_t M,
+                                               int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                                               int32_t epilogue, uint16_t *y,
+                                               gnf4_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 GNF4_API const char *gnf4_status_string(gnf4_status status);
