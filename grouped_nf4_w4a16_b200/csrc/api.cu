@@ -143,7 +143,9 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
   int32_t use = mode;
   if (use == GNF4_MODE_AUTO) {
     const int64_t groups = G < E ? G : E;
-    use = (M > kPrefillMeanRows * groups) ? GNF4_MODE_PREFILL : GNF4_MODE_DECODE;
+    // the tensor-core kernel has no fused SwiGLU yet: SwiGLU stays on the decode kernel
+    use = (M > kPrefillMeanRows * groups && epilogue == GNF4_EPI_NONE) ? GNF4_MODE_PREFILL
+                                                                       : GNF4_MODE_DECODE;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (use == GNF4_MODE_PREFILL) {

@@ -145,8 +145,11 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *   blocksize   must be 64
  *   epilogue    gnf4_epilogue
  *   mode        gnf4_mode: AUTO picks DECODE when the mean rows per possible
- *               group, M / min(G, E), is at most 64, else PREFILL. Both
- *               modes accept any group sizes; the mode only selects the kernel.
+ *               group, M / min(G, E), is at most 64 or when SwiGLU is fused,
+ *               else PREFILL. Both modes accept any group sizes; the mode only
+ *               selects the kernel. PREFILL with SWIGLU is refused with
+ *               GNF4_ERR_UNSUPPORTED_SHAPE (the tensor-core kernel has no
+ *               fused SwiGLU).
  *   y           device bf16 [M][N] or [M][N/2]; fully overwritten; must not
  *               overlap x, w, absmax or the workspace.
  *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G)

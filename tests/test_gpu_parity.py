@@ -223,3 +223,48 @@ def test_host_tensors_are_refused_on_gpu_box():
         gnf4.gnf4_grouped_gemm(x, w, a, s, e, y=torch.zeros((4, 8), dtype=torch.bfloat16),
                                workspace=torch.zeros(1 << 20, dtype=torch.uint8))
     assert ei.value.status == 2
+
+
+# ----------------------------------------------------- prefill (tensor cores)
+@pytest.mark.parametrize("E,N,K,sizes,experts", [
+    (3, 200, 192, [300, 0, 513, 7], [2, 0, 1, 1]),     # ragged groups, N % 128 != 0
+    (2, 384, 2048, [256, 255, 257], [1, 0, 1]),        # token-tile edges
+    (4, 128, 64, [1, 1000], [3, 0]),                   # one K stage, a one-row group
+    (1, 136, 640, [70], [0]),                          # a single partial tile
+])
+def test_prefill_gemm_edge_cases(E, N, K, sizes, experts):
+    rng = np.random.default_rng(E * 13 + N + K)
+    M = int(sum(sizes))
+    x = synth.activations_bf16(M, K, seed=E + N + K)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    rows = np.unique(np.concatenate([boundaries(sizes), sample_rows(M, 96, 7)]))
+    check_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_PREFILL, rows=rows)
+
+
+@pytest.mark.parametrize("gi", [0, 1])
+def test_prefill_gemm_full_size_mixtral(gi):
+    # Full Mixtral-8x22B-shaped GEMMs in the launch configuration the benchmark
+    # times (AUTO -> tensor-core kernel), checked on sampled rows. The packed
+    # stack is drawn directly (uniform codes, absmax in the quantised-N(0,0.02)
+    # range): a multi-GB quantiser run adds nothing to this check.
+    w = synth.WORKLOADS["mixtral_8x22b"]
+    g = w.gemms[gi]
+    _, sizes, experts, ng = groups_from_routing(w)
+    packed, absmax = synth.random_packed_stack(w.E, g.N, g.K, seed=0, which=g.name)
+    x = synth.activations_bf16(w.M, g.K, seed=0, which=g.name)
+    rows = np.unique(np.concatenate([boundaries(sizes), sample_rows(w.M, 16, 3)]))
+    check_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_AUTO, rows=rows)
+
+
+def test_prefill_refuses_fused_swiglu():
+    rng = np.random.default_rng(3)
+    x = synth.activations_bf16(300, 64, seed=3)
+    packed = rng.integers(0, 256, size=(1, 64, 32), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(1, 64, 1)).astype(np.float32)
+    with pytest.raises(gnf4.Gnf4Error) as ei:
+        run_gemm(x, packed, absmax, [300], [0], swiglu=True, mode=gnf4.GNF4_MODE_PREFILL)
+    assert ei.value.status == 3
+    # AUTO keeps a fused SwiGLU on the decode kernel
+    check_gemm(x, packed, absmax, [300], [0], swiglu=True, mode=gnf4.GNF4_MODE_AUTO,
+               rows=np.array([0, 150, 299]))
