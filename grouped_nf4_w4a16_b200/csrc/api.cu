@@ -124,6 +124,9 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
   if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
   if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
   if (M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  // tensor-copy coordinates are 32-bit: every weight row index a copy can
+  // start at (up to one expert plus one box past the stack) must fit
+  if (static_cast<int64_t>(E) * N + N + 256 >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return GNF4_OK;
   if (!is_device_pointer(x) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
       !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(y) ||
@@ -148,12 +151,10 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
                                                                        : GNF4_MODE_DECODE;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (use == GNF4_MODE_PREFILL) {
-    const cudaError_t e = launch_prefill_gemm(a, s);
-    if (e == cudaErrorNotSupported) return GNF4_ERR_UNSUPPORTED_SHAPE;
-    return from_cuda(e);
-  }
-  return from_cuda(launch_decode_gemm(a, s));
+  const cudaError_t e =
+      use == GNF4_MODE_PREFILL ? launch_prefill_gemm(a, s) : launch_decode_gemm(a, s);
+  if (e == cudaErrorNotSupported) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
 }
 
 gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,

@@ -157,6 +157,16 @@ cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t 
     if (err == cudaSuccess)
       err = cudaFuncSetAttribute(moe_align_kernel<kLargeWarps>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    // Same shared-memory carveout as the GEMM kernels that follow, so the SM
+    // need not be reconfigured between the launches of one MoE layer.
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(moe_align_kernel<kSmallWarps>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(moe_align_kernel<kLargeWarps>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }

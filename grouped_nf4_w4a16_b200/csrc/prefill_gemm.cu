@@ -36,9 +36,7 @@
 // free), accumulator full/empty; every wait is bounded (2 s), after which the
 // kernel records GNF4_DEVERR_TIMEOUT, drains what it started and returns.
 #include "launch.h"
-
-#include <cuda.h>
-#include <cudaTypedefs.h>
+#include "sm100.cuh"
 
 namespace gnf4 {
 namespace {
@@ -69,60 +67,7 @@ constexpr int kNumBars = 3 * kStages + 3;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;          // int[8]
 constexpr int kSmemBytes = kMiscOff + 8 * 4 + 1024;       // + alignment slack
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;
-
 // ------------------------------------------------------------------ PTX
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
-          smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-// Bounded wait; returns false (after flagging) if it ran out or another
-// thread already flagged an abort.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         WsHeader *hdr) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  while (true) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
-      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
-      return false;
-    }
-  }
-}
-
-// Warp-uniform bounded wait: lane 0 waits, every lane gets the same answer,
-// so warp-collective instructions after it are never reached by part of a warp.
-__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, WsHeader *hdr) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, hdr) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int c0, int c1,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -267,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(d_empty, kDecodeThreads);
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+    prefetch_tensormap(&xmap);
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -348,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // drain: the last issued copies must land before the CTA exits
         for (uint32_t d = 0; d < kStages && d < g; ++d) {
           const uint32_t gg = g - 1 - d;
-          wait_bar(&x_full[gg % kStages], (gg / kStages) & 1u, abort_flag, hdr);
+          drain_wait(&x_full[gg % kStages], (gg / kStages) & 1u);
         }
       }
     } else if (warp == 1) {
@@ -384,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // drain every MMA this thread issued before TMEM is released
         mma_commit(drain);
-        wait_bar(drain, 0, abort_flag, hdr);
+        drain_wait(drain, 0);
       }
     } else if (warp >= kDecodeWarp0) {
       // ---------------------------------------------------- decode + epilogue
@@ -481,20 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 }  // namespace
 
 size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu) {
@@ -504,17 +435,12 @@ size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32
 
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (a.swiglu) return cudaErrorNotSupported;   // fused SwiGLU is decode-only for now
-  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
-  if (encode == nullptr) return cudaErrorNotSupported;
   CUtensorMap xmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBN)};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.x), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // activations as [M rows][K bf16], boxes of 256 rows x 64 elements
+  if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
+                            static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M),
+                            static_cast<uint64_t>(a.K) * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
 
   static bool configured[64] = {false};
   int dev = 0;
