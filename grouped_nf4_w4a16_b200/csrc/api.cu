@@ -135,9 +135,6 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
   if (!aligned(x, 32) || !aligned(w, 32) || !aligned(y, 32) || !aligned(workspace, 32) ||
       !aligned(absmax, 4) || !aligned(sizes, 4) || !aligned(expert_ids, 4))
     return GNF4_ERR_MISALIGNED;
-  if (ws_bytes < gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G))
-    return GNF4_ERR_WORKSPACE_TOO_SMALL;
-
   GemmArgs a;
   a.x = x; a.w = w; a.absmax = absmax; a.sizes = sizes; a.expert_ids = expert_ids;
   a.G = G; a.M = M; a.N = N; a.K = K; a.E = E; a.swiglu = (epilogue == GNF4_EPI_SWIGLU);
@@ -150,6 +147,11 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
     use = (M > kPrefillMeanRows * groups && epilogue == GNF4_EPI_NONE) ? GNF4_MODE_PREFILL
                                                                        : GNF4_MODE_DECODE;
   }
+  // the workspace the chosen kernel needs (gnf4_workspace_bytes covers every mode)
+  const int32_t swg = epilogue == GNF4_EPI_SWIGLU ? 1 : 0;
+  const size_t need = use == GNF4_MODE_PREFILL ? prefill_workspace_bytes(M, N, K, G, swg)
+                                               : decode_workspace_bytes(M, N, K, G, swg);
+  if (ws_bytes < need) return GNF4_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e =
       use == GNF4_MODE_PREFILL ? launch_prefill_gemm(a, s) : launch_decode_gemm(a, s);

@@ -5,9 +5,9 @@
 // application that owns every byte of device memory through its own
 // pre-planned pool, or a latency-critical path that cannot pay for the
 // implicit synchronisation an allocation may bring. gnf4_grouped_gemm needs a
-// caller-provided workspace (split-tile counters and partial sums of the
-// decode kernel); this entry point instead uses a scratch array compiled into
-// the library, so the caller passes only inputs and outputs.
+// caller-provided workspace (the status word the kernels report device-side
+// errors in); this entry point instead uses a scratch array compiled into the
+// library, so the caller passes only inputs and outputs.
 //
 // The array is reserved on every GPU that loads the library, for the life of
 // the process. In host code its name only denotes a host-side stand-in, not a
@@ -65,14 +65,16 @@ extern "C" gnf4_status gnf4_grouped_gemm_noalloc(const uint16_t *x, const uint8_
   if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return GNF4_OK;
 
-  const size_t need = gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G);
+  // the decode kernel's workspace (the 256-byte status header with the
+  // current kernel) must fit the scratch array
+  const size_t need = decode_workspace_bytes(M, N, K, G, epilogue == GNF4_EPI_SWIGLU ? 1 : 0);
   if (need == 0 || need > GNF4_NOALLOC_SCRATCH_BYTES) return GNF4_ERR_SCRATCH_LIMIT;
 
   void *scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return GNF4_ERR_CUDA;
 
-  // The array still holds the previous call's contents: the error word and
-  // the split-tile counters must start at zero.
+  // The array still holds the previous call's contents: the status word must
+  // start at zero.
   const size_t clear =
       decode_zero_prefix_bytes(M, N, G, epilogue == GNF4_EPI_SWIGLU ? 1 : 0);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -83,7 +83,8 @@ typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1 } gnf4_op;
 #define GNF4_DEVERR_EXPERT 0x2u     /* expert_ids[g] outside [0, E) on a non-empty group */
 #define GNF4_DEVERR_TOPK 0x4u       /* a topk id outside [0, E) */
 #define GNF4_DEVERR_TIMEOUT 0x8u    /* a bounded wait ran out */
-#define GNF4_DEVERR_CAPACITY 0x10u  /* work exceeded what the workspace was sized for */
+#define GNF4_DEVERR_CAPACITY 0x10u  /* work exceeded what the workspace was sized for
+                                       (reserved: no current kernel sets it) */
 
 /* Limits. */
 #define GNF4_MAX_EXPERTS 1024       /* E (and G) */
@@ -153,9 +154,17 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *   y           device bf16 [M][N] or [M][N/2]; fully overwritten; must not
  *               overlap x, w, absmax or the workspace.
  *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G)
- *               bytes, zero-filled once by the caller before its first use;
- *               the kernels leave its counters at zero again when they finish.
+ *               bytes (which covers every mode; the call itself only checks
+ *               the need of the kernel it runs and refuses less with
+ *               GNF4_ERR_WORKSPACE_TOO_SMALL). Its first 256 bytes are the
+ *               device status word: zero it once before the first use. The
+ *               current kernels need nothing more.
  *               Two calls that may run concurrently need separate workspaces.
+ * Numerics: every product enters an fp32 accumulator with the weight carried
+ *   as two bf16 parts (hi + lo within 2^-18 relative of its fp32 value):
+ *   DECODE splits each code value and scales each 64-element block sum by
+ *   absmax in fp32; PREFILL splits each fp32 weight NF4[code] * absmax and
+ *   runs the tensor cores once on each part.
  * Alignment: x, w, y and the workspace 32-byte aligned; absmax 4-byte aligned.
  * On a device-side metadata error no output is written.
  */
@@ -220,9 +229,11 @@ GNF4_API gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uin
  *  - The first call on a device looks up that array's device address (one
  *    runtime query, once per device, with that device current). Make that
  *    first call before starting any stream capture on the device.
- *  - Problems whose scratch need (gnf4_workspace_bytes for the same sizes)
- *    exceeds GNF4_NOALLOC_SCRATCH_BYTES are refused with
- *    GNF4_ERR_SCRATCH_LIMIT before anything is launched.
+ *  - Problems whose decode-kernel workspace exceeds
+ *    GNF4_NOALLOC_SCRATCH_BYTES are refused with GNF4_ERR_SCRATCH_LIMIT
+ *    before anything is launched (the current decode kernel needs only the
+ *    256-byte status header, so no problem size reaches the limit; callers
+ *    should still handle the code).
  *  - All calls share the one array and it keeps the previous call's
  *    contents; each call first clears the part that must start at zero (an
  *    asynchronous memset on `stream`). Calls whose GPU work can overlap (on
