@@ -159,11 +159,13 @@ def _new_event(drv):
 
 
 def _elapsed_ms(drv, a, b):
-    """Elapsed time between two events recorded by external graph nodes."""
+    """Elapsed time between two events recorded by external graph nodes, or
+    NaN when the driver has no timestamps for them (e.g. under a profiler that
+    replays graph nodes one by one)."""
     out = ctypes.c_float(0.0)
     st = drv.cuEventElapsedTime(ctypes.byref(out), a, b)
     if st != 0:
-        raise RuntimeError(f"cuEventElapsedTime failed with CUresult {st}")
+        return float("nan")
     return float(out.value)
 
 
@@ -327,7 +329,7 @@ def run_ours(args, rank, world, local_rank):
     for e in evs:
         for k in range(nk):
             per_kernel[k].append(_elapsed_ms(drv, e[k], e[k + 1]))
-    kern_ms = [sum(v) / len(v) for v in per_kernel]
+    kern_ms = [sum(v) / len(v) for v in per_kernel]   # NaN if a timestamp was missing
 
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
@@ -500,9 +502,11 @@ def main():
     k_ms = kern_ms[1]
     kernel = "prefill_gemm" if prob.prefill else "decode_gemm_kernel"
     if prob.prefill:
+        # timed inside seconds of back-to-back steps: the sustained bf16 figure
         achieved = d0["flops"] / (k_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic_for(kernel, prob.name, "gate_up")}
     else:
         achieved = d0["bytes"] / (k_ms / 1e3) / 1e9
@@ -511,7 +515,9 @@ def main():
     roof["kernel"] = f"{kernel} ({d0['g'].name} launch)"
     roof["algorithmic_per_launch"] = d0["flops"] if prob.prefill else d0["bytes"]
     roof["launch_ms"] = k_ms
-    roof["peak_source"] = f"{pk['source']} (MEASURED_PEAKS.json)" if pk["source"] == "measured" else "fallback"
+    which = "bf16_tflops_sustained" if prob.prefill else "hbm_gbs"
+    roof["peak_source"] = (f"measured {which} (MEASURED_PEAKS.json)" if pk["source"] == "measured"
+                           else f"fallback {which}")
 
     kernels = {"moe_align": {"ms": kern_ms[0]}}
     for i, d in enumerate(prob.gemms):
@@ -525,7 +531,7 @@ def main():
     line = {
         "metric": METRIC, "value": val, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": prob.describe(),
         "roofline": roof,
         "kernels": kernels,
