@@ -97,4 +97,16 @@ __device__ __forceinline__ uint4 ldg128_stream(const void *p) {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// Programmatic dependent launch. Every kernel of the library is launched so
+// that it may start while the previous kernel on the stream is still
+// running; it then sets up what needs no input (shared-memory tables,
+// barriers) and calls pdl_wait() before its first read or write of global
+// memory: pdl_wait() returns once the previous kernel has finished and its
+// writes are visible (at once when there is no such dependency).
+// pdl_trigger() lets the next kernel on the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace gnf4

@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int64_t s_wsum[2][kThreads / 32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();
 
   Problem p;
   p.N = N; p.K = K; p.E = E; p.G = G; p.swiglu = swiglu;
@@ -242,6 +243,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&xmap);
   }
 
+  // ---- decode table: entry byte b, lane slot l = {bf16x2 hi, bf16x2 lo} of
+  //      the pair (NF4[b >> 4], NF4[b & 15]) (low half = even k = high nibble)
+  if (tid < 256) {
+    const uint32_t c0 = code_split(tid >> 4), c1 = code_split(tid & 15);
+    const uint32_t hp = (c0 & 0xFFFFu) | (c1 << 16);
+    const uint32_t lp = (c0 >> 16) | (c1 & 0xFFFF0000u);
+    uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + tid * 256);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) dst[i] = make_uint4(hp, lp, hp, lp);
+  }
+
+  pdl_wait();   // inputs may come from the previous kernel on the stream
+
   // ---- group table from (sizes, expert_ids), validated on the device
   const int per = (G + kThreads - 1) / kThreads;
   const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
@@ -258,16 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
   }
 
-  // ---- decode table: entry byte b, lane slot l = {bf16x2 hi, bf16x2 lo} of
-  //      the pair (NF4[b >> 4], NF4[b & 15]) (low half = even k = high nibble)
-  if (tid < 256) {
-    const uint32_t c0 = code_split(tid >> 4), c1 = code_split(tid & 15);
-    const uint32_t hp = (c0 & 0xFFFFu) | (c1 << 16);
-    const uint32_t lp = (c0 >> 16) | (c1 & 0xFFFF0000u);
-    uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + tid * 256);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) dst[i] = make_uint4(hp, lp, hp, lp);
-  }
   __syncthreads();   // barrier init and misc visible
   if (bad) atomicOr(&misc[0], bad);
 
@@ -532,10 +536,10 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  decode_gemm_kernel<<<device_sm_count(), kThreads, kSmemBytes, stream>>>(
-      wm, xmap, a.absmax, a.sizes, a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.swiglu, a.y,
-      static_cast<WsHeader *>(a.workspace));
-  return cudaGetLastError();
+  return launch_pdl(decode_gemm_kernel, dim3(device_sm_count()), dim3(kThreads),
+                    static_cast<size_t>(kSmemBytes), stream, wm, xmap, a.absmax, a.sizes,
+                    a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.swiglu, a.y,
+                    static_cast<WsHeader *>(a.workspace));
 }
 
 }  // namespace gnf4

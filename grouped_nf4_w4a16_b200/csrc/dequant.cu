@@ -19,8 +19,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
                                                       int64_t nchunks, int32_t K,
                                                       void *__restrict__ out) {
   __shared__ float lut[16];
+  pdl_trigger();
   if (threadIdx.x < 16) lut[threadIdx.x] = nf4_value(threadIdx.x);
   __syncthreads();
+  pdl_wait();   // inputs may come from the previous kernel on the stream
   const int64_t chunks_per_row = K / 32;
   const int64_t blocks_per_row = K / 64;
   for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < nchunks;
@@ -71,12 +73,11 @@ cudaError_t launch_dequant(const uint8_t *w, const float *absmax, int64_t rows, 
   int64_t want = (nchunks + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  if (out_bf16) {
-    dequant_kernel<true><<<grid, threads, 0, stream>>>(w, absmax, nchunks, K, out);
-  } else {
-    dequant_kernel<false><<<grid, threads, 0, stream>>>(w, absmax, nchunks, K, out);
-  }
-  return cudaGetLastError();
+  if (out_bf16)
+    return launch_pdl(dequant_kernel<true>, dim3(grid), dim3(threads), 0, stream, w, absmax,
+                      nchunks, K, out);
+  return launch_pdl(dequant_kernel<false>, dim3(grid), dim3(threads), 0, stream, w, absmax,
+                    nchunks, K, out);
 }
 
 }  // namespace gnf4

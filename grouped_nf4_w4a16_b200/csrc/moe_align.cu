@@ -39,8 +39,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
   __shared__ int32_t s_valid, s_groups;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();
   for (int i = tid; i < NW * E; i += NT) hist[i] = 0;
   __syncthreads();
+  pdl_wait();   // topk may come from the previous kernel on the stream
 
   const int seg = (S + NW - 1) / NW;
   const int beg = min(S, warp * seg), end = min(S, beg + seg);
@@ -172,14 +174,12 @@ cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t 
   }
   if (S <= kSmallSlots) {
     const size_t smem = static_cast<size_t>(kSmallWarps + 1) * E * sizeof(int32_t);
-    moe_align_kernel<kSmallWarps><<<1, kSmallWarps * 32, smem, stream>>>(
-        topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
-  } else {
-    const size_t smem = static_cast<size_t>(kLargeWarps + 1) * E * sizeof(int32_t);
-    moe_align_kernel<kLargeWarps><<<1, kLargeWarps * 32, smem, stream>>>(
-        topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
+    return launch_pdl(moe_align_kernel<kSmallWarps>, dim3(1), dim3(kSmallWarps * 32), smem, stream,
+                      topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
   }
-  return cudaGetLastError();
+  const size_t smem = static_cast<size_t>(kLargeWarps + 1) * E * sizeof(int32_t);
+  return launch_pdl(moe_align_kernel<kLargeWarps>, dim3(1), dim3(kLargeWarps * 32), smem, stream,
+                    topk, S, E, sorted_idx, sizes, expert_ids, num_groups, hdr);
 }
 
 }  // namespace gnf4

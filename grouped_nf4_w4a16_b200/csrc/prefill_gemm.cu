@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = &misc[1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();
 
   // ---- set-up: decode table, barriers, TMEM
   for (int i = tid; i < 256 * 32; i += kThreads) {
@@ -221,6 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+
+  pdl_wait();   // inputs may come from the previous kernel on the stream
 
   // ---- group table (validated; same rules as the decode kernel)
   __shared__ int s_wsum[2][kThreads / 32];
@@ -451,10 +454,10 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  prefill_gemm_kernel<<<device_sm_count(), kThreads, kSmemBytes, stream>>>(
-      xmap, a.w, a.absmax, a.sizes, a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
-      static_cast<WsHeader *>(a.workspace));
-  return cudaGetLastError();
+  return launch_pdl(prefill_gemm_kernel, dim3(device_sm_count()), dim3(kThreads),
+                    static_cast<size_t>(kSmemBytes), stream, xmap, a.w, a.absmax, a.sizes,
+                    a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
+                    static_cast<WsHeader *>(a.workspace));
 }
 
 }  // namespace gnf4
