@@ -169,6 +169,16 @@ def _elapsed_ms(drv, a, b):
     return float(out.value)
 
 
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks (x itself when world == 1). Every
+    rank must call it at the same point: it is one all-reduce."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ problem
 class Problem:
     """Device-resident inputs for one workload (seeded, synthetic)."""
@@ -343,13 +353,11 @@ def run_ours(args, rank, world, local_rank):
             per_kernel[k].append(_elapsed_ms(drv, e[k], e[k + 1]))
     kern_ms = [sum(v) / len(v) for v in per_kernel]   # NaN if a timestamp was missing
 
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     # end to end: host (pinned) inputs -> device, the C-ABI calls, results -> host
     e2e = run_e2e(prob, stream, max(3, min(args.steps, 2000) // 10))
+    e2e = (max_over_ranks(e2e[0], world, dev),) + tuple(e2e[1:])
     return prob, ms, kern_ms, clk, e2e, launches_per_step
 
 
@@ -448,10 +456,9 @@ def metric_value(prob, sec_per_step, n_ranks=1):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    prob = Problem(args.workload, seed=0, device="cuda" if torch.cuda.is_available() else "cpu") \
-        if torch.cuda.is_available() else None
-    if prob is None:
-        raise SystemExit("the reference arm builds its inputs with the same generator on the GPU box")
+    # the oracle runs on the host cores; its inputs are the same seeded arrays
+    prob = Problem(args.workload, seed=0, replicas=1,
+                   device="cuda" if torch.cuda.is_available() else "cpu")
     budget = max(3.0, min(60.0, 2.0 * (args.steps + args.warmup)))
     sec, sample, threads = oracle_step_sample(prob, budget)
     val, unit = metric_value(prob, sec)
@@ -464,6 +471,8 @@ def run_reference(args, rank, world):
                          "sample": sample},
         "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    line["config"]["graph"] = "none: the oracle runs on the host cores"
+    line["config"]["l2"] = "not applicable (host run)"
     return line
 
 
@@ -489,10 +498,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group(
-            "nccl", device_id=torch.device("cuda", local_rank),
-            timeout=__import__("datetime").timedelta(seconds=120))
+        timeout = __import__("datetime").timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group(
+                "nccl", device_id=torch.device("cuda", local_rank), timeout=timeout)
+        else:   # host-only runs (the reference arm, tests): gloo
+            torch.distributed.init_process_group("gloo", timeout=timeout)
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)

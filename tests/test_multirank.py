@@ -1,0 +1,45 @@
+"""The N > 1 host logic of bench.py on CPU, world size 2 over gloo: the
+max-over-ranks timing reduction, and the reference arm (rank 0 runs and
+prints one line, the other rank exits 0 without work)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _torchrun(args, timeout=600):
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port())] + args
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="2")
+    return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=timeout)
+
+
+def test_max_over_ranks_world_size_2():
+    r = _torchrun([os.path.join("tests", "multirank_worker.py")])
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "rank 0 max 2.5" in r.stdout and "rank 1 max 2.5" in r.stdout
+
+
+def test_reference_arm_world_size_2_prints_one_line():
+    r = _torchrun(["bench.py", "--impl", "reference", "--workload", "tiny", "--gpus", "2",
+                   "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
