@@ -87,21 +87,6 @@ static_assert(kBarOff % 8 == 0 && kXchgOff % 8 == 0, "8-byte aligned");
 static_assert(kSmemBytes <= 227 * 1024, "fits one CTA per SM");
 
 // ------------------------------------------------------------------ PTX
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
-// The mbarrier receives one arrival when this thread's earlier cp.async
-// copies have landed (counted in the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
 
 // Not volatile: the compiler may interleave independent accumulation chains.
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,

@@ -1,5 +1,5 @@
 // prefill_gemm.cu -- prefill-regime grouped NF4 GEMM on the 5th-generation
-// tensor cores (tcgen05, TMEM, TMA).
+// tensor cores (tcgen05, TMEM, TMA), as a 2-SM MMA over CTA pairs.
 //
 // Passage: "grouped-nf4-gemm -- single-launch W4A16 GEMM over fused NF4 MoE
 // expert stacks", opening section (one launch for all active experts, LUT
@@ -8,64 +8,97 @@
 // register-LUT M-tile mainloop). With ~1000 activation rows per expert the
 // contraction is dense and bound by tensor-core throughput.
 //
-// Tile = 128 weight rows of one expert x 256 activation rows of one group,
-// computed as D[weight row][activation row] = W . x^T (weights as the MMA's
-// M side), K in stages of 64 (one absmax block).
+// Tile = 256 weight rows of one expert x 256 activation rows of one group,
+// computed as D[weight row][activation row] = W . x^T by a pair of CTAs on
+// two SMs (a cluster of 2): CTA r of the pair owns weight rows 128 r .. +127
+// (its TMEM lanes: the MMA's A and D) and activation rows 128 r .. +127 of
+// the tile (its shared memory: half of the MMA's B). One tcgen05.mma with
+// cta_group::2, issued by the pair's leader (r = 0), reads both halves, so
+// every SM loads only half of the activation tile per K-step.
 //
-// Roles (12 warps, one CTA per SM, persistent over tiles):
-//   warp 0  TMA producer: x tile [256 rows x 64] bf16 -> shared memory ring
-//           (4 stages, 128-byte swizzle, the canonical K-major operand layout).
-//   warp 1  MMA issuer (one thread): tcgen05.mma kind::f16, A from TMEM, B
-//           from shared memory, fp32 accumulator in TMEM (256 columns).
-//   warp 2  allocates / frees the 512 TMEM columns.
-//   warps 4-11  decoders + epilogue. Warp w owns TMEM lanes 32*(w%4).. (=
-//           weight rows) and half of the stage's 64 K-elements. Each lane
-//           loads its row's 16 packed bytes, decodes every byte with one
-//           shared-memory load of the fp32 pair (NF4[hi], NF4[lo]) (table
-//           replicated per lane: no bank conflicts), multiplies by the
-//           block's absmax in fp32 (the exact fp32 weight), and splits it into
-//           bf16 hi + bf16 lo (hi + lo = weight to 2^-18 relative). Both
-//           halves go straight to TMEM with tcgen05.st: the decoded weights
-//           never touch shared or global memory.
-//   The MMA runs twice per K-step, on the hi and on the lo weights, into the
-//   same accumulator, so the result is the fp32-exact-weight contraction
-//   (a single 16-bit weight would miss the 1e-3*rms elementwise tolerance at
-//   these output sizes). After the last stage the decoders read the
-//   accumulator back (tcgen05.ld), round to bf16 and store y.
-// Synchronisation: mbarriers per stage (x landed, weights decoded, stage
-// free), accumulator full/empty; every wait is bounded (2 s), after which the
-// kernel records GNF4_DEVERR_TIMEOUT, drains what it started and returns.
+// Numerics (the tolerance needs more than one bf16 per weight): each weight
+// row is scaled by 2^S, S = beta + 14 with 2^beta * max(absmax of the row) in
+// [1, 2) (powers of two scale exactly); the scaled fp32 weight w'' = NF4 *
+// absmax * 2^S is split into hi = bf16(w'') and the exact remainder
+// w'' - hi, which is below 64 in magnitude and goes to e4m3. Per K-step of 64:
+//   hi pass: 4 x kind::f16, bf16 hi (TMEM) x bf16 x (shared memory), K = 16
+//   lo pass: 2 x kind::f8f6f4, e4m3 remainder (TMEM) x e5m2 x (shared
+//            memory, an e5m2 copy of x made by a pre-pass), K = 32
+// into one fp32 accumulator; the epilogue divides 2^S out and rounds once to
+// bf16. The lo pass runs at twice the bf16 rate, so a K-step costs 1.5 bf16
+// passes instead of 2.
+//
+// Roles per CTA (12 warps, one CTA per SM, the pair persistent over tiles):
+//   warp 0  TMA: its half of the x tile (bf16, 128-byte swizzle) and of the
+//           e5m2 tile (64-byte swizzle); both halves complete on the leader's
+//           stage barrier (cta_group::2 copies), whose byte count the leader
+//           sets for the pair. Ring of 6 stages.
+//   warp 1  (leader) MMA issuer; commits signal both CTAs.
+//   warp 2  allocates / frees the 512 TMEM columns (cta_group::2, in both CTAs).
+//   warp 3  packed weights: this CTA's 128 rows x 4 K-steps (128 bytes a row)
+//           per TMA box (128-byte swizzle), and their absmax values by
+//           cp.async, into a 2-slot shared-memory ring. Decoders then read
+//           16 contiguous bytes per row per K-step without bank conflicts,
+//           instead of scattered global loads (one sector per row).
+//   warps 4-11  decoders + epilogue: warp w owns TMEM lanes 32 (w % 4).. and
+//           half of the K-step; each lane decodes its row's 32 codes through a
+//           per-lane replicated table of the 16 code values, writes hi and
+//           remainder to TMEM (tcgen05.st, a 5-stage ring); one lane per warp
+//           then arrives on the leader's barrier. The epilogue reads the
+//           accumulator back (tcgen05.ld).
+// Every wait is bounded (2 s); on expiry the kernel records
+// GNF4_DEVERR_TIMEOUT, lets its asynchronous work drain and returns through
+// the final cluster barrier.
+#include <cuda_fp8.h>
+
 #include "launch.h"
 #include "sm100.cuh"
 
 namespace gnf4 {
 namespace {
 
-constexpr int kBM = 128;            // weight rows per tile (TMEM lanes, MMA M)
+constexpr int kBM = 128;            // weight rows per CTA (TMEM lanes)
+constexpr int kPairM = 256;         // weight rows per pair tile (MMA M)
 constexpr int kBN = 256;            // activation rows per tile (MMA N)
+constexpr int kBNh = 128;           // activation rows loaded by each CTA
 constexpr int kBK = 64;             // K per stage
-constexpr int kStages = 4;
+constexpr int kXStages = 6;         // activation ring (shared memory)
+constexpr int kWQuads = 2;          // packed-weight ring: slots of 4 K-steps (shared memory)
+constexpr int kWSlotBytes = kBM * 128;       // 16 KB: 128 rows x 128 packed bytes
+constexpr int kASlotBytes = 4 * kBM * 4;     // 2 KB: absmax [4 blocks][128 rows]
+constexpr int kAStages = 5;         // decoded-weight ring (TMEM)
 constexpr int kThreads = 384;       // 12 warps
 constexpr int kDecodeWarp0 = 4;
-constexpr int kDecodeThreads = 256; // warps 4..11
+constexpr int kDecodeWarps = 8;     // warps 4..11
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;     // accumulator: columns [0, 256)
-constexpr uint32_t kACol = 256;     // stage s: hi at kACol + 64 s, lo at +32
-constexpr int kXStageBytes = kBN * kBK * 2;   // 32 KB
+constexpr uint32_t kACol = 256;     // stage s: hi at kACol + 48 s (32 columns), lo at +32 (16)
+constexpr uint32_t kAStageCols = 48;
+constexpr int kXStageBytes = kBNh * kBK * 2;   // 16 KB: this CTA's half of the x tile, bf16
+constexpr int kX8StageBytes = kBNh * kBK;      // 8 KB: the same half, e5m2
+constexpr uint32_t kPairStageBytes = 2u * (kXStageBytes + kX8StageBytes);
+constexpr int kLoShift = 14;        // weights are scaled by 2^(beta + 14)
+static_assert(kACol + kAStages * kAStageCols <= kTmemCols, "TMEM columns");
 
-// Shared memory layout (dynamic, 1024-aligned base).
-constexpr int kXOff = 0;                                  // x ring (1024-aligned stages)
-constexpr int kLutOff = kXOff + kStages * kXStageBytes;   // float2 [256][32]
-constexpr int kLutBytes = 256 * 32 * 8;
-constexpr int kTileStartOff = kLutOff + kLutBytes;        // int[kMaxG + 1]
+// Shared memory layout (dynamic, 1024-aligned base; identical in both CTAs,
+// which the pair MMA relies on: B's second half sits at the same offset in
+// the peer).
+constexpr int kXOff = 0;                                    // x ring
+constexpr int kX8Off = kXOff + kXStages * kXStageBytes;     // e5m2 ring
+constexpr int kWOff = kX8Off + kXStages * kX8StageBytes;    // packed-weight ring
+constexpr int kAbsOff = kWOff + kWQuads * kWSlotBytes;      // absmax ring
+constexpr int kLutOff = kAbsOff + kWQuads * kASlotBytes;    // float [16 codes][32 lanes]
+constexpr int kLutBytes = 16 * 32 * 4;
+constexpr int kTileStartOff = kLutOff + kLutBytes;          // int[kMaxG + 1]
 constexpr int kRowOffOff = kTileStartOff + (kMaxG + 4) * 4;
 constexpr int kGSizeOff = kRowOffOff + kMaxG * 4;
 constexpr int kGExpOff = kGSizeOff + kMaxG * 4;
-constexpr int kBarOff = kGExpOff + kMaxG * 4;             // mbarriers
-constexpr int kNumBars = 3 * kStages + 3;
-constexpr int kMiscOff = kBarOff + kNumBars * 8;          // int[8]
-constexpr int kSmemBytes = kMiscOff + 8 * 4 + 1024;       // + alignment slack
+constexpr int kBarOff = kGExpOff + kMaxG * 4;               // mbarriers
+constexpr int kNumBars = 2 * kXStages + 2 * kAStages + 2 * kWQuads + 3;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;            // int[8]
+constexpr int kSmemBytes = kMiscOff + 8 * 4 + 1024;         // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "fits one CTA per SM");
 
 // ------------------------------------------------------------------ PTX
 __device__ __forceinline__ void tc_fence_before() {
@@ -75,21 +108,96 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[tmem] . B[smem desc]^T, kind::f16 (bf16 inputs, fp32 accumulate).
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Both CTAs of the pair, all threads: release our writes, acquire the peer's.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared::cluster address of the object at `p`'s offset in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on the mbarrier at `p`'s offset in CTA `rank` (possibly this CTA).
+// CTA-scope semantics: the arrivals only hand over TMEM contents, which the
+// tcgen05 wait and fence order, not generic memory (a cluster-scope release
+// would also wait for every load the thread has in flight).
+__device__ __forceinline__ void mbar_arrive_cta(const uint64_t *p, uint32_t rank) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr(p, rank))
+               : "memory");
+}
+
+// Bounded-wait building block (arrivals may come from the peer CTA).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity);
+}
+
+__device__ __forceinline__ bool wait_bar_cluster(uint64_t *bar, uint32_t parity,
+                                                 volatile int *abort_flag, WsHeader *hdr) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer() - t0 > kTimeoutNs) {
+      *abort_flag = 1;
+      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
+      return false;
+    }
+  }
+}
+
+// 2-D tensor copy into this CTA's shared memory whose byte count completes
+// on the mbarrier at `bar`'s offset in the pair leader (CTA 0).
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *map, int c0,
+                                                 int c1, const uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(cluster_addr(bar, 0))
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem desc]^T over the pair: kind::f16 (bf16 x bf16).
+__device__ __forceinline__ void mma_pair_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
+// The same with kind::f8f6f4: e4m3 A (TMEM) x e5m2 B (shared memory), K = 32.
+__device__ __forceinline__ void mma_pair_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in every CTA of `mask` once all
+// MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(const uint64_t *bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -99,6 +207,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 
@@ -124,17 +239,28 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory operand descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), leading offset unused (1), descriptor version 1.
+// Shared-memory operand descriptors, K-major, descriptor version 1:
+// bf16 tile: 128-byte rows with the 128-byte swizzle, 8-row groups 1024 B apart;
+// e5m2 tile: 64-byte rows with the 64-byte swizzle, 8-row groups 512 B apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
   return static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
          (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
          (static_cast<uint64_t>(2) << 61);
 }
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t smem_addr) {
+  return static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(512 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(4) << 61);
+}
 
-// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M=128, N=256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
-                            (static_cast<uint32_t>(kBM >> 4) << 24);
+// Instruction descriptors (K-major A and B, fp32 D, M = 256 over the pair,
+// N = 256): kind::f16 with bf16 A and B; kind::f8f6f4 with e4m3 A, e5m2 B.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kPairM >> 4) << 24);
+constexpr uint32_t kIdescF8 = (1u << 4) | (0u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kBN >> 3) << 17) |
+                              (static_cast<uint32_t>(kPairM >> 4) << 24);
 
 __device__ __forceinline__ uint4 ldg128_nc(const void *p) {
   uint4 r;
@@ -145,13 +271,15 @@ __device__ __forceinline__ uint4 ldg128_nc(const void *p) {
 }
 
 struct TileInfo {
-  int64_t row0;     // first activation row of the tile
+  int64_t row0;     // first activation row of the pair tile
   int32_t rows;     // valid activation rows (1..256)
-  int32_t n0;       // first weight row (within the expert)
+  int32_t n0;       // first weight row (within the expert) of the pair tile
   int32_t e;        // expert
 };
 
-__device__ __forceinline__ TileInfo tile_info(int t, int G, int NJ, const int *tile_start,
+// Pair tile t: groups in order, within a group weight-row tile j outer and
+// token tile i inner (pairs running at the same time share weight tiles).
+__device__ __forceinline__ TileInfo tile_info(int t, int G, const int *tile_start,
                                               const int *row_off, const int *gsize,
                                               const int *gexp) {
   int lo = 0, hi = G;   // tile_start[lo] <= t < tile_start[hi]
@@ -165,13 +293,24 @@ __device__ __forceinline__ TileInfo tile_info(int t, int G, int NJ, const int *t
   TileInfo ti;
   ti.row0 = static_cast<int64_t>(row_off[lo]) + static_cast<int64_t>(i) * kBN;
   ti.rows = min(kBN, gsize[lo] - i * kBN);
-  ti.n0 = j * kBM;
+  ti.n0 = j * kPairM;
   ti.e = gexp[lo];
   return ti;
 }
 
+// Warp-uniform bounded wait with cluster-scope acquire: lane 0 waits, every
+// lane gets the same answer (warp-collective instructions follow).
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort_flag, WsHeader *hdr) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar_cluster(bar, parity, abort_flag, hdr) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t *__restrict__ w,
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+                        const __grid_constant__ CUtensorMap x8map,
+                        const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ w,
                         const float *__restrict__ absmax, const int32_t *__restrict__ sizes,
                         const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
                         int32_t K, int32_t E, uint16_t *__restrict__ y, WsHeader *hdr) {
@@ -179,55 +318,69 @@ __global__ void __launch_bounds__(kThreads, 1)
   char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~static_cast<uintptr_t>(1023));
   char *xs = smem + kXOff;
+  char *x8s = smem + kX8Off;
   int *tile_start = reinterpret_cast<int *>(smem + kTileStartOff);
   int *row_off = reinterpret_cast<int *>(smem + kRowOffOff);
   int *gsize = reinterpret_cast<int *>(smem + kGSizeOff);
   int *gexp = reinterpret_cast<int *>(smem + kGExpOff);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
-  uint64_t *x_full = bars;                  // [kStages] TMA landed
-  uint64_t *a_full = bars + kStages;        // [kStages] weights decoded into TMEM
-  uint64_t *st_free = bars + 2 * kStages;   // [kStages] MMA done reading the stage
-  uint64_t *d_full = bars + 3 * kStages;    // accumulator complete
-  uint64_t *d_empty = d_full + 1;           // accumulator read out
-  uint64_t *drain = d_full + 2;             // final MMA drain
+  uint64_t *x_full = bars;                  // [kXStages] (leader) both halves landed
+  uint64_t *x_free = x_full + kXStages;     // [kXStages] (each CTA) the MMA is done with them
+  uint64_t *a_full = x_free + kXStages;     // [kAStages] (leader) both CTAs' weights in TMEM
+  uint64_t *a_free = a_full + kAStages;     // [kAStages] (each CTA) the MMA is done with them
+  uint64_t *w_full = a_free + kAStages;     // [kWQuads] (each CTA) packed bytes + absmax landed
+  uint64_t *w_free = w_full + kWQuads;      // [kWQuads] (each CTA) decoders done with the slot
+  uint64_t *d_full = w_free + kWQuads;      // (each CTA) accumulator complete
+  uint64_t *d_empty = d_full + 1;           // (leader) both CTAs read their accumulators out
+  uint64_t *drain = d_full + 2;             // (leader) final MMA drain
   int *misc = reinterpret_cast<int *>(smem + kMiscOff);
   volatile int *abort_flag = &misc[1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
   pdl_trigger();
 
-  // ---- set-up: decode table, barriers, TMEM
-  for (int i = tid; i < 256 * 32; i += kThreads) {
-    const int b = i >> 5;
-    reinterpret_cast<float2 *>(smem + kLutOff)[i] = make_float2(nf4_value(b >> 4), nf4_value(b & 15));
-  }
+  // ---- set-up: decode table, barriers, TMEM (no global memory yet)
+  for (int i = tid; i < 16 * 32; i += kThreads)
+    reinterpret_cast<float *>(smem + kLutOff)[i] = nf4_value(i >> 5);
   if (tid == 0) {
     misc[0] = 0;
     misc[1] = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&x_full[s], 1);
-      mbar_init(&a_full[s], kDecodeThreads);
-      mbar_init(&st_free[s], 1);
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(&x_full[s], 1);                  // the leader's byte-count arrival
+      mbar_init(&x_free[s], 1);                  // the leader's commit
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&a_full[s], 2 * kDecodeWarps);   // one per decoder warp of each CTA
+      mbar_init(&a_free[s], 1);                  // the leader's commit
+    }
+    for (int q = 0; q < kWQuads; ++q) {
+      mbar_init(&w_full[q], 32 + 1);             // 32 cp.async arrivals + the byte-count arrival
+      mbar_init(&w_free[q], kDecodeWarps);
     }
     mbar_init(d_full, 1);
-    mbar_init(d_empty, kDecodeThreads);
+    mbar_init(d_empty, 2 * kDecodeWarps);
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&xmap);
+    prefetch_tensormap(&x8map);
+    prefetch_tensormap(&wmap);
   }
   if (warp == 2) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&misc[4])),
                  "r"(kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
 
-  // ---- group table (validated; same rules as the decode kernel)
+  // ---- group table (validated; both CTAs compute the same one)
   __shared__ int s_wsum[2][kThreads / 32];
-  const int NJ = (N + kBM - 1) / kBM;
+  const int NJ = (N + kPairM - 1) / kPairM;
   const int per = (G + kThreads - 1) / kThreads;
   const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
   int my_rows = 0, my_tiles = 0, bad = 0;
@@ -241,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     my_rows += max(sz, 0);
     my_tiles += sz > 0 ? ((sz + kBN - 1) / kBN) * NJ : 0;
   }
+  __syncthreads();
   if (bad) atomicOr(&misc[0], bad);
   int vr = my_rows, vt = my_tiles;
 #pragma unroll
@@ -269,8 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) tile_start[G] = tot_t;
   }
   if (tid == 0 && static_cast<int64_t>(tot_r) != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
+  // both CTAs: barriers initialised and TMEM allocated before any remote access
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[4]);
   const int errbits = misc[0];
@@ -283,118 +438,233 @@ __global__ void __launch_bounds__(kThreads, 1)
       // --------------------------------------------------------- TMA producer
       if (lane == 0) {
         uint32_t g = 0;   // stage ring counter
-        for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-          const TileInfo ti = tile_info(t, G, NJ, tile_start, row_off, gsize, gexp);
+        for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
+          const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
+          const int xrow = static_cast<int>(ti.row0) + kBNh * static_cast<int>(rank);
+          bool ok = true;
           for (int kb = 0; kb < KB; ++kb, ++g) {
-            const int s = g % kStages;
-            const uint32_t ph = (g / kStages) & 1u;
-            if (!wait_bar(&st_free[s], ph ^ 1u, abort_flag, hdr)) break;
-            mbar_arrive_expect_tx(&x_full[s], kXStageBytes);
-            tma_load_2d(xs + s * kXStageBytes, &xmap, kb * kBK, static_cast<int>(ti.row0), &x_full[s]);
+            const int s = g % kXStages;
+            const uint32_t ph = (g / kXStages) & 1u;
+            if (!wait_bar_cluster(&x_free[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
+            if (leader) mbar_arrive_expect_tx(&x_full[s], kPairStageBytes);
+            tma_load_2d_pair(xs + s * kXStageBytes, &xmap, kb * kBK, xrow, &x_full[s]);
+            tma_load_2d_pair(x8s + s * kX8StageBytes, &x8map, kb * kBK, xrow, &x_full[s]);
           }
+          if (!ok) break;
         }
-        // drain: the last issued copies must land before the CTA exits
-        for (uint32_t d = 0; d < kStages && d < g; ++d) {
-          const uint32_t gg = g - 1 - d;
-          drain_wait(&x_full[gg % kStages], (gg / kStages) & 1u);
+        // the leader's stage barriers count both CTAs' bytes: the last stages
+        // issued must have landed before either CTA exits
+        if (leader) {
+          for (uint32_t d = 0; d < kXStages && d < g; ++d) {
+            const uint32_t gg = g - 1 - d;
+            drain_wait(&x_full[gg % kXStages], (gg / kXStages) & 1u);
+          }
         }
       }
     } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
+      // ------------------------------------------------- MMA issuer (leader)
+      if (leader && lane == 0) {
         uint32_t g = 0;
         uint32_t ntile = 0;
-        for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x, ++ntile) {
-          if (ntile > 0 && !wait_bar(d_empty, (ntile - 1) & 1u, abort_flag, hdr)) break;
+        for (int t = pair; t < tiles && !*abort_flag; t += npairs, ++ntile) {
+          if (ntile > 0 && !wait_bar_cluster(d_empty, (ntile - 1) & 1u, abort_flag, hdr)) break;
           tc_fence_after();
           bool ok = true;
           for (int kb = 0; kb < KB; ++kb, ++g) {
-            const int s = g % kStages;
-            const uint32_t ph = (g / kStages) & 1u;
-            if (!wait_bar(&x_full[s], ph, abort_flag, hdr) ||
-                !wait_bar(&a_full[s], ph, abort_flag, hdr)) {
+            const int s = g % kXStages, sa = g % kAStages;
+            if (!wait_bar_cluster(&x_full[s], (g / kXStages) & 1u, abort_flag, hdr) ||
+                !wait_bar_cluster(&a_full[sa], (g / kAStages) & 1u, abort_flag, hdr)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t xaddr = smem_u32(xs + s * kXStageBytes);
-            const uint32_t a_hi = tmem + kACol + 64u * s, a_lo = a_hi + 32u;
+            const uint32_t x8addr = smem_u32(x8s + s * kX8StageBytes);
+            const uint32_t a_hi = tmem + kACol + kAStageCols * sa, a_lo = a_hi + 32u;
+            // hi pass: bf16 x bf16, 4 x K=16
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t bdesc = sw128_desc(xaddr + kk * 32);
-              mma_ts(tmem + kAccCol, a_hi + 8u * kk, bdesc, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
-              mma_ts(tmem + kAccCol, a_lo + 8u * kk, bdesc, kIdesc, 1u);
-            }
-            mma_commit(&st_free[s]);
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_pair_f16(tmem + kAccCol, a_hi + 8u * kk, sw128_desc(xaddr + kk * 32), kIdesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+            // lo pass: e4m3 remainders x e5m2 activations, 2 x K=32
+#pragma unroll
+            for (int kk = 0; kk < kBK / 32; ++kk)
+              mma_pair_f8(tmem + kAccCol, a_lo + 8u * kk, sw64_desc(x8addr + kk * 32), kIdescF8,
+                          1u);
+            mma_commit_pair(&x_free[s], 0x3);
+            mma_commit_pair(&a_free[sa], 0x3);
           }
           if (!ok) break;
-          mma_commit(d_full);
+          mma_commit_pair(d_full, 0x3);
         }
-        // drain every MMA this thread issued before TMEM is released
-        mma_commit(drain);
+        // every MMA this thread issued completes before TMEM is released
+        mma_commit_pair(drain, 0x1);
         drain_wait(drain, 0);
+      }
+    } else if (warp == 3) {
+      // -------------------------------------------- packed weights + absmax
+      // Per 4 K-steps: this CTA's 128 weight rows x 128 packed bytes (one TMA
+      // box, 128-byte swizzle) and their 4 x 128 absmax values ([block][row];
+      // cp.async, 4 bytes each: absmax rows need not be 16-byte aligned).
+      const int nquads = (KB + 3) / 4;
+      uint32_t gq = 0;   // slot ring counter
+      bool ok = true;
+      for (int t = pair; t < tiles && ok && !*abort_flag; t += npairs) {
+        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
+        const int nbase = ti.n0 + kBM * static_cast<int>(rank);   // first row within the expert
+        const int64_t row0 = static_cast<int64_t>(ti.e) * N + nbase;
+        for (int qd = 0; qd < nquads; ++qd, ++gq) {
+          const int slot = static_cast<int>(gq % kWQuads);
+          const uint32_t ph = (gq / kWQuads) & 1u;
+          if (!warp_wait_cluster(&w_free[slot], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
+          char *as = smem + kAbsOff + slot * kASlotBytes;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = lane + 32 * i;
+            const bool rv = nbase + rr < N;     // a row of this expert (else zeros)
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+              const int kb = 4 * qd + blk;
+              const bool v = rv && kb < KB;
+              const float *src = v ? absmax + (row0 + rr) * KB + kb : absmax;
+              cp_async4(smem_u32(as + blk * (kBM * 4) + rr * 4), src, v ? 4u : 0u);
+            }
+          }
+          cp_async_arrive_noinc(&w_full[slot]);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&w_full[slot], kWSlotBytes);
+            tma_load_2d(smem + kWOff + slot * kWSlotBytes, &wmap, qd * 128,
+                        static_cast<int>(row0), &w_full[slot]);
+          }
+        }
+      }
+      cp_async_wait_all();
+      if (lane == 0) {   // the last copies must land before the CTA exits
+        for (uint32_t d = 0; d < kWQuads && d < gq; ++d) {
+          const uint32_t gg = gq - 1 - d;
+          drain_wait(&w_full[gg % kWQuads], (gg / kWQuads) & 1u);
+        }
       }
     } else if (warp >= kDecodeWarp0) {
       // ---------------------------------------------------- decode + epilogue
       const int dw = warp - kDecodeWarp0;
       const int quarter = warp & 3;          // TMEM lane quarter
       const int half = dw >> 2;              // K half of the stage / token half of the tile
-      const int r = quarter * 32 + lane;     // weight row within the tile
+      const int rl = quarter * 32 + lane;                      // row within this CTA's half
+      const int r = kBM * static_cast<int>(rank) + rl;         // row within the pair tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-      const char *lut = smem + kLutOff + lane * 8;
-      uint32_t g = 0;
+      const char *lut = smem + kLutOff + lane * 4;   // entry (code c) at c * 128
+      // absmax row of this thread's weight row in pair tile t (nullptr: no such row)
+      auto row_absmax = [&](int t) -> const float * {
+        if (t >= tiles) return nullptr;
+        const TileInfo tn = tile_info(t, G, tile_start, row_off, gsize, gexp);
+        const int nn = tn.n0 + r;
+        return nn < N ? absmax + (static_cast<int64_t>(tn.e) * N + nn) * KB : nullptr;
+      };
+      // Row maximum of absmax for the row scale: for the first tile read here,
+      // for every later tile gathered one block per K-step of the tile before.
+      float mx = 0.0f;
+      if (const float *a0 = row_absmax(pair)) {
+        float m[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        int b = 0;
+        for (; b + 8 <= KB; b += 8) {   // 8 independent loads in flight
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(__ldg(a0 + b + i)));
+        }
+        for (; b < KB; ++b) m[0] = fmaxf(m[0], fabsf(__ldg(a0 + b)));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, m[i]);
+      }
+      uint32_t g = 0;    // decoded-weight stage counter
+      uint32_t gq = 0;   // packed-weight slot counter
       uint32_t ntile = 0;
-      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x, ++ntile) {
-        const TileInfo ti = tile_info(t, G, NJ, tile_start, row_off, gsize, gexp);
+      for (int t = pair; t < tiles && !*abort_flag; t += npairs, ++ntile) {
+        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
+        const float *ap_next = row_absmax(t + npairs);
+        float mx_next = 0.0f;
+        float nxq[4];   // next tile's absmax values, folded 4 K-steps after their load
+#pragma unroll
+        for (int j = 0; j < 4; ++j) nxq[j] = 0.0f;
         const int n = ti.n0 + r;
         const bool rok = n < N;
-        const int64_t wrow = static_cast<int64_t>(ti.e) * N + (rok ? n : 0);
-        const uint8_t *wp = w + wrow * row_bytes + half * 16;
-        const float *ap = absmax + wrow * KB;
-        uint4 pk = rok ? ldg128_nc(wp) : make_uint4(0u, 0u, 0u, 0u);
-        float am = rok ? __ldg(ap) : 0.0f;
+        // Row scale 2^S, S = beta + 14 with 2^beta * max(absmax of the row) in
+        // [1, 2): scaled weights stay below 2^15 and their bf16 remainders
+        // below 64, inside the e4m3 range, whatever the row's magnitude.
+        const int mexp = static_cast<int>((__float_as_uint(mx) >> 23) & 0xFFu);
+        const int beta = mx > 0.0f ? (mexp == 0 ? 126 : 127 - mexp) : 0;
+        int S = beta + kLoShift;
+        S = S > 127 ? 127 : (S < -126 ? -126 : S);
+        const float rscale = __uint_as_float(static_cast<uint32_t>(S + 127) << 23);
+        const float rinv = __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb, ++g) {
-          const int s = g % kStages;
-          const uint32_t ph = (g / kStages) & 1u;
-          // prefetch the next block's bytes before decoding this one
-          uint4 pk_n = make_uint4(0u, 0u, 0u, 0u);
-          float am_n = 0.0f;
-          if (rok && kb + 1 < KB) {
-            pk_n = ldg128_nc(wp + (kb + 1) * 32);
-            am_n = __ldg(ap + kb + 1);
+        const int nquads = (KB + 3) / 4;
+        for (int qd = 0; qd < nquads && ok; ++qd, ++gq) {
+          const int slot = static_cast<int>(gq % kWQuads);
+          if (!warp_wait_cluster(&w_full[slot], (gq / kWQuads) & 1u, abort_flag, hdr)) {
+            ok = false;
+            break;
           }
-          uint32_t hi[8 * 2], lo[8 * 2];
-          const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+          // this row's 128 packed bytes (swizzled 16-byte chunks) and 4 absmax values
+          const char *wsm = smem + kWOff + slot * kWSlotBytes + rl * 128;
+          const float *asm4 = reinterpret_cast<const float *>(smem + kAbsOff + slot * kASlotBytes) + rl;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int sub = 0; sub < 4; ++sub) {
+            const int kb = 4 * qd + sub;
+            if (kb >= KB) break;
+            const uint4 pk =
+                *reinterpret_cast<const uint4 *>(wsm + (((2 * sub + half) ^ (rl & 7)) << 4));
+            const float am = asm4[sub * kBM] * rscale;
+            // next tile's absmax, first used 4 K-steps after its load (no wait here)
+            mx_next = fmaxf(mx_next, fabsf(nxq[sub]));
+            nxq[sub] = ap_next != nullptr ? __ldg(ap_next + kb) : 0.0f;
+            const int s = g % kAStages;
+            const uint32_t ph = (g / kAStages) & 1u;
+            // hi[i]: bf16 pair of k = 32 half + 2i, 2i+1; lo[i]: e4m3 of k = 32 half + 4i .. +3
+            uint32_t hi[16], lo[8];
+            const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const uint32_t off = ((words[q] >> (8 * p)) & 0xFFu) * 256u;
-              const float2 v = *reinterpret_cast<const float2 *>(lut + off);
-              const float w0 = __fmul_rn(v.x, am), w1 = __fmul_rn(v.y, am);
-              const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
-              const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
-              const float h0 = __uint_as_float(hb << 16), h1 = __uint_as_float(hb & 0xFFFF0000u);
-              const __nv_bfloat162 l = __floats2bfloat162_rn(w0 - h0, w1 - h1);
-              hi[q * 4 + p] = hb;
-              lo[q * 4 + p] = *reinterpret_cast<const uint32_t *>(&l);
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                // codes of byte p: high nibble = even k, low nibble = odd k
+                const uint32_t c0 = (words[q] >> (8 * p + 4)) & 15u, c1 = (words[q] >> (8 * p)) & 15u;
+                const float v0 = *reinterpret_cast<const float *>(lut + c0 * 128u);
+                const float v1 = *reinterpret_cast<const float *>(lut + c1 * 128u);
+                const float w0 = __fmul_rn(v0, am), w1 = __fmul_rn(v1, am);
+                const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
+                const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
+                const float h0 = __uint_as_float(hb << 16), h1 = __uint_as_float(hb & 0xFFFF0000u);
+                // remainders (exact in fp32, below 64 in magnitude) to e4m3, RNE
+                const uint32_t l8 = __nv_cvt_float2_to_fp8x2(make_float2(w0 - h0, w1 - h1),
+                                                             __NV_SATFINITE, __NV_E4M3);
+                hi[q * 4 + p] = hb;
+                if (p & 1)
+                  lo[q * 2 + (p >> 1)] |= l8 << 16;
+                else
+                  lo[q * 2 + (p >> 1)] = l8;
+              }
             }
+            if (!warp_wait_cluster(&a_free[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t col = kACol + kAStageCols * s;
+            tmem_st16(tmem + lane_base + col + 16u * half, hi);
+            tmem_st8(tmem + lane_base + col + 32u + 8u * half, lo);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cta(&a_full[s], 0);
+            ++g;
           }
-          if (!warp_wait_bar(&st_free[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t col = kACol + 64u * s + 16u * half;
-          tmem_st16(tmem + lane_base + col, hi);
-          tmem_st16(tmem + lane_base + col + 32u, lo);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&a_full[s]);
-          pk = pk_n;
-          am = am_n;
+          // done with the slot (every lane has read its bytes)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&w_free[slot]);
         }
         if (!ok) break;
-        // ---- epilogue: accumulator -> bf16 y
-        if (!warp_wait_bar(d_full, ntile & 1u, abort_flag, hdr)) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, fabsf(nxq[j]));
+        mx = mx_next;
+        // ---- epilogue: accumulator -> bf16 y (this CTA's 128 weight rows)
+        if (!warp_wait_cluster(d_full, ntile & 1u, abort_flag, hdr)) break;
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = half * (kBN / 2); c0 < (half + 1) * (kBN / 2); c0 += 32) {
@@ -405,44 +675,94 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               if (c0 + c < ti.rows) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(acc[c]));
+                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(acc[c]) * rinv);
                 y[(ti.row0 + c0 + c) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
               }
             }
           }
         }
         tc_fence_before();
-        mbar_arrive(d_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cta(d_empty, 0);
       }
     }
   } else if (blockIdx.x == 0 && tid == 0) {
     report_error(hdr, static_cast<uint32_t>(errbits), 0);
   }
 
+  // Neither CTA leaves (or frees TMEM) while the pair's MMAs, copies or
+  // remote arrivals may still touch it.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   if (warp == 2) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
                  : "memory");
   }
 }
 
+// x8 = e5m2(x) (RNE, saturating), 16 elements per thread: the activation
+// operand of the lo pass. n16 = elements / 16.
+__global__ void __launch_bounds__(256)
+    x_to_e5m2_kernel(const uint16_t *__restrict__ x, uint8_t *__restrict__ x8, int64_t n16) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x) + 2 * i;
+    const uint4 a = __ldg(src), b = __ldg(src + 1);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t p0 = in[2 * j], p1 = in[2 * j + 1];
+      const uint32_t lo16 = __nv_cvt_float2_to_fp8x2(
+          make_float2(__uint_as_float(p0 << 16), __uint_as_float(p0 & 0xFFFF0000u)),
+          __NV_SATFINITE, __NV_E5M2);
+      const uint32_t hi16 = __nv_cvt_float2_to_fp8x2(
+          make_float2(__uint_as_float(p1 << 16), __uint_as_float(p1 & 0xFFFF0000u)),
+          __NV_SATFINITE, __NV_E5M2);
+      out[j] = lo16 | (hi16 << 16);
+    }
+    reinterpret_cast<uint4 *>(x8)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+size_t x8_bytes(int64_t M, int32_t K) {
+  return ((static_cast<size_t>(M) * static_cast<size_t>(K) + 255) / 256) * 256;
+}
+
 }  // namespace
 
+// Header, then the e5m2 copy of x.
 size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu) {
-  (void)M; (void)N; (void)K; (void)G; (void)swiglu;
-  return kWsHeaderBytes;
+  (void)N; (void)G; (void)swiglu;
+  return kWsHeaderBytes + x8_bytes(M, K);
 }
 
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (a.swiglu) return cudaErrorNotSupported;   // fused SwiGLU is decode-only for now
-  CUtensorMap xmap;
-  // activations as [M rows][K bf16], boxes of 256 rows x 64 elements
+  if (a.ws_bytes < prefill_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu)) return cudaErrorInvalidValue;
+  CUtensorMap xmap, x8map, wmap;
+  // activations as [M rows][K bf16], boxes of 128 rows x 64 elements
   if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
                             static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M),
-                            static_cast<uint64_t>(a.K) * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+                            static_cast<uint64_t>(a.K) * 2, kBK, kBNh, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // the e5m2 copy lives in the workspace after the header: [M rows][K bytes],
+  // boxes of 128 rows x 64 bytes with the 64-byte swizzle
+  uint8_t *x8 = static_cast<uint8_t *>(a.workspace) + kWsHeaderBytes;
+  if (!encode_tensor_map_2d(&x8map, CU_TENSOR_MAP_DATA_TYPE_UINT8, x8, static_cast<uint64_t>(a.K),
+                            static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kBK, kBNh,
+                            CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  // packed weights as [E*N rows][K/2 bytes], boxes of 128 rows x 128 bytes
+  // (4 K-steps) with the 128-byte swizzle
+  if (!encode_tensor_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w,
+                            static_cast<uint64_t>(a.K) / 2,
+                            static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N),
+                            static_cast<uint64_t>(a.K) / 2, 128, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
   static bool configured[64] = {false};
@@ -454,10 +774,31 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  return launch_pdl(prefill_gemm_kernel, dim3(device_sm_count()), dim3(kThreads),
-                    static_cast<size_t>(kSmemBytes), stream, xmap, a.w, a.absmax, a.sizes,
-                    a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
-                    static_cast<WsHeader *>(a.workspace));
+  const int64_t n16 = a.M * static_cast<int64_t>(a.K) / 16;
+  const int64_t want = (n16 + 255) / 256;
+  const int xblocks = static_cast<int>(want < 8 * device_sm_count() ? want : 8 * device_sm_count());
+  cudaError_t err = launch_pdl(x_to_e5m2_kernel, dim3(xblocks), dim3(256), 0, stream, a.x, x8, n16);
+  if (err != cudaSuccess) return err;
+
+  // one CTA per SM, in pairs (clusters of 2) for the 2-SM MMA
+  const int grid = device_sm_count() & ~1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, a.w, a.absmax, a.sizes,
+                            a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
+                            static_cast<WsHeader *>(a.workspace));
 }
 
 }  // namespace gnf4

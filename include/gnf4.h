@@ -158,13 +158,16 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *               the need of the kernel it runs and refuses less with
  *               GNF4_ERR_WORKSPACE_TOO_SMALL). Its first 256 bytes are the
  *               device status word: zero it once before the first use. The
- *               current kernels need nothing more.
+ *               DECODE kernel needs nothing more; PREFILL also writes an e5m2
+ *               copy of x (M*K bytes, rounded up to 256) after the header.
  *               Two calls that may run concurrently need separate workspaces.
- * Numerics: every product enters an fp32 accumulator with the weight carried
- *   as two bf16 parts (hi + lo within 2^-18 relative of its fp32 value):
- *   DECODE splits each code value and scales each 64-element block sum by
- *   absmax in fp32; PREFILL splits each fp32 weight NF4[code] * absmax and
- *   runs the tensor cores once on each part.
+ * Numerics: every product enters an fp32 accumulator. DECODE carries each
+ *   code value as two bf16 parts (hi + lo within 2^-18 relative of the fp32
+ *   table value) and scales each 64-element block sum by absmax in fp32.
+ *   PREFILL scales each weight row by a power of two, multiplies the bf16
+ *   rounding of the fp32 weight NF4[code] * absmax by bf16 x, adds the e4m3
+ *   rounding of what that rounding left times e5m2 x (at most about 2^-13 of
+ *   the product), and divides the power of two out again.
  * Alignment: x, w, y and the workspace 32-byte aligned; absmax 4-byte aligned.
  * On a device-side metadata error no output is written.
  */
