@@ -21,30 +21,38 @@
 //   learns which experts are active (no sync, graph-capturable).
 //   tile   = up to 8 consecutive units of one batch.
 //
-// Inside a CTA (warp 16 = tensor copies, warp 17 = absmax copies, warps 0-15
-// = consumers)
+// Numerics: each code value is an fp16 part hi (rounded down) plus a
+// remainder times 2^13 rounded to 3 significant bits, an fp16 whose low byte
+// is zero; together within 4.6e-5 relative of the fp32 value. Activations
+// are staged as bf16 and rewritten in place as fp16 times a power of two
+// per (row, 64-element block), which the block sum divides out in fp32.
+//
+// Inside a CTA (warp 16 = tensor copies, warp 17 = absmax copies, warp 18 =
+// activation conversion, warps 0-15 = consumers)
 //   Stage = 256 K-elements of a tile: the tile's weight rows as a few TMA
 //   boxes of 128 packed bytes per row (128-byte swizzle), the batch's
 //   activations as one box of 4 blocks x 8 rows x 64 bf16, and the 8 x 4
 //   absmax values of each row group (cp.async, 4 bytes each: absmax rows
 //   need not be 16-byte aligned).
-//   Consumer warp w decodes row group w / 8 of unit w % 8. Lane (g = lane/4,
-//   q = lane%4) reads 8 packed bytes of row g per 64-element block. Each byte
-//   (two codes) is ONE 8-byte shared-memory load from a 256-entry table
-//   replicated per lane (no bank conflicts), addressed by one byte permute;
-//   the entry holds (NF4[hi], NF4[lo]) as a bf16 pair plus the bf16 pair of
-//   the remainders, so hi + lo equals the fp32 code value to within 2^-18
-//   relative. The two halves feed an m16n8k16 bf16 MMA as adjacent
-//   A-fragment registers: A rows 0-7 carry the hi parts of the 8 weight rows
-//   and rows 8-15 their lo parts, so C rows g and g+8 sum to the exact-code
-//   dot product of weight row g. The contraction index inside a block is
-//   permuted identically for weights and activations (each lane takes 16
-//   contiguous K-elements of the block). The block's fp32 result is scaled
-//   by absmax(row, block) and accumulated in fp32. With SwiGLU the up-row
-//   warp hands its accumulators to the gate-row warp through shared memory.
+//   Consumer warp w takes 64-element block w / 4 of every stage for the two
+//   units 2 (w % 4), 2 (w % 4) + 1, so one set of activation fragments
+//   serves both. Per unit, two m16n8k16 fp16 MMAs per 16 K-elements (hi,
+//   remainder) cover all 16 weight rows: A rows g and g + 8 are the unit's
+//   row groups (with SwiGLU a gate row and its up row, which the epilogue
+//   combines in registers). For each packed byte (two codes) one byte
+//   permute forms the address of a 256-byte table row replicated per lane
+//   (no bank conflicts) holding the hi pair and, 128 bytes on, the
+//   remainder pair; for some words the remainders are instead decoded in
+//   registers by byte permutes, which moves work from the shared-memory pipe
+//   to the ALU pipe. The block's fp32 result is scaled by absmax(row, block)
+//   and the activations' 2^-S and accumulated in fp32; when a tile's K loop
+//   ends, the pair's four block warps sum their partial results through
+//   shared memory (fixed order) and the block-0 warp writes y.
 // Every wait is bounded (2 s); on expiry the kernel records
 // GNF4_DEVERR_TIMEOUT, lets the producer's copies land and returns.
 #include <climits>
+
+#include <cuda_fp16.h>
 
 #include "launch.h"
 #include "sm100.cuh"
@@ -55,7 +63,8 @@ namespace {
 constexpr int kConsumerWarps = 16;
 constexpr int kTmaWarp = kConsumerWarps;          // issues the tensor copies
 constexpr int kScaleWarp = kConsumerWarps + 1;    // copies the absmax values
-constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr int kXWarp = kConsumerWarps + 2;        // converts the staged activations to fp16
+constexpr int kThreads = (kConsumerWarps + 3) * 32;
 constexpr int kTileUnits = 8;                 // units per tile (2 row groups each)
 constexpr int kStages = 6;
 constexpr int kBatch = 8;                     // activation rows per batch (MMA N)
@@ -63,45 +72,135 @@ constexpr int kBoxBytes = 1024;               // 8 rows x 128 bytes
 constexpr int kStageBlocks = 4;               // absmax blocks per stage (256 K-elements)
 constexpr int kWStage = kTileUnits * 2 * kBoxBytes;              // 16 KB
 constexpr int kXStage = kStageBlocks * kBoxBytes;                // 4 KB
+constexpr int kXsStage = kStageBlocks * kBatch * 4;              // 128 B: 2^-S per (block, row)
 constexpr int kAStage = kTileUnits * 2 * 8 * kStageBlocks * 4;   // 2 KB
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
+constexpr float kLoInv = 1.0f / 8192.0f;      // remainders are carried times 2^13
+// Words (bit uu * 4 + i; i: 0 row g bytes 4f.., 1 row g + 8, 2 row g bytes
+// 4 (f ^ 4).., 3 row g + 8) whose remainders are decoded in registers; the
+// others read them from the table. Splits the work between the ALU pipe and
+// the shared-memory pipe.
+constexpr uint32_t kAluLoWords = 0x00u;
 
-// Dynamic shared memory layout (bytes from a 1024-aligned base).
-constexpr int kWOff = 0;
-constexpr int kXOff = kWOff + kStages * kWStage;
-constexpr int kLutOff = kXOff + kStages * kXStage;   // uint2 [256 bytes][32 lanes]
-constexpr int kLutBytes = 256 * 32 * 8;
-constexpr int kAOff = kLutOff + kLutBytes;
-constexpr int kUnitStartOff = kAOff + kStages * kAStage;      // int64 [kMaxG + 1]
-constexpr int kRowOffOff = kUnitStartOff + (kMaxG + 1) * 8;   // int32 [kMaxG]
-constexpr int kGSizeOff = kRowOffOff + kMaxG * 4;             // int32 [kMaxG]
-constexpr int kGExpOff = kGSizeOff + kMaxG * 4;               // int32 [kMaxG]
-constexpr int kXchgOff = kGExpOff + kMaxG * 4;                // float2 [kTileUnits][32]
-constexpr int kBarOff = kXchgOff + kTileUnits * 32 * 8;       // mbarriers, see kNumBars
-// full[kStages], empty[kStages], then per unit slot: xfull (up accumulators
-// written), xempty (gate warp done reading them)
-constexpr int kNumBars = 2 * kStages + 2 * kTileUnits;
+// Shared memory layout, as absolute shared-window addresses. The window
+// starts with memory the driver reserves and the static tables below; the
+// dynamic part must start in [kMinDyn, kDynBase], which the kernel checks.
+// The table sits at a multiple of 65536 so that one byte permute forms a
+// lookup's whole address.
+constexpr int kMinDyn = 1024;
+constexpr int kDynBase = 2048;
+constexpr int kWOff = kDynBase;                               // 1024-aligned (128-byte swizzle)
+constexpr int kXOff = kWOff + kStages * kWStage;              // bf16, converted in place to fp16
+constexpr int kXsOff = kXOff + kStages * kXStage;             // float [kStages][4 blocks][8 rows]
+constexpr int kRowOffOff = kXsOff + kStages * kXsStage;       // int32 [kMaxG + 1]
+constexpr int kBarOff = (kRowOffOff + (kMaxG + 1) * 4 + 7) / 8 * 8;   // mbarriers, see kNumBars
+// full[kStages] (copies landed), empty[kStages] (consumers done), xready
+// [kStages] (activations converted), then per unit pair: xfull (the three
+// partial sums written), xempty (the block-0 warp done reading them)
+constexpr int kNumBars = 3 * kStages + kTileUnits;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;              // int [8]
-constexpr int kSmemBytes = kMiscOff + 8 * 4 + 1024;           // + alignment slack
-static_assert(kBarOff % 8 == 0 && kXchgOff % 8 == 0, "8-byte aligned");
-static_assert(kSmemBytes <= 227 * 1024, "fits one CTA per SM");
+// table: 256-byte row per packed byte b: lane l's hi pair at l * 4, its
+// remainder pair at 128 + l * 4
+constexpr int kLutOff = 131072;
+constexpr int kLutBytes = 256 * 256;
+constexpr int kAOff = kLutOff + kLutBytes;
+constexpr int kXchgOff = kAOff + kStages * kAStage;           // float4 [4 pairs][3][2 units][32]
+constexpr int kXchgBytes = (kTileUnits / 2) * 3 * 2 * 32 * 16;
+constexpr int kUnitStartOff = kXchgOff + kXchgBytes;          // int64 [kMaxG + 1]
+constexpr int kGExpOff = kUnitStartOff + (kMaxG + 1) * 8;     // uint16 [kMaxG]
+constexpr int kSmemEnd = kGExpOff + kMaxG * 2;
+// dynamic bytes requested: the window reaches kSmemEnd from any start >= kMinDyn
+constexpr int kSmemBytes = kSmemEnd - kMinDyn;
+static_assert(kMiscOff + 8 * 4 <= kLutOff, "low region overlaps the table");
+static_assert(kBarOff % 8 == 0 && kXOff % 1024 == 0 && kLutOff % 65536 == 0, "alignment");
+static_assert(kSmemBytes + kDynBase - kMinDyn <= 227 * 1024, "fits one CTA per SM");
 
 // ------------------------------------------------------------------ PTX
 
 // Not volatile: the compiler may interleave independent accumulation chains.
-__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// (hi pair, lo pair) of byte p of `word`, from this lane's table slot.
-__device__ __forceinline__ uint2 lut_pair(const char *lut, uint32_t word, uint32_t lane8,
-                                          uint32_t p) {
-  const uint32_t off = __byte_perm(word, lane8, 0x5504u | (p << 4));   // byte*256 + lane*8
-  return *reinterpret_cast<const uint2 *>(lut + off);
+// D = A.B with a zero accumulator in.
+__device__ __forceinline__ void mma_f16_z(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// prmt.b32 in its default mode: result byte i = byte (sel nibble i & 7) of
+// {b, a}, or, when bit 3 of that nibble is set, that byte's sign bit
+// replicated over all 8 bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Remainder pairs of the 8 codes of `word`, in the order of lut_f16's bytes
+// 0..3. Each code's remainder NF4[c] - hi[c] (>= 0, hi rounded down) times
+// 2^13, rounded to 3 significant bits, is an fp16 whose low byte is zero;
+// t[0..3] hold the 16 high bytes (codes 4i..4i+3 in t[i]), all below 0x80.
+// A selector nibble picks its code from t[0]:t[1] and, XOR 8, from
+// t[2]:t[3]; in the half that does not hold the code, bit 3 of the nibble is
+// set and sign replication of a byte below 0x80 yields zero, so one OR
+// merges the halves.
+__device__ __forceinline__ void lo_pairs(uint32_t word, const uint32_t (&t)[4],
+                                         uint32_t (&pr)[4]) {
+  const uint32_t xw = word ^ 0x88888888u;
+  const uint32_t rl = prmt(t[0], t[1], word) | prmt(t[2], t[3], xw);               // codes of bytes 0, 1
+  const uint32_t rh = prmt(t[0], t[1], word >> 16) | prmt(t[2], t[3], xw >> 16);   // bytes 2, 3
+  // byte j of rl/rh = remainder of nibble j: (odd k, even k) per packed byte;
+  // fp16 pair = even k in the low half, odd k in the high half
+  pr[0] = prmt(rl, 0u, 0x0414u);
+  pr[1] = prmt(rl, 0u, 0x2434u);
+  pr[2] = prmt(rh, 0u, 0x0414u);
+  pr[3] = prmt(rh, 0u, 0x2434u);
+}
+
+// hi and lo fp16 pairs of the 4 packed bytes of `word` (pair p: byte p),
+// the hi pairs from this lane's slots of the table, the lo pairs from the
+// table (128 bytes further) or, with kAluLo, decoded in registers.
+// lutlane = shared address of the table (a multiple of 65536) + lane * 4, so
+// one byte permute forms the whole address table + byte * 256 + lane * 4.
+template <bool kAluLo>
+__device__ __forceinline__ void decode_word(uint32_t lutlane, uint32_t word,
+                                            const uint32_t (&lot)[4], uint32_t (&hi)[4],
+                                            uint32_t (&lo)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t a = prmt(word, lutlane, 0x7604u | (p << 4));
+    if (kAluLo) {
+      asm("ld.shared.b32 %0, [%1];" : "=r"(hi[p]) : "r"(a));
+    } else {
+      asm("ld.shared.b32 %0, [%2];\n\tld.shared.b32 %1, [%2+128];"
+          : "=r"(hi[p]), "=r"(lo[p])
+          : "r"(a));
+    }
+  }
+  if (kAluLo) lo_pairs(word, lot, lo);
+}
+
+// Bounded wait by every lane of the warp (no divergent branch); the lanes
+// agree on the answer by vote.
+__device__ __forceinline__ bool warp_wait_all(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, WsHeader *hdr) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr));
+}
+
+// One arrival on `bar` for the whole (converged) warp, by an elected lane.
+__device__ __forceinline__ void mbar_arrive_elect(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
@@ -111,14 +210,22 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
   return *reinterpret_cast<const uint16_t *>(&b);
 }
 
-// bf16 (hi, lo) split of an fp32 code value: hi = RNE(v), lo = RNE(v - hi),
-// as hi | lo << 16.
-__device__ __forceinline__ uint32_t code_split(int c) {
-  const float v = nf4_value(c);
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&h)) |
-         (static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&l)) << 16);
+// hi[c]: fp16 bits of the code value rounded toward -infinity.
+__device__ __forceinline__ uint32_t code_hi(int c) {
+  const __half h = __float2half_rd(nf4_value(c));
+  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&h));
+}
+
+// High byte of the fp16 (NF4[c] - hi[c]) * 2^13 rounded to 3 significant
+// bits (to nearest even): the remainder is exact in fp32 and >= 0, below
+// 2^-11, so the scaled value is below 4 and the byte below 0x80.
+__device__ __forceinline__ uint32_t code_lo_byte(int c) {
+  const __half h = __float2half_rd(nf4_value(c));
+  const float r = (nf4_value(c) - __half2float(h)) * 8192.0f;
+  uint32_t b = __float_as_uint(r);
+  b = (b + 0x000FFFFFu + ((b >> 21) & 1u)) & 0xFFE00000u;   // keep 2 explicit mantissa bits
+  const __half l = __float2half_rn(__uint_as_float(b));
+  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&l)) >> 8;
 }
 
 struct Problem {
@@ -139,7 +246,7 @@ struct Tile {
 // The tile that starts at unit u (never past u_hi or the end of u's batch).
 __device__ __forceinline__ Tile make_tile(int64_t u, int64_t u_hi, const Problem &p,
                                           const int64_t *unit_start, const int *row_off,
-                                          const int *gsize, const int *gexp) {
+                                          const uint16_t *gexp) {
   int lo = 0, hi = p.G;   // invariant: unit_start[lo] <= u < unit_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -155,7 +262,7 @@ __device__ __forceinline__ Tile make_tile(int64_t u, int64_t u_hi, const Problem
   t.row0 = static_cast<int64_t>(row_off[lo]) + batch * kBatch;
   t.j0 = local - batch * p.upb;
   t.nunits = static_cast<int32_t>(end - u);
-  t.mrows = min(kBatch, gsize[lo] - static_cast<int32_t>(batch) * kBatch);
+  t.mrows = min(kBatch, row_off[lo + 1] - row_off[lo] - static_cast<int32_t>(batch) * kBatch);
   t.e = gexp[lo];
   return t;
 }
@@ -188,17 +295,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const int32_t *__restrict__ sizes, const int32_t *__restrict__ expert_ids,
                        int32_t G, int64_t M, int32_t N, int32_t K, int32_t E, int32_t swiglu,
                        uint16_t *__restrict__ y, WsHeader *hdr) {
-  extern __shared__ char smem_raw[];
-  char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                        ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) char smem_raw[];
+  // generic pointer of shared-window address 0: smem + kXxxOff is region kXxx
+  const uint32_t dyn0 = smem_u32(smem_raw);
+  char *smem = smem_raw - dyn0;
+  if (dyn0 > static_cast<uint32_t>(kDynBase) || dyn0 < static_cast<uint32_t>(kMinDyn)) {
+    // the layout cannot be placed (not expected on this architecture)
+    if (blockIdx.x == 0 && threadIdx.x == 0) report_error(hdr, GNF4_DEVERR_CAPACITY, dyn0);
+    return;
+  }
   int64_t *unit_start = reinterpret_cast<int64_t *>(smem + kUnitStartOff);
   int *row_off = reinterpret_cast<int *>(smem + kRowOffOff);
-  int *gsize = reinterpret_cast<int *>(smem + kGSizeOff);
-  int *gexp = reinterpret_cast<int *>(smem + kGExpOff);
+  uint16_t *gexp = reinterpret_cast<uint16_t *>(smem + kGExpOff);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
   uint64_t *empty = full + kStages;
-  uint64_t *xfull = empty + kStages;      // [kTileUnits]
-  uint64_t *xempty = xfull + kTileUnits;  // [kTileUnits]
+  uint64_t *xready = empty + kStages;
+  uint64_t *xfull = xready + kStages;          // [kTileUnits / 2]
+  uint64_t *xempty = xfull + kTileUnits / 2;   // [kTileUnits / 2]
   int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort
   volatile int *abort_flag = &misc[1];
   __shared__ int64_t s_wsum[2][kThreads / 32];
@@ -218,9 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 32 + 1);            // 32 cp.async arrivals + the byte-count arrival
       mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&xready[s], 1);
     }
-    for (int i = 0; i < kTileUnits; ++i) {
-      mbar_init(&xfull[i], 1);
+    for (int i = 0; i < kTileUnits / 2; ++i) {
+      mbar_init(&xfull[i], 3);
       mbar_init(&xempty[i], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -228,15 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&xmap);
   }
 
-  // ---- decode table: entry byte b, lane slot l = {bf16x2 hi, bf16x2 lo} of
-  //      the pair (NF4[b >> 4], NF4[b & 15]) (low half = even k = high nibble)
+  // ---- decode table: row b, lane slot l: the fp16 pair (hi[b >> 4],
+  //      hi[b & 15]) at l * 4 and the pair of remainders at 128 + l * 4 (low
+  //      half = even k = high nibble)
   if (tid < 256) {
-    const uint32_t c0 = code_split(tid >> 4), c1 = code_split(tid & 15);
-    const uint32_t hp = (c0 & 0xFFFFu) | (c1 << 16);
-    const uint32_t lp = (c0 >> 16) | (c1 & 0xFFFF0000u);
+    const uint32_t hp = code_hi(tid >> 4) | (code_hi(tid & 15) << 16);
+    const uint32_t lp = (code_lo_byte(tid >> 4) << 8) | (code_lo_byte(tid & 15) << 24);
     uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + tid * 256);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) dst[i] = make_uint4(hp, lp, hp, lp);
+    for (int i = 0; i < 8; ++i) {
+      dst[i] = make_uint4(hp, hp, hp, hp);
+      dst[8 + i] = make_uint4(lp, lp, lp, lp);
+    }
   }
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
@@ -251,8 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e = expert_ids[g];
     if (sz < 0) bad |= GNF4_DEVERR_SIZES;
     if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
-    gsize[g] = sz;
-    gexp[g] = e;
+    gexp[g] = static_cast<uint16_t>(e);
     my_rows += max(sz, 0);
     my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
   }
@@ -278,13 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     int64_t r = wr + vr - my_rows, c = wu + vu - my_units;
     for (int g = g0; g < g1; ++g) {
-      const int sz = max(gsize[g], 0);
+      const int sz = max(sizes[g], 0);
       row_off[g] = static_cast<int>(r);
       unit_start[g] = c;
       r += sz;
       c += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
     }
-    if (tid == 0) unit_start[G] = tot_u;
+    if (tid == 0) {
+      unit_start[G] = tot_u;
+      row_off[G] = static_cast<int>(tot_r);
+    }
   }
   if (tid == 0 && tot_r != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
   __syncthreads();
@@ -297,6 +416,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t u_lo = tot_u * blockIdx.x / P;
   const int64_t u_hi = tot_u * (blockIdx.x + 1) / P;
   if (u_lo >= u_hi) return;
+
+  if (warp == kXWarp) {
+    // ------------------------------------------------ activation conversion
+    // Per stage, lane (block b = lane / 8, row r = lane % 8) rewrites its 64
+    // staged bf16 activations in place as fp16 x * 2^S, S putting the
+    // largest magnitude of those 64 in [2^14, 2^15) (0 for all zeros, Inf or
+    // NaN): exact for every value above 2^-28 of that maximum. 2^-S goes to
+    // the stage's scale table for the consumers' block sums.
+    const int b = lane >> 3, r = lane & 7;
+    uint32_t it = 0;
+    for (int64_t u = u_lo; u < u_hi;) {
+      const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
+      for (int kc = 0; kc < p.KC; ++kc, ++it) {
+        const int s = static_cast<int>(it % kStages);
+        const uint32_t ph = (it / kStages) & 1u;
+        if (!warp_wait_bar(&full[s], ph, abort_flag, hdr)) return;
+        char *row = smem + kXOff + s * kXStage + b * kBoxBytes + r * 128;
+        uint4 v[8];
+        uint32_t mx2 = 0;   // bf16 magnitudes compare as integers, two per word
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          v[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ r) << 4));
+          mx2 = __vmaxu2(mx2, v[c].x & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[c].y & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[c].z & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[c].w & 0x7FFF7FFFu);
+        }
+        const uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
+        const int eb = static_cast<int>(mx >> 7);   // biased exponent of the largest magnitude
+        int S = 0;
+        if (mx != 0 && eb < 255) S = 14 - (eb == 0 ? -126 : eb - 127);
+        S = S > 126 ? 126 : S;
+        const float sc = __uint_as_float(static_cast<uint32_t>(S + 127) << 23);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t in[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          uint32_t out[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16) * sc,
+                                                __uint_as_float(in[j] & 0xFFFF0000u) * sc);
+            out[j] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          *reinterpret_cast<uint4 *>(row + ((c ^ r) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        reinterpret_cast<float *>(smem + kXsOff + s * kXsStage)[lane] =
+            __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xready[s]);
+      }
+      u += t.nunits;
+    }
+    return;
+  }
 
   if (warp >= kTmaWarp) {
     // ------------------------------------------------------------ producers
@@ -312,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int64_t u = u_lo; u < u_hi && ok;) {
-      const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gsize, gexp);
+      const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
       const int64_t row0 = static_cast<int64_t>(t.e) * N + di * t.j0;   // first weight row
       // absmax source of this lane (row r, block blk) for each row group slot
       const int64_t arow = row0 + r;
@@ -373,101 +546,145 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // --------------------------------------------------------------- consumers
+  // Warp w takes 64-element block w / 4 of every stage for units 2 (w % 4)
+  // and 2 (w % 4) + 1 of the tile; the four block warps of a unit pair sum
+  // their partial results when the tile's K loop ends.
   const int g = lane >> 2, q = lane & 3;
-  const int ui = warp % kTileUnits;         // unit slot within the tile
-  const int rgi = warp / kTileUnits;        // row group of the unit (SwiGLU: 0 gate, 1 up)
-  const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
-  const char *lut = smem + kLutOff;
+  const int up = warp & 3;                  // unit pair
+  const int blk = warp >> 2;                // block of the stage
+  // This lane's K-elements of a block: the 8 of 16-byte activation chunk f
+  // and the 8 of chunk f ^ 4 (packed bytes 4 f .. 4 f + 3 and 4 (f ^ 4) ..),
+  // f = 0, 1, 6, 7 for q = 0..3: with the 128-byte swizzle (chunk ^ row),
+  // the packed-word reads and the activation reads are both free of bank
+  // conflicts.
+  const int f = (q & 1) | ((q & 2) ? 6 : 0);
+  const int offA = g * 128 + (((2 * blk + (f >> 2)) ^ g) << 4) + 4 * (f & 3);
+  const int offB = g * 128 + (((2 * blk + 1 - (f >> 2)) ^ g) << 4) + 4 * (f & 3);
+  const int xoffA = blk * kBoxBytes + g * 128 + ((f ^ g) << 4);
+  const int xoffB = blk * kBoxBytes + g * 128 + ((f ^ 4 ^ g) << 4);
+  const uint32_t lutlane = static_cast<uint32_t>(kLutOff) | (static_cast<uint32_t>(lane) * 4u);
+  uint32_t lot[4];   // remainder high bytes, codes 4i..4i+3 in lot[i]
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    lot[i] = code_lo_byte(4 * i) | (code_lo_byte(4 * i + 1) << 8) |
+             (code_lo_byte(4 * i + 2) << 16) | (code_lo_byte(4 * i + 3) << 24);
   const int64_t ncols = swiglu ? N / 2 : N;
-  // this warp's 8 weight rows in a stage (SwiGLU: gate rows first, up rows 8 KB on)
-  const int wslot = swiglu ? rgi * kTileUnits + ui : 2 * ui + rgi;
-  float2 *xchg = reinterpret_cast<float2 *>(smem + kXchgOff) + ui * 32;
+  // partial sums of block warp b (1..3) for unit uu of the pair
+  auto xchg_at = [&](int b, int uu) -> float4 * {
+    return reinterpret_cast<float4 *>(smem + kXchgOff) + ((up * 3 + (b - 1)) * 2 + uu) * 32 + lane;
+  };
   uint32_t it = 0, ep = 0;
   for (int64_t u = u_lo; u < u_hi;) {
-    const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gsize, gexp);
-    const bool active = ui < t.nunits;
-    const int64_t j = t.j0 + ui;
-    float acc0 = 0.0f, acc1 = 0.0f;   // weight row g, activation rows 2q and 2q+1
+    const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
+    const bool act0 = 2 * up < t.nunits, act1 = 2 * up + 1 < t.nunits;
+    // C fragment: [0] weight row g, activation row 2q; [1] row g, 2q + 1;
+    // [2] row g + 8 (SwiGLU: the matching up row), 2q; [3] row g + 8, 2q + 1
+    float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     for (int kc = 0; kc < p.KC; ++kc, ++it) {
       const int s = static_cast<int>(it % kStages);
       const uint32_t ph = (it / kStages) & 1u;
-      if (!warp_wait_bar(&full[s], ph, abort_flag, hdr)) return;
-      if (active) {
-        // 4 blocks = 4 independent accumulation chains, interleaved per k-step.
-        // Blocks past K read zero-filled weights, activations and absmax: they add 0.
-        const char *wst = smem + kWOff + s * kWStage + wslot * kBoxBytes + g * 128;
-        const char *xst = smem + kXOff + s * kXStage + g * 128;
-        const char *ast = smem + kAOff + s * kAStage + ((2 * ui + rgi) * 8 + g) * 16;
-#pragma unroll 1
-        for (int bp = 0; bp < kStageBlocks; bp += 2) {
-          uint32_t xr[2][8];
-          uint2 wd[2];
-          float am[2];
+      if (!warp_wait_all(&full[s], ph, abort_flag, hdr) ||
+          !warp_wait_all(&xready[s], ph, abort_flag, hdr))
+        return;
+      if (act0) {
+        // A block past K reads zero-filled activations and absmax: it adds 0.
+        const char *wst = smem + kWOff + s * kWStage;
+        // 2^-S of activation rows 2q and 2q + 1 in this block
+        const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + s * kXsStage)[blk * 4 + q];
+        const char *ast = smem + kAOff + s * kAStage + g * 16 + blk * 4;
+        // (rows past the batch feed only outputs that are never stored)
+        const char *xst = smem + kXOff + s * kXStage;
+        const uint4 xa = *reinterpret_cast<const uint4 *>(xst + xoffA);
+        const uint4 xb = *reinterpret_cast<const uint4 *>(xst + xoffB);
 #pragma unroll
-          for (int bb = 0; bb < 2; ++bb) {
-            const int b = bp + bb;
-            uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
-            if (g < t.mrows) {
-              xa = *reinterpret_cast<const uint4 *>(xst + b * kBoxBytes + (((2 * q) ^ g) << 4));
-              xb = *reinterpret_cast<const uint4 *>(xst + b * kBoxBytes + (((2 * q + 1) ^ g) << 4));
-            }
-            xr[bb][0] = xa.x; xr[bb][1] = xa.y; xr[bb][2] = xa.z; xr[bb][3] = xa.w;
-            xr[bb][4] = xb.x; xr[bb][5] = xb.y; xr[bb][6] = xb.z; xr[bb][7] = xb.w;
-            const int c = 2 * b + (q >> 1);
-            wd[bb] = *reinterpret_cast<const uint2 *>(wst + ((c ^ g) << 4) + 8 * (q & 1));
-            am[bb] = *reinterpret_cast<const float *>(ast + b * 4);
+        for (int uu = 0; uu < 2; ++uu) {
+          if (uu == 1 && !act1) break;
+          const int ui = 2 * up + uu;
+          // weight rows g and g + 8 of the unit (1 KB boxes of 8 rows)
+          const char *r0 = wst + (swiglu ? ui : 2 * ui) * kBoxBytes;
+          const char *r1 = wst + (swiglu ? kTileUnits + ui : 2 * ui + 1) * kBoxBytes;
+          const uint32_t wa0 = *reinterpret_cast<const uint32_t *>(r0 + offA);
+          const uint32_t wb0 = *reinterpret_cast<const uint32_t *>(r0 + offB);
+          const uint32_t wa1 = *reinterpret_cast<const uint32_t *>(r1 + offA);
+          const uint32_t wb1 = *reinterpret_cast<const uint32_t *>(r1 + offB);
+          const float am0 = *reinterpret_cast<const float *>(ast + (2 * ui) * 128);
+          const float am1 = *reinterpret_cast<const float *>(ast + (2 * ui + 1) * 128);
+          // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
+          // then (2, 3) of each word; activation registers in the same order.
+          uint32_t ha0[4], la0[4], ha1[4], la1[4], hb0[4], lb0[4], hb1[4], lb1[4];
+          if (uu == 0) {
+            decode_word<(kAluLoWords & 1u) != 0>(lutlane, wa0, lot, ha0, la0);
+            decode_word<(kAluLoWords & 2u) != 0>(lutlane, wa1, lot, ha1, la1);
+            decode_word<(kAluLoWords & 4u) != 0>(lutlane, wb0, lot, hb0, lb0);
+            decode_word<(kAluLoWords & 8u) != 0>(lutlane, wb1, lot, hb1, lb1);
+          } else {
+            decode_word<(kAluLoWords & 16u) != 0>(lutlane, wa0, lot, ha0, la0);
+            decode_word<(kAluLoWords & 32u) != 0>(lutlane, wa1, lot, ha1, la1);
+            decode_word<(kAluLoWords & 64u) != 0>(lutlane, wb0, lot, hb0, lb0);
+            decode_word<(kAluLoWords & 128u) != 0>(lutlane, wb1, lot, hb1, lb1);
           }
-          float cc[2][4];
-#pragma unroll
-          for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cc[bb][i] = 0.0f;
-#pragma unroll
-          for (int st = 0; st < 4; ++st) {
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-              const uint32_t word = st < 2 ? wd[bb].x : wd[bb].y;
-              const uint32_t pp = (st & 1) * 2;
-              const uint2 e0 = lut_pair(lut, word, lane8, pp);
-              const uint2 e1 = lut_pair(lut, word, lane8, pp + 1);
-              mma_bf16(cc[bb], e0.x, e0.y, e1.x, e1.y, xr[bb][2 * st], xr[bb][2 * st + 1]);
-            }
-          }
-#pragma unroll
-          for (int bb = 0; bb < 2; ++bb) {
-            acc0 = fmaf(cc[bb][0] + cc[bb][2], am[bb], acc0);
-            acc1 = fmaf(cc[bb][1] + cc[bb][3], am[bb], acc1);
-          }
+          float ch[4], cl[4];
+          mma_f16_z(ch, ha0[0], ha1[0], ha0[1], ha1[1], xa.x, xa.y);
+          mma_f16(ch, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);
+          mma_f16(ch, hb0[0], hb1[0], hb0[1], hb1[1], xb.x, xb.y);
+          mma_f16(ch, hb0[2], hb1[2], hb0[3], hb1[3], xb.z, xb.w);
+          mma_f16_z(cl, la0[0], la1[0], la0[1], la1[1], xa.x, xa.y);
+          mma_f16(cl, la0[2], la1[2], la0[3], la1[3], xa.z, xa.w);
+          mma_f16(cl, lb0[0], lb1[0], lb0[1], lb1[1], xb.x, xb.y);
+          mma_f16(cl, lb0[2], lb1[2], lb0[3], lb1[3], xb.z, xb.w);
+          // block sum times absmax(row) and the activation rows' 2^-S
+          acc[uu][0] = fmaf(fmaf(cl[0], kLoInv, ch[0]), am0 * xs.x, acc[uu][0]);
+          acc[uu][1] = fmaf(fmaf(cl[1], kLoInv, ch[1]), am0 * xs.y, acc[uu][1]);
+          acc[uu][2] = fmaf(fmaf(cl[2], kLoInv, ch[2]), am1 * xs.x, acc[uu][2]);
+          acc[uu][3] = fmaf(fmaf(cl[3], kLoInv, ch[3]), am1 * xs.y, acc[uu][3]);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      mbar_arrive_elect(&empty[s]);
     }
-    if (active) {
-      if (!swiglu) {
-        const int64_t col = 16 * j + 8 * rgi + g;
+    if (act0) {
+      if (blk != 0) {
+        // hand the partial sums to the pair's block-0 warp
+        if (ep > 0 && !warp_wait_bar(&xempty[up], (ep - 1) & 1u, abort_flag, hdr)) return;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int m = 2 * q + i;
-          if (m < t.mrows && col < N) y[(t.row0 + m) * ncols + col] = bf16_bits(i ? acc1 : acc0);
-        }
-      } else if (rgi == 1) {
-        // up rows: hand the accumulators to the gate warp of the same unit
-        if (ep > 0 && !warp_wait_bar(&xempty[ui], (ep - 1) & 1u, abort_flag, hdr)) return;
-        xchg[lane] = make_float2(acc0, acc1);
+        for (int uu = 0; uu < 2; ++uu)
+          *xchg_at(blk, uu) = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&xfull[ui]);
+        if (lane == 0) mbar_arrive(&xfull[up]);
       } else {
-        if (!warp_wait_bar(&xfull[ui], ep & 1u, abort_flag, hdr)) return;
-        const float2 up = xchg[lane];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xempty[ui]);
-        const int64_t col = 8 * j + g;
+        if (!warp_wait_bar(&xfull[up], ep & 1u, abort_flag, hdr)) return;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int m = 2 * q + i;
-          if (m < t.mrows && col < ncols)
-            y[(t.row0 + m) * ncols + col] = bf16_bits(silu(i ? acc1 : acc0) * (i ? up.y : up.x));
+        for (int b = 1; b < 4; ++b) {
+#pragma unroll
+          for (int uu = 0; uu < 2; ++uu) {
+            const float4 v = *xchg_at(b, uu);
+            acc[uu][0] += v.x;
+            acc[uu][1] += v.y;
+            acc[uu][2] += v.z;
+            acc[uu][3] += v.w;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xempty[up]);
+#pragma unroll
+        for (int uu = 0; uu < 2; ++uu) {
+          if (uu == 1 && !act1) break;
+          const int64_t j = t.j0 + 2 * up + uu;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int m = 2 * q + i;
+            if (m >= t.mrows) continue;
+            uint16_t *yr = y + (t.row0 + m) * ncols;
+            const float a0 = acc[uu][i], a1 = acc[uu][2 + i];
+            if (!swiglu) {
+              const int64_t c0 = 16 * j + g, c1 = 16 * j + 8 + g;
+              if (c0 < N) yr[c0] = bf16_bits(a0);
+              if (c1 < N) yr[c1] = bf16_bits(a1);
+            } else {
+              const int64_t c = 8 * j + g;
+              if (c < ncols) yr[c] = bf16_bits(silu(a0) * a1);
+            }
+          }
         }
       }
       ++ep;

@@ -136,25 +136,11 @@ __device__ __forceinline__ void mbar_arrive_cta(const uint64_t *p, uint32_t rank
                : "memory");
 }
 
-// Bounded-wait building block (arrivals may come from the peer CTA).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity);
-}
-
+// Bounded wait on a barrier of this CTA that the peer CTA may also arrive
+// on (the arrivals carry no data this wait has to acquire beyond CTA scope).
 __device__ __forceinline__ bool wait_bar_cluster(uint64_t *bar, uint32_t parity,
                                                  volatile int *abort_flag, WsHeader *hdr) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  while (true) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
-      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
-      return false;
-    }
-  }
+  return wait_bar(bar, parity, abort_flag, hdr);
 }
 
 // 2-D tensor copy into this CTA's shared memory whose byte count completes

@@ -13,6 +13,7 @@ namespace gnf4 {
 // Every wait in these kernels gives up after this long, records
 // GNF4_DEVERR_TIMEOUT and lets the kernel drain and return.
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kWaitHintNs = 100000;   // longest single suspension of a bounded wait
 
 __device__ __forceinline__ uint64_t global_timer() {
   uint64_t t;
@@ -36,8 +37,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   while (true) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    // suspended rather than spinning: a waiting warp leaves the issue slots
+    // of its scheduler to the warps that have work
+    if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
     if (*abort_flag) return false;
     if (global_timer() - t0 > kTimeoutNs) {
       *abort_flag = 1;

@@ -83,8 +83,9 @@ typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1 } gnf4_op;
 #define GNF4_DEVERR_EXPERT 0x2u     /* expert_ids[g] outside [0, E) on a non-empty group */
 #define GNF4_DEVERR_TOPK 0x4u       /* a topk id outside [0, E) */
 #define GNF4_DEVERR_TIMEOUT 0x8u    /* a bounded wait ran out */
-#define GNF4_DEVERR_CAPACITY 0x10u  /* work exceeded what the workspace was sized for
-                                       (reserved: no current kernel sets it) */
+#define GNF4_DEVERR_CAPACITY 0x10u  /* a kernel's on-chip layout did not fit what the
+                                       device provides (the decode kernel's shared
+                                       memory window; not expected on sm_100a) */
 
 /* Limits. */
 #define GNF4_MAX_EXPERTS 1024       /* E (and G) */
@@ -162,8 +163,11 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *               copy of x (M*K bytes, rounded up to 256) after the header.
  *               Two calls that may run concurrently need separate workspaces.
  * Numerics: every product enters an fp32 accumulator. DECODE carries each
- *   code value as two bf16 parts (hi + lo within 2^-18 relative of the fp32
- *   table value) and scales each 64-element block sum by absmax in fp32.
+ *   code value as an fp16 part (rounded down) plus a 3-significant-bit
+ *   remainder, together within 4.6e-5 relative of the fp32 table value, and
+ *   x per row and 64-element block scaled by a power of two into fp16 (exact
+ *   for every element above 2^-28 of that block's largest magnitude); each
+ *   block sum is scaled by absmax and the power of two in fp32.
  *   PREFILL scales each weight row by a power of two, multiplies the bf16
  *   rounding of the fp32 weight NF4[code] * absmax by bf16 x, adds the e4m3
  *   rounding of what that rounding left times e5m2 x (at most about 2^-13 of
