@@ -502,14 +502,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (it / kStages) & 1u;
         if (!warp_wait_bar(&empty[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
         if (scale_warp) {
-          char *as = smem + kAOff + s * kAStage + r * 16 + blk * 4;
+          // stage layout [unit][block][row][row group]: a consumer lane reads
+          // both row groups of its row in one 8-byte load
+          char *as = smem + kAOff + s * kAStage + (blk * 8 + r) * 8;
           const bool kok = kc * kStageBlocks + blk < p.KB;
           for (int i = 0; i < t.nunits; ++i) {
 #pragma unroll
             for (int rgi = 0; rgi < 2; ++rgi) {
               const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
               const float *src = abase + ((i * di + rgi * dr) * p.KB + kc * kStageBlocks);
-              cp_async4(smem_u32(as + (i * 2 + rgi) * 8 * 16), v ? src : absmax, v ? 4u : 0u);
+              cp_async4(smem_u32(as + i * 256 + rgi * 4), v ? src : absmax, v ? 4u : 0u);
             }
           }
           cp_async_arrive_noinc(&full[s]);
@@ -583,15 +585,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kc = 0; kc < p.KC; ++kc, ++it) {
       const int s = static_cast<int>(it % kStages);
       const uint32_t ph = (it / kStages) & 1u;
-      if (!warp_wait_all(&full[s], ph, abort_flag, hdr) ||
-          !warp_wait_all(&xready[s], ph, abort_flag, hdr))
-        return;
+      // the activation warp arrives on xready only after it has observed
+      // this stage's copies complete (full), so this one wait also orders
+      // the copied weights and absmax before the reads below
+      if (!warp_wait_all(&xready[s], ph, abort_flag, hdr)) return;
       if (act0) {
         // A block past K reads zero-filled activations and absmax: it adds 0.
         const char *wst = smem + kWOff + s * kWStage;
         // 2^-S of activation rows 2q and 2q + 1 in this block
         const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + s * kXsStage)[blk * 4 + q];
-        const char *ast = smem + kAOff + s * kAStage + g * 16 + blk * 4;
+        const char *ast = smem + kAOff + s * kAStage + (blk * 8 + g) * 8;
         // (rows past the batch feed only outputs that are never stored)
         const char *xst = smem + kXOff + s * kXStage;
         const uint4 xa = *reinterpret_cast<const uint4 *>(xst + xoffA);
@@ -607,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t wb0 = *reinterpret_cast<const uint32_t *>(r0 + offB);
           const uint32_t wa1 = *reinterpret_cast<const uint32_t *>(r1 + offA);
           const uint32_t wb1 = *reinterpret_cast<const uint32_t *>(r1 + offB);
-          const float am0 = *reinterpret_cast<const float *>(ast + (2 * ui) * 128);
-          const float am1 = *reinterpret_cast<const float *>(ast + (2 * ui + 1) * 128);
+          const float2 amv = *reinterpret_cast<const float2 *>(ast + ui * 256);
+          const float am0 = amv.x, am1 = amv.y;   // rows g and g + 8
           // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
           // then (2, 3) of each word; activation registers in the same order.
           uint32_t ha0[4], la0[4], ha1[4], la1[4], hb0[4], lb0[4], hb1[4], lb1[4];
