@@ -432,37 +432,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = static_cast<int>(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
         if (!warp_wait_bar(&full[s], ph, abort_flag, hdr)) return;
-        char *row = smem + kXOff + s * kXStage + b * kBoxBytes + r * 128;
-        uint4 v[8];
-        uint32_t mx2 = 0;   // bf16 magnitudes compare as integers, two per word
+        // rows past the batch feed only outputs that are never stored: skipped
+        if (r < t.mrows) {
+          char *row = smem + kXOff + s * kXStage + b * kBoxBytes + r * 128;
+          uint4 v[8];
+          uint32_t mx2 = 0;   // bf16 magnitudes compare as integers, two per word
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          v[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ r) << 4));
-          mx2 = __vmaxu2(mx2, v[c].x & 0x7FFF7FFFu);
-          mx2 = __vmaxu2(mx2, v[c].y & 0x7FFF7FFFu);
-          mx2 = __vmaxu2(mx2, v[c].z & 0x7FFF7FFFu);
-          mx2 = __vmaxu2(mx2, v[c].w & 0x7FFF7FFFu);
-        }
-        const uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
-        const int eb = static_cast<int>(mx >> 7);   // biased exponent of the largest magnitude
-        int S = 0;
-        if (mx != 0 && eb < 255) S = 14 - (eb == 0 ? -126 : eb - 127);
-        S = S > 126 ? 126 : S;
-        const float sc = __uint_as_float(static_cast<uint32_t>(S + 127) << 23);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t in[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          uint32_t out[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16) * sc,
-                                                __uint_as_float(in[j] & 0xFFFF0000u) * sc);
-            out[j] = *reinterpret_cast<const uint32_t *>(&h);
+          for (int c = 0; c < 8; ++c) {
+            v[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ r) << 4));
+            mx2 = __vmaxu2(mx2, v[c].x & 0x7FFF7FFFu);
+            mx2 = __vmaxu2(mx2, v[c].y & 0x7FFF7FFFu);
+            mx2 = __vmaxu2(mx2, v[c].z & 0x7FFF7FFFu);
+            mx2 = __vmaxu2(mx2, v[c].w & 0x7FFF7FFFu);
           }
-          *reinterpret_cast<uint4 *>(row + ((c ^ r) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+          const uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
+          const int eb = static_cast<int>(mx >> 7);   // biased exponent of the largest magnitude
+          int S = 0;
+          if (mx != 0 && eb < 255) S = 14 - (eb == 0 ? -126 : eb - 127);
+          S = S > 126 ? 126 : S;
+          const float sc = __uint_as_float(static_cast<uint32_t>(S + 127) << 23);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t in[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+            uint32_t out[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16) * sc,
+                                                  __uint_as_float(in[j] & 0xFFFF0000u) * sc);
+              out[j] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            *reinterpret_cast<uint4 *>(row + ((c ^ r) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+          }
+          reinterpret_cast<float *>(smem + kXsOff + s * kXsStage)[lane] =
+              __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
         }
-        reinterpret_cast<float *>(smem + kXsOff + s * kXsStage)[lane] =
-            __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
         __syncwarp();
         if (lane == 0) mbar_arrive(&xready[s]);
       }
