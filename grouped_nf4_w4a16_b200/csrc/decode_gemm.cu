@@ -253,7 +253,10 @@ __device__ __forceinline__ Tile make_tile(int64_t u, int64_t u_hi, const Problem
     if (unit_start[mid] <= u) lo = mid; else hi = mid;
   }
   const int64_t local = u - unit_start[lo];
-  const int64_t batch = local / p.upb;
+  const int64_t batch = local < (int64_t{1} << 31)
+                            ? static_cast<int64_t>(static_cast<uint32_t>(local) /
+                                                   static_cast<uint32_t>(p.upb))
+                            : local / p.upb;
   const int64_t run_end = unit_start[lo] + (batch + 1) * p.upb;
   int64_t end = u + kTileUnits;
   if (end > u_hi) end = u_hi;
@@ -369,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (sz < 0) bad |= GNF4_DEVERR_SIZES;
     if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
     gexp[g] = static_cast<uint16_t>(e);
+    row_off[g] = sz;   // kept here until the offsets are known (one global read)
     my_rows += max(sz, 0);
     my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
   }
@@ -394,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     int64_t r = wr + vr - my_rows, c = wu + vu - my_units;
     for (int g = g0; g < g1; ++g) {
-      const int sz = max(sizes[g], 0);
+      const int sz = max(row_off[g], 0);
       row_off[g] = static_cast<int>(r);
       unit_start[g] = c;
       r += sz;
@@ -412,9 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
     return;
   }
+  // this CTA's units [tot_u * b / P, tot_u * (b + 1) / P), in 32-bit
+  // arithmetic when tot_u fits (q P + r: q b + r b / P)
   const int64_t P = gridDim.x;
-  const int64_t u_lo = tot_u * blockIdx.x / P;
-  const int64_t u_hi = tot_u * (blockIdx.x + 1) / P;
+  int64_t u_lo, u_hi;
+  if (tot_u < (int64_t{1} << 31)) {
+    const uint32_t tu = static_cast<uint32_t>(tot_u), Pu = gridDim.x, bu = blockIdx.x;
+    const uint32_t q = tu / Pu, rr = tu - q * Pu;
+    u_lo = static_cast<int64_t>(q * bu + rr * bu / Pu);
+    u_hi = static_cast<int64_t>(q * (bu + 1) + rr * (bu + 1) / Pu);
+  } else {
+    u_lo = tot_u * blockIdx.x / P;
+    u_hi = tot_u * (blockIdx.x + 1) / P;
+  }
   if (u_lo >= u_hi) return;
 
   if (warp == kXWarp) {
