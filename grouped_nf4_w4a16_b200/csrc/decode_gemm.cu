@@ -21,9 +21,9 @@
 //   learns which experts are active (no sync, graph-capturable).
 //   tile   = up to 8 consecutive units of one batch.
 //
-// Numerics: each code value is an fp16 part hi (rounded down) plus a
-// remainder times 2^13 rounded to 3 significant bits, an fp16 whose low byte
-// is zero; together within 4.6e-5 relative of the fp32 value. Activations
+// Numerics: each code value is an fp16 part hi plus the fp16 of the
+// remainder times 2^13 (both round to nearest even), together within 1e-7
+// relative of the fp32 value. Activations
 // are staged as bf16 and rewritten in place as fp16 times a power of two
 // per (row, 64-element block), which the block sum divides out in fp32.
 //
@@ -42,9 +42,7 @@
 //   combines in registers). For each packed byte (two codes) one byte
 //   permute forms the address of a 256-byte table row replicated per lane
 //   (no bank conflicts) holding the hi pair and, 128 bytes on, the
-//   remainder pair; for some words the remainders are instead decoded in
-//   registers by byte permutes, which moves work from the shared-memory pipe
-//   to the ALU pipe. The block's fp32 result is scaled by absmax(row, block)
+//   remainder pair. The block's fp32 result is scaled by absmax(row, block)
 //   and the activations' 2^-S and accumulated in fp32; when a tile's K loop
 //   ends, the pair's four block warps sum their partial results through
 //   shared memory (fixed order) and the block-0 warp writes y.
@@ -76,11 +74,6 @@ constexpr int kXsStage = kStageBlocks * kBatch * 4;              // 128 B: 2^-S 
 constexpr int kAStage = kTileUnits * 2 * 8 * kStageBlocks * 4;   // 2 KB
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
 constexpr float kLoInv = 1.0f / 8192.0f;      // remainders are carried times 2^13
-// Words (bit uu * 4 + i; i: 0 row g bytes 4f.., 1 row g + 8, 2 row g bytes
-// 4 (f ^ 4).., 3 row g + 8) whose remainders are decoded in registers; the
-// others read them from the table. Splits the work between the ALU pipe and
-// the shared-memory pipe.
-constexpr uint32_t kAluLoWords = 0x00u;
 
 // Shared memory layout, as absolute shared-window addresses. The window
 // starts with memory the driver reserves and the static tables below; the
@@ -136,56 +129,26 @@ __device__ __forceinline__ void mma_f16_z(float (&c)[4], uint32_t a0, uint32_t a
 }
 
 // prmt.b32 in its default mode: result byte i = byte (sel nibble i & 7) of
-// {b, a}, or, when bit 3 of that nibble is set, that byte's sign bit
-// replicated over all 8 bits.
+// {b, a} (the selectors used here never set bit 3 of a nibble).
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
 
-// Remainder pairs of the 8 codes of `word`, in the order of lut_f16's bytes
-// 0..3. Each code's remainder NF4[c] - hi[c] (>= 0, hi rounded down) times
-// 2^13, rounded to 3 significant bits, is an fp16 whose low byte is zero;
-// t[0..3] hold the 16 high bytes (codes 4i..4i+3 in t[i]), all below 0x80.
-// A selector nibble picks its code from t[0]:t[1] and, XOR 8, from
-// t[2]:t[3]; in the half that does not hold the code, bit 3 of the nibble is
-// set and sign replication of a byte below 0x80 yields zero, so one OR
-// merges the halves.
-__device__ __forceinline__ void lo_pairs(uint32_t word, const uint32_t (&t)[4],
-                                         uint32_t (&pr)[4]) {
-  const uint32_t xw = word ^ 0x88888888u;
-  const uint32_t rl = prmt(t[0], t[1], word) | prmt(t[2], t[3], xw);               // codes of bytes 0, 1
-  const uint32_t rh = prmt(t[0], t[1], word >> 16) | prmt(t[2], t[3], xw >> 16);   // bytes 2, 3
-  // byte j of rl/rh = remainder of nibble j: (odd k, even k) per packed byte;
-  // fp16 pair = even k in the low half, odd k in the high half
-  pr[0] = prmt(rl, 0u, 0x0414u);
-  pr[1] = prmt(rl, 0u, 0x2434u);
-  pr[2] = prmt(rh, 0u, 0x0414u);
-  pr[3] = prmt(rh, 0u, 0x2434u);
-}
-
 // hi and lo fp16 pairs of the 4 packed bytes of `word` (pair p: byte p),
-// the hi pairs from this lane's slots of the table, the lo pairs from the
-// table (128 bytes further) or, with kAluLo, decoded in registers.
-// lutlane = shared address of the table (a multiple of 65536) + lane * 4, so
-// one byte permute forms the whole address table + byte * 256 + lane * 4.
-template <bool kAluLo>
-__device__ __forceinline__ void decode_word(uint32_t lutlane, uint32_t word,
-                                            const uint32_t (&lot)[4], uint32_t (&hi)[4],
+// from this lane's slots of the table: lutlane = shared address of the table
+// (a multiple of 65536) + lane * 4, so one byte permute forms the whole
+// address table + byte * 256 + lane * 4; the lo pair sits 128 bytes on.
+__device__ __forceinline__ void decode_word(uint32_t lutlane, uint32_t word, uint32_t (&hi)[4],
                                             uint32_t (&lo)[4]) {
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const uint32_t a = prmt(word, lutlane, 0x7604u | (p << 4));
-    if (kAluLo) {
-      asm("ld.shared.b32 %0, [%1];" : "=r"(hi[p]) : "r"(a));
-    } else {
-      asm("ld.shared.b32 %0, [%2];\n\tld.shared.b32 %1, [%2+128];"
-          : "=r"(hi[p]), "=r"(lo[p])
-          : "r"(a));
-    }
+    asm("ld.shared.b32 %0, [%2];\n\tld.shared.b32 %1, [%2+128];"
+        : "=r"(hi[p]), "=r"(lo[p])
+        : "r"(a));
   }
-  if (kAluLo) lo_pairs(word, lot, lo);
 }
 
 // Bounded wait by every lane of the warp (no divergent branch); the lanes
@@ -210,22 +173,19 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
   return *reinterpret_cast<const uint16_t *>(&b);
 }
 
-// hi[c]: fp16 bits of the code value rounded toward -infinity.
+// hi[c]: fp16 bits of the code value (round to nearest even).
 __device__ __forceinline__ uint32_t code_hi(int c) {
-  const __half h = __float2half_rd(nf4_value(c));
+  const __half h = __float2half_rn(nf4_value(c));
   return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&h));
 }
 
-// High byte of the fp16 (NF4[c] - hi[c]) * 2^13 rounded to 3 significant
-// bits (to nearest even): the remainder is exact in fp32 and >= 0, below
-// 2^-11, so the scaled value is below 4 and the byte below 0x80.
-__device__ __forceinline__ uint32_t code_lo_byte(int c) {
-  const __half h = __float2half_rd(nf4_value(c));
-  const float r = (nf4_value(c) - __half2float(h)) * 8192.0f;
-  uint32_t b = __float_as_uint(r);
-  b = (b + 0x000FFFFFu + ((b >> 21) & 1u)) & 0xFFE00000u;   // keep 2 explicit mantissa bits
-  const __half l = __float2half_rn(__uint_as_float(b));
-  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&l)) >> 8;
+// lo[c]: fp16 bits of (NF4[c] - hi[c]) * 2^13 (round to nearest even). The
+// remainder is exact in fp32 and at most 2^-12 in magnitude, so the scaled
+// value stays below 2; hi + lo * 2^-13 is within 1e-7 relative of NF4[c].
+__device__ __forceinline__ uint32_t code_lo(int c) {
+  const __half h = __float2half_rn(nf4_value(c));
+  const __half l = __float2half_rn((nf4_value(c) - __half2float(h)) * 8192.0f);
+  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&l));
 }
 
 struct Problem {
@@ -350,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   //      half = even k = high nibble)
   if (tid < 256) {
     const uint32_t hp = code_hi(tid >> 4) | (code_hi(tid & 15) << 16);
-    const uint32_t lp = (code_lo_byte(tid >> 4) << 8) | (code_lo_byte(tid & 15) << 24);
+    const uint32_t lp = code_lo(tid >> 4) | (code_lo(tid & 15) << 16);
     uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + tid * 256);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -582,11 +542,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int xoffA = blk * kBoxBytes + g * 128 + ((f ^ g) << 4);
   const int xoffB = blk * kBoxBytes + g * 128 + ((f ^ 4 ^ g) << 4);
   const uint32_t lutlane = static_cast<uint32_t>(kLutOff) | (static_cast<uint32_t>(lane) * 4u);
-  uint32_t lot[4];   // remainder high bytes, codes 4i..4i+3 in lot[i]
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    lot[i] = code_lo_byte(4 * i) | (code_lo_byte(4 * i + 1) << 8) |
-             (code_lo_byte(4 * i + 2) << 16) | (code_lo_byte(4 * i + 3) << 24);
   const int64_t ncols = swiglu ? N / 2 : N;
   // partial sums of block warp b (1..3) for unit uu of the pair
   auto xchg_at = [&](int b, int uu) -> float4 * {
@@ -632,17 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
           // then (2, 3) of each word; activation registers in the same order.
           uint32_t ha0[4], la0[4], ha1[4], la1[4], hb0[4], lb0[4], hb1[4], lb1[4];
-          if (uu == 0) {
-            decode_word<(kAluLoWords & 1u) != 0>(lutlane, wa0, lot, ha0, la0);
-            decode_word<(kAluLoWords & 2u) != 0>(lutlane, wa1, lot, ha1, la1);
-            decode_word<(kAluLoWords & 4u) != 0>(lutlane, wb0, lot, hb0, lb0);
-            decode_word<(kAluLoWords & 8u) != 0>(lutlane, wb1, lot, hb1, lb1);
-          } else {
-            decode_word<(kAluLoWords & 16u) != 0>(lutlane, wa0, lot, ha0, la0);
-            decode_word<(kAluLoWords & 32u) != 0>(lutlane, wa1, lot, ha1, la1);
-            decode_word<(kAluLoWords & 64u) != 0>(lutlane, wb0, lot, hb0, lb0);
-            decode_word<(kAluLoWords & 128u) != 0>(lutlane, wb1, lot, hb1, lb1);
-          }
+          decode_word(lutlane, wa0, ha0, la0);
+          decode_word(lutlane, wa1, ha1, la1);
+          decode_word(lutlane, wb0, hb0, lb0);
+          decode_word(lutlane, wb1, hb1, lb1);
           float ch[4], cl[4];
           mma_f16_z(ch, ha0[0], ha1[0], ha0[1], ha1[1], xa.x, xa.y);
           mma_f16(ch, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);

@@ -163,8 +163,8 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *               copy of x (M*K bytes, rounded up to 256) after the header.
  *               Two calls that may run concurrently need separate workspaces.
  * Numerics: every product enters an fp32 accumulator. DECODE carries each
- *   code value as an fp16 part (rounded down) plus a 3-significant-bit
- *   remainder, together within 4.6e-5 relative of the fp32 table value, and
+ *   code value as an fp16 part plus an fp16 remainder (scaled by 2^13),
+ *   together within 1e-7 relative of the fp32 table value, and
  *   x per row and 64-element block scaled by a power of two into fp16 (exact
  *   for every element above 2^-28 of that block's largest magnitude); each
  *   block sum is scaled by absmax and the power of two in fp32.
