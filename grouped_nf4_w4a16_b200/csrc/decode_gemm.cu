@@ -533,10 +533,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int blk = warp >> 2;                // block of the stage
   // This lane's K-elements of a block: the 8 of 16-byte activation chunk f
   // and the 8 of chunk f ^ 4 (packed bytes 4 f .. 4 f + 3 and 4 (f ^ 4) ..),
-  // f = 0, 1, 6, 7 for q = 0..3: with the 128-byte swizzle (chunk ^ row),
-  // the packed-word reads and the activation reads are both free of bank
-  // conflicts.
-  const int f = (q & 1) | ((q & 2) ? 6 : 0);
+  // f = 0, 5, 2, 7 for q = 0..3. With the 128-byte swizzle (chunk ^ row):
+  // f & 3 takes every value, so a warp's 4-byte packed-word reads hit 32
+  // distinct banks; and no two values of f differ only in bit 0, so the 8
+  // lanes (rows g, g + 1) that share a 16-byte activation read's wavefront
+  // hit 8 distinct chunks. Both reads run free of bank conflicts.
+  const int f = (q & 2) | ((q & 1) ? 5 : 0);
   const int offA = g * 128 + (((2 * blk + (f >> 2)) ^ g) << 4) + 4 * (f & 3);
   const int offB = g * 128 + (((2 * blk + 1 - (f >> 2)) ^ g) << 4) + 4 * (f & 3);
   const int xoffA = blk * kBoxBytes + g * 128 + ((f ^ g) << 4);
