@@ -262,9 +262,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // generic pointer of shared-window address 0: smem + kXxxOff is region kXxx
   const uint32_t dyn0 = smem_u32(smem_raw);
   char *smem = smem_raw - dyn0;
-  if (dyn0 > static_cast<uint32_t>(kDynBase) || dyn0 < static_cast<uint32_t>(kMinDyn)) {
+  // the dynamic window [dyn0, dyn0 + its size) must hold [kDynBase, kSmemEnd)
+  const uint32_t dyn_size = dynamic_smem_size();
+  if (dyn0 > static_cast<uint32_t>(kDynBase) || dyn0 + dyn_size < static_cast<uint32_t>(kSmemEnd)) {
     // the layout cannot be placed (not expected on this architecture)
-    if (blockIdx.x == 0 && threadIdx.x == 0) report_error(hdr, GNF4_DEVERR_CAPACITY, dyn0);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      hdr->reserved[60] = dyn0;
+      hdr->reserved[61] = dyn_size;
+      report_error(hdr, GNF4_DEVERR_CAPACITY, dyn0);
+    }
     return;
   }
   int64_t *unit_start = reinterpret_cast<int64_t *>(smem + kUnitStartOff);

@@ -15,6 +15,13 @@ namespace gnf4 {
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kWaitHintNs = 100000;   // longest single suspension of a bounded wait
 
+// Bytes of dynamic shared memory this CTA was launched with.
+__device__ __forceinline__ uint32_t dynamic_smem_size() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t global_timer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
