@@ -166,6 +166,76 @@ def test_decode_gemm_edge_cases(E, N, K, sizes, experts, swiglu):
     check_gemm(x, packed, absmax, sizes, experts, swiglu=swiglu, mode=gnf4.GNF4_MODE_DECODE)
 
 
+def _pow2_rows_bf16(base_bits, scales):
+    """bf16 bits of x * scales (exact: scaling a bf16 value by a power of two
+    inside the normal range only changes its exponent)."""
+    x = synth.bf16_bits_to_f32(base_bits).astype(np.float64) * scales
+    return oracle.f32_to_bf16(x.astype(np.float32))
+
+
+@pytest.mark.parametrize("swiglu,exps,spread", [
+    (False, (-120, -60, -20, 0, 20, 60, 100), 40),
+    # SwiGLU multiplies gate by up: keep both products inside bf16's normal range
+    (True, (-50, -25, 0, 25, 50), 20),
+])
+def test_decode_gemm_activation_dynamic_range(swiglu, exps, spread):
+    # The decode kernel converts activations to fp16 with one power-of-two
+    # scale per (row, 64-block). Rows whose only non-zero block sits at a
+    # scale from exps, and rows whose blocks each carry their own scale within
+    # 2^-spread .. 2^spread, must all match the oracle, each row to the
+    # tolerance taken over its own rms.
+    rng = np.random.default_rng(31)
+    E, N, K = 3, 96, 512
+    M = len(exps) + 9
+    base = synth.activations_bf16(M, K, seed=31)
+    scales = np.zeros((M, K))
+    for i, e in enumerate(exps):                 # one non-zero block per row
+        b = i % (K // 64)
+        scales[i, 64 * b:64 * b + 64] = 2.0 ** e
+    for i in range(len(exps), M):                # every block its own scale
+        for b in range(K // 64):
+            scales[i, 64 * b:64 * b + 64] = 2.0 ** int(rng.integers(-spread, spread + 1))
+    x = _pow2_rows_bf16(base, scales)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    sizes, experts = [5, 0, M - 5], [2, 0, 1]
+    yd = run_gemm(x, packed, absmax, sizes, experts, swiglu=swiglu, mode=gnf4.GNF4_MODE_DECODE)
+    y = bf16_from_dev(yd)
+    ref = oracle.grouped_gemm_f64(x, packed, absmax, sizes, experts)
+    if swiglu:
+        ref = oracle.swiglu_f64(ref)
+    assert np.isfinite(y).all()
+    for m in range(M):
+        bad = tolerance_violations(y[m], ref[m])
+        assert not bad.any(), f"row {m}: {bad.sum()} elements out of tolerance"
+
+
+def test_decode_gemm_nonfinite_rows_stay_in_their_group():
+    # A batch tile holds 8 activation rows; group 0 has 3, so rows 3..7 of
+    # its tile belong to group 1 (another expert). NaN and Inf there must not
+    # reach group 0's outputs, and all-zero rows give exact zeros.
+    rng = np.random.default_rng(32)
+    E, N, K = 2, 64, 256
+    x = synth.activations_bf16(9, K, seed=32).copy()
+    x[3] = 0x7FC0                       # NaN row (group 1)
+    x[4, :64] = 0x7F80                  # +Inf block (group 1)
+    x[5] = 0                            # all-zero row (group 1)
+    x[1] = 0                            # all-zero row (group 0)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    sizes, experts = [3, 6], [1, 0]
+    for swiglu in (False, True):
+        yd = run_gemm(x, packed, absmax, sizes, experts, swiglu=swiglu, mode=gnf4.GNF4_MODE_DECODE)
+        y = bf16_from_dev(yd)
+        ref = oracle.grouped_gemm_f64(x, packed, absmax, sizes, experts, rows=np.arange(3))
+        if swiglu:
+            ref = oracle.swiglu_f64(ref)
+        assert np.isfinite(y[:3]).all()
+        assert not tolerance_violations(y[:3], ref).any()
+        assert np.all(y[1] == 0.0) and np.all(y[5] == 0.0)
+        assert np.isnan(y[3]).all()
+
+
 def test_decode_gemm_large_groups_chunked():
     # Groups far above 8 rows go through the decode kernel in 8-row chunks.
     rng = np.random.default_rng(11)
