@@ -382,18 +382,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
     return;
   }
-  // this CTA's units [tot_u * b / P, tot_u * (b + 1) / P), in 32-bit
-  // arithmetic when tot_u fits (q P + r: q b + r b / P)
+  // Whole tiles, not units, are split across CTAs: a tile costs KC stages
+  // whatever its unit count, so a unit range cutting through a batch's tiles
+  // would cost its CTA an extra tile (twice the stages when every CTA holds
+  // about one tile). Each batch has upb units in tpb = ceil(upb / 8) tiles;
+  // this CTA takes tiles [T b / P, T (b + 1) / P) of the T = B tpb, B =
+  // tot_u / upb batches (32-bit arithmetic when T fits: q P + r gives
+  // q b + r b / P).
+  const int64_t tpb = (p.upb + kTileUnits - 1) / kTileUnits;
+  const int64_t T = (tot_u / p.upb) * tpb;
   const int64_t P = gridDim.x;
   int64_t u_lo, u_hi;
-  if (tot_u < (int64_t{1} << 31)) {
-    const uint32_t tu = static_cast<uint32_t>(tot_u), Pu = gridDim.x, bu = blockIdx.x;
-    const uint32_t q = tu / Pu, rr = tu - q * Pu;
-    u_lo = static_cast<int64_t>(q * bu + rr * bu / Pu);
-    u_hi = static_cast<int64_t>(q * (bu + 1) + rr * (bu + 1) / Pu);
+  if (T < (int64_t{1} << 31) && p.upb < (int64_t{1} << 31)) {
+    const uint32_t tt = static_cast<uint32_t>(T), Pu = gridDim.x, bu = blockIdx.x;
+    const uint32_t q = tt / Pu, rr = tt - q * Pu;
+    const uint32_t t_lo = q * bu + rr * bu / Pu, t_hi = q * (bu + 1) + rr * (bu + 1) / Pu;
+    const uint32_t tp = static_cast<uint32_t>(tpb);
+    u_lo = static_cast<int64_t>(t_lo / tp) * p.upb + static_cast<int64_t>(t_lo % tp) * kTileUnits;
+    u_hi = static_cast<int64_t>(t_hi / tp) * p.upb + static_cast<int64_t>(t_hi % tp) * kTileUnits;
   } else {
-    u_lo = tot_u * blockIdx.x / P;
-    u_hi = tot_u * (blockIdx.x + 1) / P;
+    const int64_t t_lo = T * blockIdx.x / P, t_hi = T * (blockIdx.x + 1) / P;
+    u_lo = (t_lo / tpb) * p.upb + (t_lo % tpb) * kTileUnits;
+    u_hi = (t_hi / tpb) * p.upb + (t_hi % tpb) * kTileUnits;
   }
   if (u_lo >= u_hi) return;
 
