@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *xempty = xfull + kTileUnits / 2;   // [kTileUnits / 2]
   int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort
   volatile int *abort_flag = &misc[1];
-  __shared__ int64_t s_wsum[2][kThreads / 32];
+  __shared__ int64_t s_tot;   // total units (written by warp 0 with the group table)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();
@@ -327,42 +327,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
 
-  // ---- group table from (sizes, expert_ids), validated on the device
-  const int per = (G + kThreads - 1) / kThreads;
-  const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
-  int64_t my_rows = 0, my_units = 0;
-  int bad = 0;
-  for (int g = g0; g < g1; ++g) {
-    const int sz = sizes[g];
-    const int e = expert_ids[g];
-    if (sz < 0) bad |= GNF4_DEVERR_SIZES;
-    if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
-    gexp[g] = static_cast<uint16_t>(e);
-    row_off[g] = sz;   // kept here until the offsets are known (one global read)
-    my_rows += max(sz, 0);
-    my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
-  }
-
-  __syncthreads();   // barrier init and misc visible
-  if (bad) atomicOr(&misc[0], bad);
-
-  int64_t vr = my_rows, vu = my_units;
+  // ---- group table from (sizes, expert_ids), validated on the device: built
+  //      by warp 0 alone (its lanes' loads in flight together, one warp scan),
+  //      then one block barrier publishes it with the barrier set-up.
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int64_t my_rows = 0, my_units = 0;
+    int bad = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int sz = sizes[g];
+      const int e = expert_ids[g];
+      if (sz < 0) bad |= GNF4_DEVERR_SIZES;
+      if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
+      gexp[g] = static_cast<uint16_t>(e);
+      row_off[g] = sz;   // kept here until the offsets are known
+      my_rows += max(sz, 0);
+      my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
+    }
+    int64_t vr = my_rows, vu = my_units;   // inclusive scan over the lanes
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int64_t a = __shfl_up_sync(0xffffffffu, vr, o);
-    const int64_t b = __shfl_up_sync(0xffffffffu, vu, o);
-    if (lane >= o) { vr += a; vu += b; }
-  }
-  if (lane == 31) { s_wsum[0][warp] = vr; s_wsum[1][warp] = vu; }
-  __syncthreads();
-  int64_t wr = 0, wu = 0, tot_r = 0, tot_u = 0;
-  for (int i = 0; i < kThreads / 32; ++i) {
-    if (i < warp) { wr += s_wsum[0][i]; wu += s_wsum[1][i]; }
-    tot_r += s_wsum[0][i];
-    tot_u += s_wsum[1][i];
-  }
-  {
-    int64_t r = wr + vr - my_rows, c = wu + vu - my_units;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t a = __shfl_up_sync(0xffffffffu, vr, o);
+      const int64_t b = __shfl_up_sync(0xffffffffu, vu, o);
+      if (lane >= o) { vr += a; vu += b; }
+    }
+    const int64_t tot_r = __shfl_sync(0xffffffffu, vr, 31);
+    const int64_t tot_u = __shfl_sync(0xffffffffu, vu, 31);
+    int64_t r = vr - my_rows, c = vu - my_units;
     for (int g = g0; g < g1; ++g) {
       const int sz = max(row_off[g], 0);
       row_off[g] = static_cast<int>(r);
@@ -370,13 +362,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       r += sz;
       c += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
     }
-    if (tid == 0) {
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (lane == 0) {
       unit_start[G] = tot_u;
       row_off[G] = static_cast<int>(tot_r);
+      if (tot_r != M) bad |= GNF4_DEVERR_SIZES;
+      s_tot = tot_u;
+      misc[0] = bad;
     }
   }
-  if (tid == 0 && tot_r != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
-  __syncthreads();
+  __syncthreads();   // group table, barrier set-up and misc visible
+  const int64_t tot_u = s_tot;
   const int errbits = misc[0];
   if (errbits) {
     if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
@@ -426,15 +422,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r < t.mrows) {
           char *row = smem + kXOff + s * kXStage + b * kBoxBytes + r * 128;
           uint4 v[8];
-          uint32_t mx2 = 0;   // bf16 magnitudes compare as integers, two per word
+          // bf16 magnitudes compare as integers, two per word; four
+          // independent chains keep the reduction short
+          uint32_t m4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             v[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ r) << 4));
-            mx2 = __vmaxu2(mx2, v[c].x & 0x7FFF7FFFu);
-            mx2 = __vmaxu2(mx2, v[c].y & 0x7FFF7FFFu);
-            mx2 = __vmaxu2(mx2, v[c].z & 0x7FFF7FFFu);
-            mx2 = __vmaxu2(mx2, v[c].w & 0x7FFF7FFFu);
+            m4[0] = __vmaxu2(m4[0], v[c].x & 0x7FFF7FFFu);
+            m4[1] = __vmaxu2(m4[1], v[c].y & 0x7FFF7FFFu);
+            m4[2] = __vmaxu2(m4[2], v[c].z & 0x7FFF7FFFu);
+            m4[3] = __vmaxu2(m4[3], v[c].w & 0x7FFF7FFFu);
           }
+          const uint32_t mx2 = __vmaxu2(__vmaxu2(m4[0], m4[1]), __vmaxu2(m4[2], m4[3]));
           const uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
           const int eb = static_cast<int>(mx >> 7);   // biased exponent of the largest magnitude
           int S = 0;
