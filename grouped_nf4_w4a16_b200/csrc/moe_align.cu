@@ -5,8 +5,8 @@
 // usual token->expert sort. The sort fixed here (gnf4.h documents it):
 // groups = non-empty experts in ascending id, slots ascending within a group.
 //
-// Design: a single CTA (8 warps up to 4096 slots, else 32), everything in
-// shared memory, one launch.
+// Design: up to 32 slots, one warp (below); otherwise a single CTA (8 warps
+// up to 4096 slots, else 32), everything in shared memory, one launch.
 //   1. each warp owns a contiguous segment of the S = T*top_k slots and builds
 //      its own per-expert histogram (shared-memory atomics);
 //   2. per expert, an exclusive scan over the 32 warp histograms gives each
@@ -134,6 +134,52 @@ __global__ void __launch_bounds__(NW * 32, 1)
   for (int i = s_valid + tid; i < S; i += NT) sorted_idx[i] = -1;
 }
 
+// S <= 32 (a decode step of a few tokens): one warp, slot s in lane s, no
+// shared memory and no block barrier. A slot's position is the number of
+// valid slots with a smaller expert id plus its rank among the slots of its
+// own expert (lanes found with __match_any_sync); its expert's group index is
+// the number of distinct smaller experts. Same output as the general kernel.
+__global__ void __launch_bounds__(32, 1)
+    moe_align_warp_kernel(const int32_t *__restrict__ topk, int32_t S, int32_t E,
+                          int32_t *__restrict__ sorted_idx, int32_t *__restrict__ sizes,
+                          int32_t *__restrict__ expert_ids, int32_t *__restrict__ num_groups,
+                          WsHeader *hdr) {
+  const int lane = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();   // topk may come from the previous kernel on the stream
+  const int e = lane < S ? topk[lane] : -1;
+  const bool valid = lane < S && e >= 0 && e < E;
+  if (lane < S && !valid) report_error(hdr, GNF4_DEVERR_TOPK, static_cast<uint32_t>(lane));
+  const int key = valid ? e : -1 - lane;   // invalid lanes never match each other
+  const unsigned peers = __match_any_sync(0xffffffffu, key);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const bool leader = valid && (peers & lt_mask) == 0u;   // lowest slot of its expert
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const unsigned lmask = __ballot_sync(0xffffffffu, leader);
+  int before = 0, grp = 0;   // valid slots / distinct experts with a smaller id
+  for (int j = 0; j < 32; ++j) {
+    const int ej = __shfl_sync(0xffffffffu, key, j);
+    if (((vmask >> j) & 1u) && ej < e) {
+      ++before;
+      grp += static_cast<int>((lmask >> j) & 1u);
+    }
+  }
+  if (valid) sorted_idx[before + __popc(peers & lt_mask)] = lane;
+  if (leader) {
+    sizes[grp] = __popc(peers);
+    expert_ids[grp] = e;
+  }
+  const int ngroups = __popc(lmask), nvalid = __popc(vmask);
+  for (int g = ngroups + lane; g < E; g += 32) {
+    sizes[g] = 0;
+    expert_ids[g] = -1;
+  }
+  if (lane == 0) *num_groups = ngroups;
+  // slots with an invalid id are left out; pad the tail of the permutation
+  for (int i = nvalid + lane; i < S; i += 32) sorted_idx[i] = -1;
+}
+
+constexpr int kWarpSlots = 32;    // up to this many slots: the one-warp kernel
 constexpr int kSmallWarps = 8;    // up to kSmallSlots slots
 constexpr int kLargeWarps = 32;
 constexpr int kSmallSlots = 4096;
@@ -172,6 +218,9 @@ cudaError_t launch_moe_align(const int32_t *topk, int32_t S, int32_t E, int32_t 
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
+  if (S <= kWarpSlots)
+    return launch_pdl(moe_align_warp_kernel, dim3(1), dim3(32), 0, stream, topk, S, E, sorted_idx,
+                      sizes, expert_ids, num_groups, hdr);
   if (S <= kSmallSlots) {
     const size_t smem = static_cast<size_t>(kSmallWarps + 1) * E * sizeof(int32_t);
     return launch_pdl(moe_align_kernel<kSmallWarps>, dim3(1), dim3(kSmallWarps * 32), smem, stream,
