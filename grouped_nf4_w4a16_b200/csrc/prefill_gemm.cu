@@ -97,8 +97,11 @@ constexpr int kGExpOff = kGSizeOff + kMaxG * 4;
 constexpr int kBarOff = kGExpOff + kMaxG * 4;               // mbarriers
 constexpr int kNumBars = 2 * kXStages + 2 * kAStages + 2 * kWQuads + 3;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;            // int[8]
-constexpr int kSmemBytes = kMiscOff + 8 * 4 + 1024;         // + alignment slack
+constexpr int kSmemBytes = kMiscOff + 8 * 4 + 2048;         // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "fits one CTA per SM");
+// The base is 2048-aligned and so is the table: a lookup address is the
+// lane's slot OR code * 128 (bits 7..10), with no add.
+static_assert(kLutOff % 2048 == 0, "table alignment");
 
 // ------------------------------------------------------------------ PTX
 __device__ __forceinline__ void tc_fence_before() {
@@ -301,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
                         int32_t K, int32_t E, uint16_t *__restrict__ y, WsHeader *hdr) {
   extern __shared__ char smem_raw[];
-  char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                        ~static_cast<uintptr_t>(1023));
+  char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) &
+                                        ~static_cast<uintptr_t>(2047));
   char *xs = smem + kXOff;
   char *x8s = smem + kX8Off;
   int *tile_start = reinterpret_cast<int *>(smem + kTileStartOff);
@@ -539,7 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rl = quarter * 32 + lane;                      // row within this CTA's half
       const int r = kBM * static_cast<int>(rank) + rl;         // row within the pair tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-      const char *lut = smem + kLutOff + lane * 4;   // entry (code c) at c * 128
+      // shared address of this lane's table slot (bits 7..10 clear): the
+      // entry of code c is at lut_lane | c * 128
+      const uint32_t lut_lane = smem_u32(smem + kLutOff) + static_cast<uint32_t>(lane) * 4u;
       // absmax row of this thread's weight row in pair tile t (nullptr: no such row)
       auto row_absmax = [&](int t) -> const float * {
         if (t >= tiles) return nullptr;
@@ -606,16 +611,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = g % kAStages;
             const uint32_t ph = (g / kAStages) & 1u;
             // hi[i]: bf16 pair of k = 32 half + 2i, 2i+1; lo[i]: e4m3 of k = 32 half + 4i .. +3
-            uint32_t hi[16], lo[8];
+            uint32_t hi[16], lo[8], lo_even = 0u;
             const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
               for (int p = 0; p < 4; ++p) {
-                // codes of byte p: high nibble = even k, low nibble = odd k
-                const uint32_t c0 = (words[q] >> (8 * p + 4)) & 15u, c1 = (words[q] >> (8 * p)) & 15u;
-                const float v0 = *reinterpret_cast<const float *>(lut + c0 * 128u);
-                const float v1 = *reinterpret_cast<const float *>(lut + c1 * 128u);
+                // codes of byte p: high nibble = even k, low nibble = odd k;
+                // each moved straight to bits 7..10 of its table address
+                const uint32_t w = words[q];
+                const uint32_t s0 = p == 0 ? (w << 3) : (w >> (8 * p - 3));
+                const uint32_t s1 = p == 0 ? (w << 7) : (w >> (8 * p - 7));
+                float v0, v1;
+                asm("ld.shared.f32 %0, [%1];" : "=f"(v0) : "r"(lut_lane | (s0 & 0x780u)));
+                asm("ld.shared.f32 %0, [%1];" : "=f"(v1) : "r"(lut_lane | (s1 & 0x780u)));
                 const float w0 = __fmul_rn(v0, am), w1 = __fmul_rn(v1, am);
                 const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
                 const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
@@ -625,9 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                              __NV_SATFINITE, __NV_E4M3);
                 hi[q * 4 + p] = hb;
                 if (p & 1)
-                  lo[q * 2 + (p >> 1)] |= l8 << 16;
+                  lo[q * 2 + (p >> 1)] = __byte_perm(lo_even, l8, 0x5410u);
                 else
-                  lo[q * 2 + (p >> 1)] = l8;
+                  lo_even = l8;
               }
             }
             if (!warp_wait_cluster(&a_free[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
