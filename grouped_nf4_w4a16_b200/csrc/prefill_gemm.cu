@@ -251,14 +251,6 @@ constexpr uint32_t kIdescF8 = (1u << 4) | (0u << 7) | (1u << 10) |
                               (static_cast<uint32_t>(kBN >> 3) << 17) |
                               (static_cast<uint32_t>(kPairM >> 4) << 24);
 
-__device__ __forceinline__ uint4 ldg128_nc(const void *p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
 struct TileInfo {
   int64_t row0;     // first activation row of the pair tile
   int32_t rows;     // valid activation rows (1..256)
@@ -300,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                         const __grid_constant__ CUtensorMap x8map,
                         const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ w,
-                        const float *__restrict__ absmax, const int32_t *__restrict__ sizes,
+                        const float *__restrict__ absmax, const float *__restrict__ tok_inv,
+                        const int32_t *__restrict__ sizes,
                         const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
                         int32_t K, int32_t E, uint16_t *__restrict__ y, WsHeader *hdr) {
   extern __shared__ char smem_raw[];
@@ -420,7 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int errbits = misc[0];
   const int KB = K / kBK;
   const int tiles = tot_t;
-  const int64_t row_bytes = K / 2;
 
   if (errbits == 0) {
     if (warp == 0) {
@@ -666,13 +658,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t acc[32];
           tmem_ld32(tmem + lane_base + kAccCol + c0, acc);
           tmem_wait_ld();
-          if (rok) {
+          // lane c holds 2^-s of activation row c0 + c of the tile
+          const float tinv = c0 + lane < ti.rows ? __ldg(tok_inv + ti.row0 + c0 + lane) : 0.0f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c0 + c < ti.rows) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(acc[c]) * rinv);
-                y[(ti.row0 + c0 + c) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
-              }
+          for (int c = 0; c < 32; ++c) {
+            const float tc = __shfl_sync(0xffffffffu, tinv, c);
+            if (rok && c0 + c < ti.rows) {
+              // 2^-S of the weight row, then 2^-s of the activation row
+              const float v = __uint_as_float(acc[c]) * rinv;
+              const __nv_bfloat16 b = __float2bfloat16_rn(v * tc);
+              y[(ti.row0 + c0 + c) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
             }
           }
         }
@@ -697,30 +692,96 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// x8 = e5m2(x) (RNE, saturating), 16 elements per thread: the activation
-// operand of the lo pass. n16 = elements / 16.
-__global__ void __launch_bounds__(256)
-    x_to_e5m2_kernel(const uint16_t *__restrict__ x, uint8_t *__restrict__ x8, int64_t n16) {
+// The activation operands, one block per row m of x (rows strided over the
+// grid): with s the power of two that puts the row's largest finite
+// magnitude in [2^14, 2^15) (0 for a row of zeros or with an infinity;
+// clamped to [-126, 127]),
+//   xs[m] = bf16(x[m] * 2^s)   (exact: only the exponent changes)
+//   x8[m] = e5m2(x[m] * 2^s)   (RNE, saturating)
+//   tok_inv[m] = 2^-s
+// so the remainder pass keeps e5m2's precision whatever the row's magnitude,
+// and the epilogue divides the row's scale back out. A thread keeps its
+// kPrepChunks 8-element chunks of the row in registers between the maximum
+// and the conversion (K <= 16384 with 256 threads); longer rows are read twice.
+constexpr int kPrepThreads = 256;
+constexpr int kPrepChunks = 8;
+
+__device__ __forceinline__ float bf16_abs_max2(uint32_t w) {
+  return fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xFFFF0000u)));
+}
+
+__device__ __forceinline__ void scale_chunk(const uint4 v, float f, uint4 *dst, uint2 *dst8) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o16[4], o8[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float a = __uint_as_float(w[j] << 16) * f, b = __uint_as_float(w[j] & 0xFFFF0000u) * f;
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    o16[j] = *reinterpret_cast<const uint32_t *>(&h);
+    o8[j] = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E5M2);
+  }
+  *dst = make_uint4(o16[0], o16[1], o16[2], o16[3]);
+  *dst8 = make_uint2(o8[0] | (o8[1] << 16), o8[2] | (o8[3] << 16));
+}
+
+__global__ void __launch_bounds__(kPrepThreads)
+    prefill_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
+                        uint8_t *__restrict__ x8, float *__restrict__ tok_inv, int64_t M,
+                        int32_t K) {
+  __shared__ float s_max[kPrepThreads / 32];
   pdl_trigger();
   pdl_wait();
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(x) + 2 * i;
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
-    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t out[4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c8 = K / 8;   // 8-element chunks per row
+  const bool in_regs = c8 <= kPrepThreads * kPrepChunks;
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
+    uint4 v[kPrepChunks];
+    float mx = 0.0f;
+    if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t p0 = in[2 * j], p1 = in[2 * j + 1];
-      const uint32_t lo16 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__uint_as_float(p0 << 16), __uint_as_float(p0 & 0xFFFF0000u)),
-          __NV_SATFINITE, __NV_E5M2);
-      const uint32_t hi16 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__uint_as_float(p1 << 16), __uint_as_float(p1 & 0xFFFF0000u)),
-          __NV_SATFINITE, __NV_E5M2);
-      out[j] = lo16 | (hi16 << 16);
+      for (int u = 0; u < kPrepChunks; ++u) {
+        const int i = tid + u * kPrepThreads;
+        v[u] = i < c8 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kPrepChunks; ++u)
+        mx = fmaxf(mx, fmaxf(fmaxf(bf16_abs_max2(v[u].x), bf16_abs_max2(v[u].y)),
+                             fmaxf(bf16_abs_max2(v[u].z), bf16_abs_max2(v[u].w))));
+    } else {
+      for (int i = tid; i < c8; i += kPrepThreads) {
+        const uint4 a = __ldg(src + i);
+        mx = fmaxf(mx, fmaxf(fmaxf(bf16_abs_max2(a.x), bf16_abs_max2(a.y)),
+                             fmaxf(bf16_abs_max2(a.z), bf16_abs_max2(a.w))));
+      }
     }
-    reinterpret_cast<uint4 *>(x8)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_max[warp] = mx;
+    __syncthreads();
+    mx = s_max[0];
+#pragma unroll
+    for (int w = 1; w < kPrepThreads / 32; ++w) mx = fmaxf(mx, s_max[w]);
+    __syncthreads();   // s_max is rewritten for the next row
+    const uint32_t eb = (__float_as_uint(mx) >> 23) & 0xFFu;
+    int sc = 0;
+    if (mx > 0.0f && eb != 0xFFu) sc = eb == 0 ? 127 : 14 - (static_cast<int>(eb) - 127);
+    sc = sc > 127 ? 127 : (sc < -126 ? -126 : sc);
+    const float f = __uint_as_float(static_cast<uint32_t>(sc + 127) << 23);
+    if (tid == 0)
+      tok_inv[m] = sc == 127 ? __uint_as_float(0x00400000u)   // 2^-127 (subnormal)
+                             : __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
+    uint4 *dst = reinterpret_cast<uint4 *>(xs + m * K);
+    uint2 *dst8 = reinterpret_cast<uint2 *>(x8 + m * K);
+    if (in_regs) {
+#pragma unroll
+      for (int u = 0; u < kPrepChunks; ++u) {
+        const int i = tid + u * kPrepThreads;
+        if (i < c8) scale_chunk(v[u], f, dst + i, dst8 + i);
+      }
+    } else {
+      for (int i = tid; i < c8; i += kPrepThreads) scale_chunk(__ldg(src + i), f, dst + i, dst8 + i);
+    }
   }
 }
 
@@ -728,26 +789,32 @@ size_t x8_bytes(int64_t M, int32_t K) {
   return ((static_cast<size_t>(M) * static_cast<size_t>(K) + 255) / 256) * 256;
 }
 
+size_t tok_bytes(int64_t M) { return ((static_cast<size_t>(M) * 4 + 255) / 256) * 256; }
+
 }  // namespace
 
-// Header, then the e5m2 copy of x.
+// Header, the e5m2 operand [M][K], the bf16 operand [M][K], the per-row
+// factors 2^-s [M].
 size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu) {
   (void)N; (void)G; (void)swiglu;
-  return kWsHeaderBytes + x8_bytes(M, K);
+  return kWsHeaderBytes + 3 * x8_bytes(M, K) + tok_bytes(M);
 }
 
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (a.swiglu) return cudaErrorNotSupported;   // fused SwiGLU is decode-only for now
   if (a.ws_bytes < prefill_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu)) return cudaErrorInvalidValue;
   CUtensorMap xmap, x8map, wmap;
-  // activations as [M rows][K bf16], boxes of 128 rows x 64 elements
-  if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
+  // the row-scaled operands live in the workspace after the header
+  uint8_t *x8 = static_cast<uint8_t *>(a.workspace) + kWsHeaderBytes;
+  uint16_t *xs = reinterpret_cast<uint16_t *>(x8 + x8_bytes(a.M, a.K));
+  float *tok_inv = reinterpret_cast<float *>(x8 + 3 * x8_bytes(a.M, a.K));
+  // bf16 operand as [M rows][K bf16], boxes of 128 rows x 64 elements
+  if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs,
                             static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M),
                             static_cast<uint64_t>(a.K) * 2, kBK, kBNh, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // the e5m2 copy lives in the workspace after the header: [M rows][K bytes],
-  // boxes of 128 rows x 64 bytes with the 64-byte swizzle
-  uint8_t *x8 = static_cast<uint8_t *>(a.workspace) + kWsHeaderBytes;
+  // e5m2 operand as [M rows][K bytes], boxes of 128 rows x 64 bytes with the
+  // 64-byte swizzle
   if (!encode_tensor_map_2d(&x8map, CU_TENSOR_MAP_DATA_TYPE_UINT8, x8, static_cast<uint64_t>(a.K),
                             static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kBK, kBNh,
                             CU_TENSOR_MAP_SWIZZLE_64B))
@@ -769,10 +836,11 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  const int64_t n16 = a.M * static_cast<int64_t>(a.K) / 16;
-  const int64_t want = (n16 + 255) / 256;
-  const int xblocks = static_cast<int>(want < 8 * device_sm_count() ? want : 8 * device_sm_count());
-  cudaError_t err = launch_pdl(x_to_e5m2_kernel, dim3(xblocks), dim3(256), 0, stream, a.x, x8, n16);
+  // one block per activation row (rows strided over the grid)
+  const int64_t want = a.M;   // 4 blocks of 256 threads fit an SM at 64 registers
+  const int xblocks = static_cast<int>(want < 4 * device_sm_count() ? want : 4 * device_sm_count());
+  cudaError_t err = launch_pdl(prefill_prep_kernel, dim3(xblocks), dim3(kPrepThreads), 0, stream,
+                               static_cast<const uint16_t *>(a.x), xs, x8, tok_inv, a.M, a.K);
   if (err != cudaSuccess) return err;
 
   // one CTA per SM, in pairs (clusters of 2) for the 2-SM MMA
@@ -791,7 +859,8 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, a.w, a.absmax, a.sizes,
+  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, a.w, a.absmax, tok_inv,
+                            a.sizes,
                             a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
                             static_cast<WsHeader *>(a.workspace));
 }

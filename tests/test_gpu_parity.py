@@ -310,6 +310,41 @@ def test_prefill_gemm_edge_cases(E, N, K, sizes, experts):
     check_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_PREFILL, rows=rows)
 
 
+@pytest.mark.parametrize("exps,spread", [
+    ((-120, -60, -20, 0, 20, 60, 100), 40),
+    ((-8, 0, 8, 16, 24), 6),
+])
+def test_prefill_gemm_activation_dynamic_range(exps, spread):
+    # The tensor-core kernel scales each activation row by a power of two
+    # before its bf16 and e5m2 operands are made (e5m2 alone saturates above
+    # 57344 and flushes below 2^-16). Rows whose only non-zero block sits at a
+    # scale from exps, and rows whose blocks each carry their own scale within
+    # 2^-spread .. 2^spread, must all match the oracle, each row to the
+    # tolerance taken over its own rms.
+    rng = np.random.default_rng(37)
+    E, N, K = 3, 160, 512
+    M = len(exps) + 9
+    base = synth.activations_bf16(M, K, seed=37)
+    scales = np.zeros((M, K))
+    for i, e in enumerate(exps):                 # one non-zero block per row
+        b = i % (K // 64)
+        scales[i, 64 * b:64 * b + 64] = 2.0 ** e
+    for i in range(len(exps), M):                # every block its own scale
+        for b in range(K // 64):
+            scales[i, 64 * b:64 * b + 64] = 2.0 ** int(rng.integers(-spread, spread + 1))
+    x = _pow2_rows_bf16(base, scales)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    sizes, experts = [5, 0, M - 5], [2, 0, 1]
+    yd = run_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_PREFILL)
+    y = bf16_from_dev(yd)
+    ref = oracle.grouped_gemm_f64(x, packed, absmax, sizes, experts)
+    assert np.isfinite(y).all()
+    for m in range(M):
+        bad = tolerance_violations(y[m], ref[m])
+        assert not bad.any(), f"row {m}: {bad.sum()} elements out of tolerance"
+
+
 @pytest.mark.parametrize("gi", [0, 1])
 def test_prefill_gemm_full_size_mixtral(gi):
     # Full Mixtral-8x22B-shaped GEMMs in the launch configuration the benchmark
