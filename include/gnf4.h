@@ -159,8 +159,10 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *               the need of the kernel it runs and refuses less with
  *               GNF4_ERR_WORKSPACE_TOO_SMALL). Its first 256 bytes are the
  *               device status word: zero it once before the first use. The
- *               DECODE kernel needs nothing more; PREFILL also writes an e5m2
- *               copy of x (M*K bytes, rounded up to 256) after the header.
+ *               DECODE kernel needs nothing more; PREFILL also writes, after
+ *               the header, the row-scaled operands of x: an e5m2 copy (M*K
+ *               bytes, rounded up to 256), a bf16 copy (twice that) and one
+ *               fp32 factor per row (M*4 bytes, rounded up to 256).
  *               Two calls that may run concurrently need separate workspaces.
  * Numerics: every product enters an fp32 accumulator. DECODE carries each
  *   code value as an fp16 part plus an fp16 remainder (scaled by 2^13),
@@ -168,10 +170,12 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *   x per row and 64-element block scaled by a power of two into fp16 (exact
  *   for every element above 2^-28 of that block's largest magnitude); each
  *   block sum is scaled by absmax and the power of two in fp32.
- *   PREFILL scales each weight row by a power of two, multiplies the bf16
- *   rounding of the fp32 weight NF4[code] * absmax by bf16 x, adds the e4m3
- *   rounding of what that rounding left times e5m2 x (at most about 2^-13 of
- *   the product), and divides the power of two out again.
+ *   PREFILL scales each weight row and each row of x by a power of two,
+ *   multiplies the bf16 rounding of the fp32 weight NF4[code] * absmax by the
+ *   scaled x (exact in bf16), adds the e4m3 rounding of what that rounding
+ *   left times the e5m2 rounding of the scaled x (at most about 2^-13 of the
+ *   product, whatever the magnitude of the row), and divides both powers of
+ *   two out again.
  * Alignment: x, w, y and the workspace 32-byte aligned; absmax 4-byte aligned.
  * On a device-side metadata error no output is written.
  */
