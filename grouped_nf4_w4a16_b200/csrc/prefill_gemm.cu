@@ -97,7 +97,10 @@ constexpr int kGExpOff = kGSizeOff + kMaxG * 4;
 constexpr int kBarOff = kGExpOff + kMaxG * 4;               // mbarriers
 constexpr int kNumBars = 2 * kXStages + 2 * kAStages + 2 * kWQuads + 3;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;            // int[8]
-constexpr int kSmemBytes = kMiscOff + 8 * 4 + 2048;         // + alignment slack
+// epilogue staging: per decoder warp one box of 32 tokens x 32 rows bf16
+constexpr int kOutChunkBytes = 32 * 32 * 2;
+constexpr int kOutOff = ((kMiscOff + 8 * 4 + 1023) / 1024) * 1024;
+constexpr int kSmemBytes = kOutOff + kDecodeWarps * kOutChunkBytes + 2048;   // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "fits one CTA per SM");
 // The base is 2048-aligned and so is the table: a lookup address is the
 // lane's slot OR code * 128 (bits 7..10), with no add.
@@ -155,6 +158,33 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorM
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(cluster_addr(bar, 0))
       : "memory");
+}
+
+// Bulk tensor store shared -> global of one box (c0 innermost, its byte
+// offset a multiple of 16; elements outside the tensor are not written), in
+// this thread's bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *smem_src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(smem_u32(smem_src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// none of this thread's bulk groups is still reading shared memory
+__device__ __forceinline__ void bulk_wait_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every bulk group of this thread complete (its writes done)
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// this thread's shared-memory writes visible to the bulk copy engine
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // D[tmem] (+)= A[tmem] . B[smem desc]^T over the pair: kind::f16 (bf16 x bf16).
@@ -291,11 +321,13 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t *bar, uint32_t parity
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                         const __grid_constant__ CUtensorMap x8map,
-                        const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ w,
+                        const __grid_constant__ CUtensorMap wmap,
+                        const __grid_constant__ CUtensorMap ymap, const uint8_t *__restrict__ w,
                         const float *__restrict__ absmax, const float *__restrict__ tok_inv,
                         const int32_t *__restrict__ sizes,
                         const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
-                        int32_t K, int32_t E, uint16_t *__restrict__ y, WsHeader *hdr) {
+                        int32_t K, int32_t E, uint16_t *__restrict__ y, int32_t bulk_out,
+                        WsHeader *hdr) {
   extern __shared__ char smem_raw[];
   char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) &
                                         ~static_cast<uintptr_t>(2047));
@@ -349,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&xmap);
     prefetch_tensormap(&x8map);
     prefetch_tensormap(&wmap);
+    if (bulk_out) prefetch_tensormap(&ymap);
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -650,31 +683,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, fabsf(nxq[j]));
         mx = mx_next;
-        // ---- epilogue: accumulator -> bf16 y (this CTA's 128 weight rows)
+        // ---- epilogue: accumulator -> bf16 y (this CTA's 128 weight rows).
+        // Chunks of 32 tokens: scaled and rounded into a shared-memory box
+        // [32 tokens][32 rows] and written by one bulk tensor store; a chunk
+        // that runs past the tile's tokens (the group's last tile) is stored
+        // element by element instead, so that no other group's rows are
+        // touched. The accumulator is released after its last chunk is read.
         if (!warp_wait_cluster(d_full, ntile & 1u, abort_flag, hdr)) break;
         tc_fence_after();
+        const int nbox = ti.n0 + kBM * static_cast<int>(rank) + 32 * quarter;   // first row of the box
 #pragma unroll 1
-        for (int c0 = half * (kBN / 2); c0 < (half + 1) * (kBN / 2); c0 += 32) {
+        for (int k = 0; k < 4; ++k) {
+          const int c0 = half * (kBN / 2) + 32 * k;
           uint32_t acc[32];
           tmem_ld32(tmem + lane_base + kAccCol + c0, acc);
           tmem_wait_ld();
+          if (k == 3) {   // the accumulator is read out: the next tile's MMAs may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cta(d_empty, 0);
+          }
           // lane c holds 2^-s of activation row c0 + c of the tile
           const float tinv = c0 + lane < ti.rows ? __ldg(tok_inv + ti.row0 + c0 + lane) : 0.0f;
+          if (bulk_out && c0 + 32 <= ti.rows) {
+            if (nbox >= N) continue;   // none of this warp's rows exists (nor does its box)
+            uint16_t *box = reinterpret_cast<uint16_t *>(smem + kOutOff) + dw * 1024;
+            // the previous chunk's store has read the box
+            if (lane == 0) bulk_wait_read_0();
+            __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float tc = __shfl_sync(0xffffffffu, tinv, c);
-            if (rok && c0 + c < ti.rows) {
+            for (int c = 0; c < 32; ++c) {
+              const float tc = __shfl_sync(0xffffffffu, tinv, c);
               // 2^-S of the weight row, then 2^-s of the activation row
-              const float v = __uint_as_float(acc[c]) * rinv;
-              const __nv_bfloat16 b = __float2bfloat16_rn(v * tc);
-              y[(ti.row0 + c0 + c) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+              const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(acc[c]) * rinv * tc);
+              box[c * 32 + lane] = *reinterpret_cast<const uint16_t *>(&b);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&ymap, box, nbox, static_cast<int>(ti.row0) + c0);
+              bulk_commit();
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float tc = __shfl_sync(0xffffffffu, tinv, c);
+              if (rok && c0 + c < ti.rows) {
+                const float v = __uint_as_float(acc[c]) * rinv;
+                const __nv_bfloat16 b = __float2bfloat16_rn(v * tc);
+                y[(ti.row0 + c0 + c) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+              }
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cta(d_empty, 0);
       }
+      // every bulk store of this warp has finished before the CTA exits
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   } else if (blockIdx.x == 0 && tid == 0) {
     report_error(hdr, static_cast<uint32_t>(errbits), 0);
@@ -803,7 +868,7 @@ size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (a.swiglu) return cudaErrorNotSupported;   // fused SwiGLU is decode-only for now
   if (a.ws_bytes < prefill_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu)) return cudaErrorInvalidValue;
-  CUtensorMap xmap, x8map, wmap;
+  CUtensorMap xmap, x8map, wmap, ymap;
   // the row-scaled operands live in the workspace after the header
   uint8_t *x8 = static_cast<uint8_t *>(a.workspace) + kWsHeaderBytes;
   uint16_t *xs = reinterpret_cast<uint16_t *>(x8 + x8_bytes(a.M, a.K));
@@ -819,6 +884,17 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
                             static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kBK, kBNh,
                             CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
+  // output as [M rows][N bf16], boxes of 32 rows x 32 elements, for the
+  // epilogue's bulk stores; they need rows of a multiple of 16 bytes
+  // (otherwise every output is stored element by element and the map is a
+  // placeholder the kernel does not touch)
+  const int32_t bulk_out = a.N % 8 == 0 ? 1 : 0;
+  if (bulk_out) {
+    if (!encode_tensor_map_2d(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y,
+                              static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
+                              static_cast<uint64_t>(a.N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
   // packed weights as [E*N rows][K/2 bytes], boxes of 128 rows x 128 bytes
   // (4 K-steps) with the 128-byte swizzle
   if (!encode_tensor_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w,
@@ -826,6 +902,7 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
                             static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N),
                             static_cast<uint64_t>(a.K) / 2, 128, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  if (!bulk_out) ymap = wmap;
 
   static bool configured[64] = {false};
   int dev = 0;
@@ -859,9 +936,9 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, a.w, a.absmax, tok_inv,
+  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, ymap, a.w, a.absmax, tok_inv,
                             a.sizes,
-                            a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y,
+                            a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y, bulk_out,
                             static_cast<WsHeader *>(a.workspace));
 }
 
