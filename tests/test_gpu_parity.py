@@ -281,6 +281,23 @@ def test_decode_gemm_bad_metadata_sets_error_and_writes_nothing():
         assert bool((y == 7.0).all())
 
 
+def test_prefill_gemm_bad_metadata_sets_error_and_writes_nothing():
+    rng = np.random.default_rng(13)
+    E, N, K = 3, 256, 256
+    M = 300
+    x = synth.activations_bf16(M, K, seed=13)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    for sizes, experts, bit in [([100, 100], [0, 1], "sizes"), ([150, 150], [0, 3], "expert"),
+                                ([301, -1], [0, 1], "sizes")]:
+        ws = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_GEMM, M, N, K, E, 2))
+        y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+        run_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_PREFILL, ws=ws, y=y)
+        st, bits = gnf4.gnf4_read_device_status(ws)
+        assert st == 6 and bits & gnf4.DEVERR_BITS[bit]
+        assert bool((y == 7.0).all())
+
+
 def test_host_tensors_are_refused_on_gpu_box():
     x = torch.zeros((4, 64), dtype=torch.bfloat16)
     w = torch.zeros((1, 8, 32), dtype=torch.uint8)
@@ -299,6 +316,8 @@ def test_host_tensors_are_refused_on_gpu_box():
     (2, 384, 2048, [256, 255, 257], [1, 0, 1]),        # token-tile edges
     (4, 128, 64, [1, 1000], [3, 0]),                   # one K stage, a one-row group
     (1, 136, 640, [70], [0]),                          # a single partial tile
+    (2, 100, 128, [300, 40], [1, 0]),                  # rows of y not a multiple of 16 bytes
+    (2, 264, 256, [512, 64], [0, 1]),                  # whole 32-token chunks only, N % 256 = 8
 ])
 def test_prefill_gemm_edge_cases(E, N, K, sizes, experts):
     rng = np.random.default_rng(E * 13 + N + K)
