@@ -354,11 +354,54 @@ def run_ours(args, rank, world, local_rank):
     kern_ms = [sum(v) / len(v) for v in per_kernel]   # NaN if a timestamp was missing
 
     ms = max_over_ranks(ms, world, dev)
+    glue = time_glue(prob, stream)
 
     # end to end: host (pinned) inputs -> device, the C-ABI calls, results -> host
     e2e = run_e2e(prob, stream, max(3, min(args.steps, 2000) // 10))
     e2e = (max_over_ranks(e2e[0], world, dev),) + tuple(e2e[1:])
-    return prob, ms, kern_ms, clk, e2e, launches_per_step
+    return prob, ms, kern_ms, clk, e2e, launches_per_step, glue
+
+
+def time_glue(prob, stream, reps=50):
+    """The steps either side of the GEMMs, timed outside the step: the router's
+    top-k on seeded N(0,1) logits [T, E] and the weighted combine of the last
+    GEMM's output [T*top_k, H]. CUDA events around `reps` back-to-back launches
+    after a warm-up; the inputs stay in L2 between launches (they are small)."""
+    gnf4 = prob.gnf4
+    w = prob.w
+    dev = prob.topk.device
+    rng = np.random.default_rng(1)
+    logits = torch.from_numpy(rng.standard_normal((w.T, w.E)).astype(np.float32)).to(dev)
+    ids = torch.empty((w.T, w.top_k), dtype=torch.int32, device=dev)
+    wts = torch.empty((w.T, w.top_k), dtype=torch.float32, device=dev)
+    y = prob.gemms[-1]["y"]
+    H = y.shape[1]
+    out = torch.empty((w.T, H), dtype=torch.bfloat16, device=dev)
+    ws = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_MOE_COMBINE, w.T * w.top_k), dev)
+    S = w.T * w.top_k
+    calls = {
+        "router_topk": (lambda: gnf4.gnf4_router_topk(logits, w.top_k, renormalize=True,
+                                                      topk_ids=ids, topk_weights=wts),
+                        w.T * w.E * 4 + S * 8),
+        "combine": (lambda: gnf4.gnf4_moe_combine(y, prob.sorted_idx, wts, out=out, workspace=ws),
+                    S * H * 2 + w.T * H * 2 + S * 8),
+    }
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, (fn, nbytes) in calls.items():
+            for _ in range(5):
+                fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            b.synchronize()
+            ms = a.elapsed_time(b) / reps
+            res[name] = {"ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms / 1e3) / 1e9}
+    res["how"] = (f"outside the timed step; {reps} back-to-back launches per entry point "
+                  f"(router: T x E fp32 logits; combine: T*top_k x {H} bf16 rows), inputs L2-resident")
+    return res
 
 
 def run_e2e(prob, stream, steps):
@@ -516,7 +559,7 @@ def main():
 
     import grouped_nf4_w4a16_b200 as gnf4
     gnf4.load_library()    # fails loudly if the CUDA library is missing
-    prob, ms, kern_ms, clk, e2e, lps = run_ours(args, rank, world, local_rank)
+    prob, ms, kern_ms, clk, e2e, lps, glue = run_ours(args, rank, world, local_rank)
     sec = ms / 1e3 / args.steps
     val, unit = metric_value(prob, sec, world)
     pk = peaks()
@@ -559,6 +602,7 @@ def main():
         "data": "synthetic", "config": prob.describe(),
         "roofline": roof,
         "kernels": kernels,
+        "glue": glue,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "how": "eager C-ABI calls; pinned host inputs copied in and results copied out every step"},

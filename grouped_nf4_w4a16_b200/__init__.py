@@ -18,6 +18,8 @@ from .binding import (  # noqa: F401
     GNF4_OUT_BF16,
     GNF4_OP_MOE_ALIGN,
     GNF4_OP_GROUPED_GEMM,
+    GNF4_OP_MOE_COMBINE,
+    GNF4_MAX_TOPK,
     DEVERR_BITS,
     EXPORTED_SYMBOLS,
     library_path,
@@ -28,6 +30,8 @@ from .binding import (  # noqa: F401
     gnf4_moe_align,
     gnf4_grouped_gemm,
     gnf4_grouped_gemm_noalloc,
+    gnf4_router_topk,
+    gnf4_moe_combine,
     GNF4_NOALLOC_SCRATCH_BYTES,
     gnf4_dequant_debug,
     gnf4_read_device_status,

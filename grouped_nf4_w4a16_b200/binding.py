@@ -28,14 +28,16 @@ GNF4_NOALLOC_SCRATCH_BYTES = 8 << 20
 GNF4_EPI_NONE, GNF4_EPI_SWIGLU = 0, 1
 GNF4_MODE_AUTO, GNF4_MODE_DECODE, GNF4_MODE_PREFILL = 0, 1, 2
 GNF4_OUT_F32, GNF4_OUT_BF16 = 0, 1
-GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM = 0, 1
-DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capacity": 0x10}
+GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM, GNF4_OP_MOE_COMBINE = 0, 1, 2
+GNF4_MAX_TOPK = 32
+DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capacity": 0x10,
+               "slot": 0x20}
 
 # Every symbol include/gnf4.h declares.
 EXPORTED_SYMBOLS = (
     "gnf4_moe_align", "gnf4_grouped_gemm", "gnf4_dequant_debug", "gnf4_workspace_bytes",
     "gnf4_read_device_status", "gnf4_status_string", "gnf4_version",
-    "gnf4_grouped_gemm_noalloc",
+    "gnf4_grouped_gemm_noalloc", "gnf4_router_topk", "gnf4_moe_combine",
 )
 
 _lib = None
@@ -80,6 +82,10 @@ def load_library():
     lib.gnf4_status_string.restype = ctypes.c_char_p
     lib.gnf4_version.argtypes = []
     lib.gnf4_version.restype = ctypes.c_int32
+    lib.gnf4_router_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
+    lib.gnf4_router_topk.restype = ctypes.c_int
+    lib.gnf4_moe_combine.argtypes = [P, P, P, i64, i32, i32, P, P, sz, P]
+    lib.gnf4_moe_combine.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -220,6 +226,47 @@ def gnf4_dequant_debug(w: torch.Tensor, absmax: torch.Tensor, out_dtype: int = G
     st = load_library().gnf4_dequant_debug(_ptr(w), _ptr(absmax), rows, K, blocksize, out_dtype,
                                            _ptr(out), _stream(stream))
     _check(st, "gnf4_dequant_debug")
+    return out
+
+
+def gnf4_router_topk(logits: torch.Tensor, top_k: int, *, renormalize: bool = True,
+                     topk_ids=None, topk_weights=None, stream=None):
+    """-> (topk_ids int32 [T, top_k], topk_weights fp32 [T, top_k]) from fp32 logits [T, E]."""
+    _need(logits, "logits", torch.float32)
+    T, E = logits.shape
+    dev = logits.device
+    topk_ids = topk_ids if topk_ids is not None else torch.empty((T, top_k), dtype=torch.int32,
+                                                                 device=dev)
+    topk_weights = (topk_weights if topk_weights is not None
+                    else torch.empty((T, top_k), dtype=torch.float32, device=dev))
+    st = load_library().gnf4_router_topk(_ptr(logits), T, E, top_k, 1 if renormalize else 0,
+                                         _ptr(topk_ids), _ptr(topk_weights), _stream(stream))
+    _check(st, "gnf4_router_topk")
+    return topk_ids, topk_weights
+
+
+def gnf4_moe_combine(y: torch.Tensor, sorted_idx: torch.Tensor, topk_weights: torch.Tensor, *,
+                     out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """out bf16 [T, H] = top-k weighted sum of the rows of y bf16 [T*top_k, H] (sorted order)."""
+    _need(y, "y", torch.bfloat16)
+    _need(sorted_idx, "sorted_idx", torch.int32)
+    _need(topk_weights, "topk_weights", torch.float32)
+    T, k = topk_weights.shape
+    H = y.shape[1]
+    if y.shape[0] != T * k or sorted_idx.numel() != T * k:
+        raise ValueError(f"y has {y.shape[0]} rows and sorted_idx {sorted_idx.numel()} entries; "
+                         f"expected T*top_k = {T * k}")
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    else:
+        _need(out, "out", torch.bfloat16)
+    if workspace is None:
+        workspace = make_workspace(gnf4_workspace_bytes(GNF4_OP_MOE_COMBINE, T * k), y.device)
+    st = load_library().gnf4_moe_combine(_ptr(y), _ptr(sorted_idx), _ptr(topk_weights), T, k, H,
+                                         _ptr(out), _ptr(workspace), workspace.numel(),
+                                         _stream(stream))
+    _check(st, "gnf4_moe_combine")
     return out
 
 

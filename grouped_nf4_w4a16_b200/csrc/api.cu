@@ -75,6 +75,7 @@ const char *gnf4_status_string(gnf4_status s) {
 size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t E, int32_t G) {
   (void)E;
   if (op == GNF4_OP_MOE_ALIGN) return kWsHeaderBytes;
+  if (op == GNF4_OP_MOE_COMBINE) return M < 0 ? 0 : combine_workspace_bytes(M);
   if (op != GNF4_OP_GROUPED_GEMM || M < 0 || N < 1 || K < 1 || G < 1) return 0;
   const size_t d = decode_workspace_bytes(M, N, K, G, 1);
   const size_t d2 = decode_workspace_bytes(M, N, K, G, 0);
@@ -174,6 +175,43 @@ gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t ro
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+gnf4_status gnf4_router_topk(const float *logits, int64_t T, int32_t E, int32_t top_k,
+                             int32_t renormalize, int32_t *topk_ids, float *topk_weights,
+                             gnf4_stream_t stream) {
+  if (T < 0 || E < 1 || top_k < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (renormalize != 0 && renormalize != 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (E > GNF4_MAX_EXPERTS || top_k > GNF4_MAX_TOPK || top_k > E) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (T * static_cast<int64_t>(E) >= (static_cast<int64_t>(1) << 62)) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return GNF4_OK;
+  if (!logits || !topk_ids || !topk_weights) return GNF4_ERR_INVALID_ARGUMENT;
+  if (!is_device_pointer(logits) || !is_device_pointer(topk_ids) || !is_device_pointer(topk_weights))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_weights, 4))
+    return GNF4_ERR_MISALIGNED;
+  return from_cuda(launch_router_topk(logits, T, E, top_k, renormalize, topk_ids, topk_weights,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gnf4_status gnf4_moe_combine(const uint16_t *y, const int32_t *sorted_idx,
+                             const float *topk_weights, int64_t T, int32_t top_k, int32_t H,
+                             uint16_t *out, void *workspace, size_t ws_bytes,
+                             gnf4_stream_t stream) {
+  if (T < 0 || top_k < 1 || H < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (top_k > GNF4_MAX_TOPK || T * static_cast<int64_t>(top_k) >= INT_MAX)
+    return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return GNF4_OK;
+  if (!y || !sorted_idx || !topk_weights || !out || !workspace) return GNF4_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < combine_workspace_bytes(T * top_k)) return GNF4_ERR_WORKSPACE_TOO_SMALL;
+  if (!is_device_pointer(y) || !is_device_pointer(sorted_idx) || !is_device_pointer(topk_weights) ||
+      !is_device_pointer(out) || !is_device_pointer(workspace))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(y, 2) || !aligned(out, 2) || !aligned(sorted_idx, 4) || !aligned(topk_weights, 4) ||
+      !aligned(workspace, 16))
+    return GNF4_ERR_MISALIGNED;
+  return from_cuda(launch_moe_combine(y, sorted_idx, topk_weights, T, top_k, H, out, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uint32_t *error_bits,
                                     gnf4_stream_t stream) {
   if (!workspace) return GNF4_ERR_INVALID_ARGUMENT;
@@ -188,7 +226,8 @@ gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uint32_t *er
   }
   if (e != cudaSuccess) return GNF4_ERR_CUDA;
   if (error_bits) *error_bits = h[0];
-  if (h[0] & (GNF4_DEVERR_SIZES | GNF4_DEVERR_EXPERT | GNF4_DEVERR_TOPK | GNF4_DEVERR_CAPACITY))
+  if (h[0] & (GNF4_DEVERR_SIZES | GNF4_DEVERR_EXPERT | GNF4_DEVERR_TOPK | GNF4_DEVERR_CAPACITY |
+              GNF4_DEVERR_SLOT))
     return GNF4_ERR_DEVICE_METADATA;
   if (h[0] & GNF4_DEVERR_TIMEOUT) return GNF4_ERR_TIMEOUT;
   return GNF4_OK;

@@ -49,6 +49,14 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream);
 size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu);
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream);
 
+// ---- router top-k and weighted combine (router.cu)
+size_t combine_workspace_bytes(int64_t S);
+cudaError_t launch_router_topk(const float *logits, int64_t T, int32_t E, int32_t k, int32_t renorm,
+                               int32_t *ids, float *weights, cudaStream_t stream);
+cudaError_t launch_moe_combine(const uint16_t *y, const int32_t *sorted_idx, const float *w,
+                               int64_t T, int32_t k, int32_t H, uint16_t *out, void *workspace,
+                               cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

@@ -76,7 +76,7 @@ typedef enum {
 typedef enum { GNF4_EPI_NONE = 0, GNF4_EPI_SWIGLU = 1 } gnf4_epilogue;
 typedef enum { GNF4_MODE_AUTO = 0, GNF4_MODE_DECODE = 1, GNF4_MODE_PREFILL = 2 } gnf4_mode;
 typedef enum { GNF4_OUT_F32 = 0, GNF4_OUT_BF16 = 1 } gnf4_out_dtype;
-typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1 } gnf4_op;
+typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1, GNF4_OP_MOE_COMBINE = 2 } gnf4_op;
 
 /* Bits of the device error word (gnf4_read_device_status). */
 #define GNF4_DEVERR_SIZES 0x1u      /* a size < 0, or sum(sizes) != M */
@@ -86,10 +86,13 @@ typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1 } gnf4_op;
 #define GNF4_DEVERR_CAPACITY 0x10u  /* a kernel's on-chip layout did not fit what the
                                        device provides (the decode kernel's shared
                                        memory window; not expected on sm_100a) */
+#define GNF4_DEVERR_SLOT 0x20u      /* (moe_combine) a sorted_idx entry outside
+                                       [-1, T*top_k) */
 
 /* Limits. */
 #define GNF4_MAX_EXPERTS 1024       /* E (and G) */
 #define GNF4_BLOCKSIZE 64           /* the only absmax block size */
+#define GNF4_MAX_TOPK 32            /* top_k of gnf4_router_topk */
 
 /*
  * gnf4_moe_align -- the token->expert sort that produces (sizes, expert_ids).
@@ -205,9 +208,64 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
                                gnf4_stream_t stream);
 
 /*
+ * gnf4_router_topk -- the router's choice of experts per token, the input of
+ * gnf4_moe_align.
+ *
+ * Passage: package page "grouped-nf4-gemm", "Owns" (the decode glue around the
+ * grouped GEMM, router top-k among it). The pages fix no formula; this
+ * library takes the usual softmax router: per token t, the top_k experts with
+ * the largest logits (equal logits: lower expert id first; a NaN logit ranks
+ * as -inf) in descending order, and their softmax weights
+ *   renormalize == 0: exp(l_e - l_max) / sum over all E experts
+ *   renormalize == 1: exp(l_e - l_max) / sum over the top_k selected experts
+ * computed in fp32 (weights within about 1e-6 relative of the exact values;
+ * weights are unspecified if a logit is infinite or every logit is NaN).
+ *
+ *   logits        device fp32 [T][E], 4-byte aligned
+ *   T >= 0, 1 <= E <= GNF4_MAX_EXPERTS, 1 <= top_k <= min(E, GNF4_MAX_TOPK)
+ *   topk_ids      device int32 [T][top_k] (written)
+ *   topk_weights  device fp32 [T][top_k] (written)
+ * One kernel launch, no workspace.
+ */
+GNF4_API gnf4_status gnf4_router_topk(const float *logits, int64_t T, int32_t E, int32_t top_k,
+                                      int32_t renormalize, int32_t *topk_ids, float *topk_weights,
+                                      gnf4_stream_t stream);
+
+/*
+ * gnf4_moe_combine -- the top-k weighted combine after the down projection:
+ *   out[t][h] = bf16( sum_{j < top_k} topk_weights[t][j] * y[p(t*top_k + j)][h] )
+ * where p(s) is the row of y that holds slot s (the position of s in
+ * sorted_idx), summed in fp32 with j ascending and rounded once (RNE).
+ *
+ * Passage: package page "grouped-nf4-gemm", "Owns" (the weighted combine of
+ * the decode glue).
+ *
+ *   y             device bf16 [T*top_k][H]: row i is the down-projection output
+ *                 of slot sorted_idx[i] (the grouped GEMM's row order)
+ *   sorted_idx    device int32 [T*top_k] from gnf4_moe_align; entries of -1
+ *                 (slots left out) contribute nothing; an entry outside
+ *                 [-1, T*top_k) sets GNF4_DEVERR_SLOT and is skipped;
+ *                 a slot listed twice is the caller's error (one row wins)
+ *   topk_weights  device fp32 [T][top_k]
+ *   T >= 0, 1 <= top_k <= GNF4_MAX_TOPK, H >= 1, T*top_k < 2^31
+ *   out           device bf16 [T][H] (written); must not overlap y
+ *   workspace     device, >= gnf4_workspace_bytes(GNF4_OP_MOE_COMBINE, T*top_k, ...)
+ *                 bytes (header, then the inverse of sorted_idx); its first 256
+ *                 bytes are the device status word, zero-filled once.
+ * Alignment: y, out 2-byte aligned (16-byte aligned rows, H % 8 == 0, take the
+ * vectorised path); sorted_idx, topk_weights 4-byte aligned; workspace 16-byte.
+ * Two kernel launches.
+ */
+GNF4_API gnf4_status gnf4_moe_combine(const uint16_t *y, const int32_t *sorted_idx,
+                                      const float *topk_weights, int64_t T, int32_t top_k,
+                                      int32_t H, uint16_t *out, void *workspace, size_t ws_bytes,
+                                      gnf4_stream_t stream);
+
+/*
  * gnf4_workspace_bytes -- workspace size for an op and problem size (no GPU
  * work; queries the current device's SM count once). For GNF4_OP_MOE_ALIGN
- * only E matters; for GNF4_OP_GROUPED_GEMM the size covers every mode.
+ * only E matters; for GNF4_OP_GROUPED_GEMM the size covers every mode; for
+ * GNF4_OP_MOE_COMBINE, M is T*top_k and nothing else matters.
  */
 GNF4_API size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t E, int32_t G);
 

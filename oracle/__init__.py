@@ -23,6 +23,9 @@ grouped_nf4_gemm 0.1.0, opening section, unless stated):
   "grouped-nf4-gemm", "Owns": the decode glue includes swiglu).
 * :func:`baseline_bf16` -- dequantise-to-bf16 then fp32-accumulated matmul,
   the fidelity comparator of the page's "The claim" section.
+* :func:`router_topk` / :func:`moe_combine` -- the router's top-k with softmax
+  weights, and the top-k weighted combine after the down projection (package
+  page "grouped-nf4-gemm", "Owns": the decode glue around the grouped GEMM).
 """
 from __future__ import annotations
 
@@ -46,7 +49,7 @@ class OracleError(RuntimeError):
 
 
 _STATUS = {1: "bad shape", 2: "sizes do not sum to M (or negative)", 3: "expert id out of range",
-           4: "topk id out of range"}
+           4: "topk id out of range", 5: "sorted_idx entry out of range"}
 
 
 def build(force: bool = False) -> str:
@@ -75,9 +78,11 @@ def _load():
         lib.oracle_grouped_gemm_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
         lib.oracle_swiglu_f64.argtypes = [P, i64, i32, P]
         lib.oracle_baseline_bf16.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
+        lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, P, P]
+        lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i32, P]
         for name in ("oracle_quantize_nf4", "oracle_dequant_f32", "oracle_dequant_bf16",
                      "oracle_moe_align", "oracle_grouped_gemm_f64", "oracle_swiglu_f64",
-                     "oracle_baseline_bf16"):
+                     "oracle_baseline_bf16", "oracle_router_topk", "oracle_moe_combine"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -217,3 +222,28 @@ def quantized_stack(E: int, N: int, K: int, weights_fn) -> Tuple[np.ndarray, np.
     for e in range(E):
         packed[e], absmax[e] = quantize_nf4(weights_fn(e))
     return packed, absmax
+
+
+def router_topk(logits: np.ndarray, k: int, renormalize: bool):
+    """-> (topk_ids int32 [T, k], weights fp64 [T, k]) for fp32 logits [T, E]."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    ids = np.empty((T, k), dtype=np.int32)
+    wts = np.empty((T, k), dtype=np.float64)
+    _check(_load().oracle_router_topk(_p(logits), T, E, k, 1 if renormalize else 0, _p(ids),
+                                      _p(wts)))
+    return ids, wts
+
+
+def moe_combine(y: np.ndarray, sorted_idx: np.ndarray, weights: np.ndarray) -> np.ndarray:
+    """out fp64 [T, H] from y bf16 bits [T*k, H] (sorted order), sorted_idx [T*k], weights fp32 [T, k]."""
+    y = np.ascontiguousarray(y, dtype=np.uint16)
+    sorted_idx = np.ascontiguousarray(sorted_idx, dtype=np.int32)
+    weights = np.ascontiguousarray(weights, dtype=np.float32)
+    T, k = weights.shape
+    H = y.shape[1]
+    if y.shape[0] != T * k or sorted_idx.size != T * k:
+        raise OracleError("bad shape")
+    out = np.empty((T, H), dtype=np.float64)
+    _check(_load().oracle_moe_combine(_p(y), _p(sorted_idx), _p(weights), T, k, H, _p(out)))
+    return out

@@ -53,7 +53,8 @@
 #define GNF4O_BLOCK 64
 
 /* Status codes returned by the oracle (0 = ok). */
-enum { ORC_OK = 0, ORC_BAD_SHAPE = 1, ORC_BAD_SIZES = 2, ORC_BAD_EXPERT = 3, ORC_BAD_TOPK = 4 };
+enum { ORC_OK = 0, ORC_BAD_SHAPE = 1, ORC_BAD_SIZES = 2, ORC_BAD_EXPERT = 3, ORC_BAD_TOPK = 4,
+       ORC_BAD_SLOT = 5 };
 
 static const float NF4_TABLE[16] = {
     -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
@@ -307,4 +308,79 @@ int oracle_baseline_bf16(const uint16_t *x, const uint8_t *w, const float *absma
     }
     free(row_expert);
     return ORC_OK;
+}
+
+/* ------------------------------------------------------ router top-k */
+/* Per token: the top_k experts by logit, picked one at a time as the largest
+   remaining logit (equal logits: the lower expert id; a NaN logit counts as
+   -inf), and their softmax weights in fp64, exp(l - l_max) over the sum of
+   exp(l_e - l_max) for all E experts (renorm == 0) or for the selected ones
+   (renorm == 1). Package page "grouped-nf4-gemm", "Owns" (router top-k). */
+int oracle_router_topk(const float *logits, int64_t T, int32_t E, int32_t k, int32_t renorm,
+                       int32_t *ids, double *weights) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return ORC_BAD_SHAPE;
+  for (int64_t t = 0; t < T; ++t) {
+    const float *row = logits + t * E;
+    int32_t *sel = ids + t * k;
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      double bv = 0.0;
+      for (int e = 0; e < E; ++e) {
+        int taken = 0;
+        for (int i = 0; i < j; ++i) taken |= sel[i] == e;
+        if (taken) continue;
+        const double v = isnan(row[e]) ? -INFINITY : (double)row[e];
+        if (best < 0 || v > bv) {   /* strict: an equal logit keeps the lower id */
+          best = e;
+          bv = v;
+        }
+      }
+      sel[j] = best;
+    }
+    const double lmax = isnan(row[sel[0]]) ? -INFINITY : (double)row[sel[0]];
+    double den = 0.0;
+    if (renorm) {
+      for (int j = 0; j < k; ++j) den += exp((double)row[sel[j]] - lmax);
+    } else {
+      for (int e = 0; e < E; ++e) den += exp((double)row[e] - lmax);
+    }
+    for (int j = 0; j < k; ++j) weights[t * k + j] = exp((double)row[sel[j]] - lmax) / den;
+  }
+  return ORC_OK;
+}
+
+/* ---------------------------------------------------- weighted combine */
+/* out[t][h] = sum_{j < k} w[t][j] * y[p(t*k + j)][h] in fp64, where p(s) is
+   the position of slot s in sorted_idx (entries of -1 are slots left out and
+   contribute nothing). Package page "grouped-nf4-gemm", "Owns" (the weighted
+   combine). */
+int oracle_moe_combine(const uint16_t *y, const int32_t *sorted_idx, const float *w, int64_t T,
+                       int32_t k, int32_t H, double *out) {
+  if (T < 0 || k < 1 || H < 1) return ORC_BAD_SHAPE;
+  const int64_t S = T * k;
+  int64_t *pos = (int64_t *)malloc((size_t)(S > 0 ? S : 1) * sizeof(int64_t));
+  if (!pos) return ORC_BAD_SHAPE;
+  for (int64_t s = 0; s < S; ++s) pos[s] = -1;
+  for (int64_t i = 0; i < S; ++i) {
+    const int32_t s = sorted_idx[i];
+    if (s == -1) continue;
+    if (s < 0 || s >= S) {
+      free(pos);
+      return ORC_BAD_SLOT;
+    }
+    pos[s] = i;
+  }
+  for (int64_t t = 0; t < T; ++t) {
+    for (int32_t h = 0; h < H; ++h) {
+      double acc = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        const int64_t p = pos[t * k + j];
+        if (p < 0) continue;
+        acc += (double)w[t * k + j] * (double)bf16_to_f32(y[p * H + h]);
+      }
+      out[t * H + h] = acc;
+    }
+  }
+  free(pos);
+  return ORC_OK;
 }

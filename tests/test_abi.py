@@ -82,9 +82,33 @@ def test_moe_align_and_dequant_host_checks():
     assert lib.gnf4_dequant_debug(1, 1, 0, 64, 64, 0, 1, None) == 0
 
 
+def test_router_topk_and_combine_host_checks():
+    lib = gnf4.load_library()
+    # gnf4_router_topk(logits, T, E, top_k, renormalize, ids, weights, stream)
+    assert lib.gnf4_router_topk(1, -1, 8, 2, 1, 1, 1, None) == 1
+    assert lib.gnf4_router_topk(1, 4, 8, 0, 1, 1, 1, None) == 1
+    assert lib.gnf4_router_topk(1, 4, 8, 2, 2, 1, 1, None) == 1
+    assert lib.gnf4_router_topk(1, 4, 8, 9, 1, 1, 1, None) == 3       # top_k > E
+    assert lib.gnf4_router_topk(1, 4, 64, 33, 1, 1, 1, None) == 3     # top_k > GNF4_MAX_TOPK
+    assert lib.gnf4_router_topk(1, 4, 2048, 2, 1, 1, 1, None) == 3    # E > GNF4_MAX_EXPERTS
+    assert lib.gnf4_router_topk(None, 0, 8, 2, 1, None, None, None) == 0
+    assert lib.gnf4_router_topk(None, 4, 8, 2, 1, 1, 1, None) == 1
+    # gnf4_moe_combine(y, sorted_idx, weights, T, top_k, H, out, ws, ws_bytes, stream)
+    ws = gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_MOE_COMBINE, 8)
+    assert ws >= 256 + 8 * 4
+    assert lib.gnf4_moe_combine(1, 1, 1, -1, 2, 64, 1, 1, ws, None) == 1
+    assert lib.gnf4_moe_combine(1, 1, 1, 4, 2, 0, 1, 1, ws, None) == 1
+    assert lib.gnf4_moe_combine(1, 1, 1, 4, 33, 64, 1, 1, 1 << 20, None) == 3
+    assert lib.gnf4_moe_combine(None, None, None, 0, 2, 64, None, None, 0, None) == 0
+    assert lib.gnf4_moe_combine(None, 1, 1, 4, 2, 64, 1, 1, ws, None) == 1
+    assert lib.gnf4_moe_combine(1, 1, 1, 4, 2, 64, 1, 1, ws - 1, None) == 4
+
+
 def test_host_buffers_are_refused():
     # Host memory is refused with GNF4_ERR_HOST_POINTER (no host path exists).
     buf = (ctypes.c_uint8 * (1 << 16))()
     p = ctypes.addressof(buf)
     assert _gemm(gnf4.load_library(), x=p, w=p, absmax=p, sizes=p, expert_ids=p, y=p, ws=p) == 2
     assert gnf4.load_library().gnf4_dequant_debug(p, p, 4, 64, 64, 0, p, None) == 2
+    assert gnf4.load_library().gnf4_router_topk(p, 4, 8, 2, 1, p, p, None) == 2
+    assert gnf4.load_library().gnf4_moe_combine(p, p, p, 4, 2, 64, p, p, 1 << 12, None) == 2

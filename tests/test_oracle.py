@@ -357,3 +357,110 @@ def test_nf4_bytes_vs_bf16_ratio():
     nbytes = packed.nbytes + absmax.nbytes
     assert nbytes == 0.5625 * E * N * K
     assert round(2 * E * N * K / nbytes, 2) == 3.56
+
+
+# ---------------------------------------------------------------------------
+# Router top-k and weighted combine (package page "grouped-nf4-gemm", "Owns":
+# the decode glue around the grouped GEMM)
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (37, 64, 8), (200, 128, 4), (16, 1000, 32), (5, 3, 3)])
+@pytest.mark.parametrize("renorm", [False, True])
+def test_router_topk_matches_stable_argsort_and_scipy_softmax(T, E, k, renorm):
+    rng = np.random.default_rng(T * 7 + E + k)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ids, w = oracle.router_topk(logits, k, renorm)
+    # ids: a library sort (stable: equal logits keep the lower expert id first)
+    assert np.array_equal(ids, np.argsort(-logits, axis=1, kind="stable")[:, :k])
+    lg = logits.astype(np.float64)
+    if renorm:
+        ref = scipy.special.softmax(np.take_along_axis(lg, ids, axis=1), axis=1)
+    else:
+        ref = np.take_along_axis(scipy.special.softmax(lg, axis=1), ids, axis=1)
+    np.testing.assert_allclose(w, ref, rtol=1e-12, atol=0)
+    if renorm:
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-12)
+    else:
+        assert (w.sum(axis=1) <= 1.0 + 1e-12).all()
+    assert (np.diff(w, axis=1) <= 0).all()   # descending logits -> descending weights
+
+
+def test_router_topk_ties_nan_and_shift():
+    rng = np.random.default_rng(5)
+    # many equal logits: the lower expert id goes first
+    logits = rng.integers(0, 3, size=(64, 40)).astype(np.float32)
+    ids, w = oracle.router_topk(logits, 6, True)
+    assert np.array_equal(ids, np.argsort(-logits, axis=1, kind="stable")[:, :6])
+    # all equal: the first top_k experts, equal weights
+    ids, w = oracle.router_topk(np.zeros((3, 10), np.float32), 4, False)
+    assert (ids == np.arange(4)).all() and np.allclose(w, 0.1)
+    # a NaN logit ranks as -inf: it is chosen only after every number
+    logits = rng.standard_normal((8, 12)).astype(np.float32)
+    logits[:, 3] = np.nan
+    ids, _ = oracle.router_topk(logits, 11, True)
+    assert not (ids == 3).any()
+    ids, _ = oracle.router_topk(logits, 12, True)
+    assert (ids[:, -1] == 3).all()
+    # shifting every logit of a token changes neither the choice nor the weights
+    logits = rng.standard_normal((16, 32)).astype(np.float32)
+    a_ids, a_w = oracle.router_topk(logits, 4, False)
+    b_ids, b_w = oracle.router_topk(logits + np.float32(8.0), 4, False)
+    assert np.array_equal(a_ids, b_ids)
+    np.testing.assert_allclose(a_w, b_w, rtol=1e-6)   # the shift itself rounds in fp32
+
+
+def _combine_numpy(y_bits, sorted_idx, w):
+    # independent of the C oracle: inverse permutation by fancy indexing,
+    # weighted sum by broadcasting
+    T, k = w.shape
+    yf = synth.bf16_bits_to_f32(y_bits).astype(np.float64)
+    inv = np.full(T * k, -1, dtype=np.int64)
+    valid = sorted_idx >= 0
+    inv[sorted_idx[valid]] = np.nonzero(valid)[0]
+    rows = np.where(inv >= 0, inv, 0).reshape(T, k)
+    contrib = yf[rows] * w.astype(np.float64)[:, :, None] * (inv >= 0).reshape(T, k)[:, :, None]
+    return contrib.sum(axis=1)
+
+
+@pytest.mark.parametrize("T,E,k,H", [(1, 4, 1, 16), (37, 16, 2, 64), (64, 128, 8, 40)])
+def test_moe_combine_matches_numpy_through_the_real_sort(T, E, k, H):
+    rng = np.random.default_rng(T + E + k + H)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ids, w = oracle.router_topk(logits, k, True)
+    sorted_idx, _, _, _ = oracle.moe_align(ids, E)
+    y = synth.activations_bf16(T * k, H, seed=T + H)
+    out = oracle.moe_combine(y, sorted_idx, w.astype(np.float32))
+    np.testing.assert_allclose(out, _combine_numpy(y, sorted_idx, w.astype(np.float32)),
+                               rtol=1e-12, atol=1e-300)
+
+
+def test_moe_combine_special_cases():
+    rng = np.random.default_rng(9)
+    T, k, H = 12, 3, 24
+    perm = rng.permutation(T * k).astype(np.int32)
+    y = synth.activations_bf16(T * k, H, seed=9)
+    yf = synth.bf16_bits_to_f32(y).astype(np.float64)
+    # one-hot weights read back exactly the row that holds slot t*k + j
+    for j in range(k):
+        w = np.zeros((T, k), np.float32)
+        w[:, j] = 1.0
+        out = oracle.moe_combine(y, perm, w)
+        pos = np.argsort(perm)
+        assert np.array_equal(out, yf[pos[np.arange(T) * k + j]])
+    # slots left out (-1) contribute nothing
+    w = rng.uniform(0.1, 1.0, size=(T, k)).astype(np.float32)
+    cut = perm.copy()
+    cut[::5] = -1
+    full = oracle.moe_combine(y, perm, w)
+    part = oracle.moe_combine(y, cut, w)
+    missing = perm[::5]
+    w2 = w.copy().reshape(-1)
+    w2[missing] = 0.0
+    assert np.allclose(part, oracle.moe_combine(y, perm, w2.reshape(T, k)), rtol=0, atol=0)
+    assert not np.allclose(part, full)
+    # linear in the weights
+    assert np.array_equal(oracle.moe_combine(y, perm, 2 * w), 2 * full)
+    # an entry outside [-1, T*k) is refused
+    bad = perm.copy()
+    bad[0] = T * k
+    with pytest.raises(oracle.OracleError):
+        oracle.moe_combine(y, bad, w)
