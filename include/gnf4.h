@@ -219,7 +219,7 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
  *   renormalize == 0: exp(l_e - l_max) / sum over all E experts
  *   renormalize == 1: exp(l_e - l_max) / sum over the top_k selected experts
  * computed in fp32 (weights within about 1e-6 relative of the exact values;
- * weights are unspecified if a logit is infinite or every logit is NaN).
+ * weights are unspecified if a logit is infinite or NaN).
  *
  *   logits        device fp32 [T][E], 4-byte aligned
  *   T >= 0, 1 <= E <= GNF4_MAX_EXPERTS, 1 <= top_k <= min(E, GNF4_MAX_TOPK)

@@ -48,10 +48,10 @@ def test_router_topk_ties_and_nan():
     ref_ids, ref_w = oracle.router_topk(logits, 7, True)
     assert np.array_equal(ids, ref_ids)
     np.testing.assert_allclose(w, ref_w, rtol=2e-5)
-    logits = rng.standard_normal((40, 50)).astype(np.float32)
+    logits = rng.standard_normal((40, 30)).astype(np.float32)
     logits[:, 7] = np.nan
     logits[::3, 11] = np.nan
-    for k in (4, 49, 50):
+    for k in (4, 29, 30):   # NaN logits are chosen last (top_k <= GNF4_MAX_TOPK)
         ids, _ = _router(logits, k, True)
         ref_ids, _ = oracle.router_topk(logits, k, True)
         assert np.array_equal(ids, ref_ids)
