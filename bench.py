@@ -354,11 +354,16 @@ def run_ours(args, rank, world, local_rank):
     kern_ms = [sum(v) / len(v) for v in per_kernel]   # NaN if a timestamp was missing
 
     ms = max_over_ranks(ms, world, dev)
-    glue = time_glue(prob, stream)
 
     # end to end: host (pinned) inputs -> device, the C-ABI calls, results -> host
     e2e = run_e2e(prob, stream, max(3, min(args.steps, 2000) // 10))
     e2e = (max_over_ranks(e2e[0], world, dev),) + tuple(e2e[1:])
+    # the glue entry points last: an error there is reported in the line
+    # instead of costing the step's numbers
+    try:
+        glue = time_glue(prob, stream)
+    except Exception as exc:   # noqa: BLE001
+        glue = {"error": f"{type(exc).__name__}: {exc}"}
     return prob, ms, kern_ms, clk, e2e, launches_per_step, glue
 
 
