@@ -28,6 +28,7 @@ import argparse
 import ctypes
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -63,7 +64,14 @@ def peaks():
 
 
 def source_hash(path):
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    """sha256 prefix of a kernel source's code: comments, trailing blanks and
+    empty lines removed (they do not change what the compiler emits), so a
+    comment edit keeps the committed counters valid and a code edit does not."""
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode("utf-8")).hexdigest()[:16]
 
 
 def traffic_for(kernel, workload, gemm):
