@@ -20,13 +20,16 @@
 // row is scaled by 2^S, S = beta + 14 with 2^beta * max(absmax of the row) in
 // [1, 2) (powers of two scale exactly); the scaled fp32 weight w'' = NF4 *
 // absmax * 2^S is split into hi = bf16(w'') and the exact remainder
-// w'' - hi, which is below 64 in magnitude and goes to e4m3. Per K-step of 64:
+// w'' - hi, which is below 64 in magnitude and goes to e4m3. Each activation
+// row is scaled by 2^s (its largest magnitude into [2^14, 2^15)) by a
+// pre-pass that writes its bf16 copy (exact) and its e5m2 copy. Per K-step
+// of 64:
 //   hi pass: 4 x kind::f16, bf16 hi (TMEM) x bf16 x (shared memory), K = 16
 //   lo pass: 2 x kind::f8f6f4, e4m3 remainder (TMEM) x e5m2 x (shared
-//            memory, an e5m2 copy of x made by a pre-pass), K = 32
-// into one fp32 accumulator; the epilogue divides 2^S out and rounds once to
-// bf16. The lo pass runs at twice the bf16 rate, so a K-step costs 1.5 bf16
-// passes instead of 2.
+//            memory), K = 32
+// into one fp32 accumulator; the epilogue divides 2^S and 2^s out and rounds
+// once to bf16. The lo pass runs at twice the bf16 rate, so a K-step costs
+// 1.5 bf16 passes instead of 2.
 //
 // Roles per CTA (12 warps, one CTA per SM, the pair persistent over tiles):
 //   warp 0  TMA: its half of the x tile (bf16, 128-byte swizzle) and of the
@@ -45,7 +48,9 @@
 //           per-lane replicated table of the 16 code values, writes hi and
 //           remainder to TMEM (tcgen05.st, a 5-stage ring); one lane per warp
 //           then arrives on the leader's barrier. The epilogue reads the
-//           accumulator back (tcgen05.ld).
+//           accumulator back (tcgen05.ld) 32 tokens at a time and writes
+//           each chunk through a shared-memory box with one bulk tensor
+//           store.
 // Every wait is bounded (2 s); on expiry the kernel records
 // GNF4_DEVERR_TIMEOUT, lets its asynchronous work drain and returns through
 // the final cluster barrier.
