@@ -43,3 +43,19 @@ def test_reference_arm_world_size_2_prints_one_line():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_counter_key_ignores_comments_but_not_code(tmp_path):
+    # bench.py keys the committed ncu counters by a hash of a kernel source's
+    # code: editing a comment keeps them, editing code drops them
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    base = "int f(int a) {\n  return a + 1;   // one\n}\n/* block\n comment */\n"
+    p = tmp_path / "k.cu"
+    p.write_text(base)
+    h0 = bench.source_hash(str(p))
+    p.write_text(base.replace("// one", "// the successor").replace("block", "other block") + "\n\n")
+    assert bench.source_hash(str(p)) == h0
+    p.write_text(base.replace("a + 1", "a + 2"))
+    assert bench.source_hash(str(p)) != h0
