@@ -2,10 +2,13 @@
 // top-k (gnf4_router_topk) before the token->expert sort, and the top-k
 // weighted combine (gnf4_moe_combine) after the down projection.
 //
-// Passage: "grouped-nf4-gemm" package page, "Owns" (the decode glue around
-// the grouped GEMM: router top-k, swiglu and the weighted combine), and the
-// README's opening section (the GEMM consumes (sizes, expert_ids) produced
-// after the token->expert sort of the router's choices).
+// Passage: "grouped-nf4-gemm" package page, "Use this when" (the tail of
+// small launches around the expert GEMMs in a batch-1 decode step, router
+// softmax and top-k and the top-k combine among them, each to be folded into
+// one launch) and its header block ("Owns": the decode glue kernels, combine
+// among them); the README's opening section (the GEMM consumes
+// (sizes, expert_ids) produced by the token->expert sort of the router's
+// choices).
 //
 // router_topk: one warp per token. Each lane holds the logits of experts
 // lane, lane + 32, ... in registers (E <= 1024); top_k rounds of a warp

@@ -211,8 +211,9 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
  * gnf4_router_topk -- the router's choice of experts per token, the input of
  * gnf4_moe_align.
  *
- * Passage: package page "grouped-nf4-gemm", "Owns" (the decode glue around the
- * grouped GEMM, router top-k among it). The pages fix no formula; this
+ * Passage: package page "grouped-nf4-gemm", "Use this when" (router softmax
+ * and top-k among the small decode launches to fold into one each). The
+ * pages fix no formula; this
  * library takes the usual softmax router: per token t, the top_k experts with
  * the largest logits (equal logits: lower expert id first; a NaN logit ranks
  * as -inf) in descending order, and their softmax weights
@@ -237,8 +238,9 @@ GNF4_API gnf4_status gnf4_router_topk(const float *logits, int64_t T, int32_t E,
  * where p(s) is the row of y that holds slot s (the position of s in
  * sorted_idx), summed in fp32 with j ascending and rounded once (RNE).
  *
- * Passage: package page "grouped-nf4-gemm", "Owns" (the weighted combine of
- * the decode glue).
+ * Passage: package page "grouped-nf4-gemm", header block ("Owns": the decode
+ * glue kernels, combine among them) and "Use this when" (the top-k combine
+ * among the small decode launches to fold into one each).
  *
  *   y             device bf16 [T*top_k][H]: row i is the down-projection output
  *                 of slot sorted_idx[i] (the grouped GEMM's row order)

@@ -25,7 +25,9 @@ grouped_nf4_gemm 0.1.0, opening section, unless stated):
   the fidelity comparator of the page's "The claim" section.
 * :func:`router_topk` / :func:`moe_combine` -- the router's top-k with softmax
   weights, and the top-k weighted combine after the down projection (package
-  page "grouped-nf4-gemm", "Owns": the decode glue around the grouped GEMM).
+  page "grouped-nf4-gemm", "Use this when": router softmax and top-k and the
+  top-k combine among the small decode launches; "Owns": combine among the
+  decode glue kernels).
 """
 from __future__ import annotations
 

@@ -315,7 +315,8 @@ int oracle_baseline_bf16(const uint16_t *x, const uint8_t *w, const float *absma
    remaining logit (equal logits: the lower expert id; a NaN logit counts as
    -inf), and their softmax weights in fp64, exp(l - l_max) over the sum of
    exp(l_e - l_max) for all E experts (renorm == 0) or for the selected ones
-   (renorm == 1). Package page "grouped-nf4-gemm", "Owns" (router top-k). */
+   (renorm == 1). Package page "grouped-nf4-gemm", "Use this when" (router
+   softmax and top-k). */
 int oracle_router_topk(const float *logits, int64_t T, int32_t E, int32_t k, int32_t renorm,
                        int32_t *ids, double *weights) {
   if (T < 0 || E < 1 || k < 1 || k > E) return ORC_BAD_SHAPE;
@@ -352,8 +353,8 @@ int oracle_router_topk(const float *logits, int64_t T, int32_t E, int32_t k, int
 /* ---------------------------------------------------- weighted combine */
 /* out[t][h] = sum_{j < k} w[t][j] * y[p(t*k + j)][h] in fp64, where p(s) is
    the position of slot s in sorted_idx (entries of -1 are slots left out and
-   contribute nothing). Package page "grouped-nf4-gemm", "Owns" (the weighted
-   combine). */
+   contribute nothing). Package page "grouped-nf4-gemm", "Owns" and "Use this
+   when" (the top-k combine). */
 int oracle_moe_combine(const uint16_t *y, const int32_t *sorted_idx, const float *w, int64_t T,
                        int32_t k, int32_t H, double *out) {
   if (T < 0 || k < 1 || H < 1) return ORC_BAD_SHAPE;

@@ -360,7 +360,8 @@ def test_nf4_bytes_vs_bf16_ratio():
 
 
 # ---------------------------------------------------------------------------
-# Router top-k and weighted combine (package page "grouped-nf4-gemm", "Owns":
+# Router top-k and weighted combine (package page "grouped-nf4-gemm", "Use
+# this when" and "Owns":
 # the decode glue around the grouped GEMM)
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (37, 64, 8), (200, 128, 4), (16, 1000, 32), (5, 3, 3)])

@@ -1,5 +1,6 @@
 """GPU parity for the steps either side of the grouped GEMM (package page
-"grouped-nf4-gemm", "Owns": the decode glue): the router's top-k and the
+"grouped-nf4-gemm", "Use this when" and "Owns": the decode glue): the
+router's top-k and the
 top-k weighted combine, through the C ABI, against the CPU oracle.
 
 * router top-k: expert ids bit-exact (the choice compares the fp32 logits
