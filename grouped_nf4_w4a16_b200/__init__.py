@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     GNF4_OP_MOE_ALIGN,
     GNF4_OP_GROUPED_GEMM,
     GNF4_OP_MOE_COMBINE,
+    GNF4_OP_GROUPED_DGRAD,
     GNF4_MAX_TOPK,
     DEVERR_BITS,
     EXPORTED_SYMBOLS,
@@ -32,6 +33,7 @@ from .binding import (  # noqa: F401
     gnf4_grouped_gemm_noalloc,
     gnf4_router_topk,
     gnf4_moe_combine,
+    gnf4_grouped_dgrad,
     GNF4_NOALLOC_SCRATCH_BYTES,
     gnf4_dequant_debug,
     gnf4_read_device_status,

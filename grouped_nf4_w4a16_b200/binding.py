@@ -28,7 +28,7 @@ GNF4_NOALLOC_SCRATCH_BYTES = 8 << 20
 GNF4_EPI_NONE, GNF4_EPI_SWIGLU = 0, 1
 GNF4_MODE_AUTO, GNF4_MODE_DECODE, GNF4_MODE_PREFILL = 0, 1, 2
 GNF4_OUT_F32, GNF4_OUT_BF16 = 0, 1
-GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM, GNF4_OP_MOE_COMBINE = 0, 1, 2
+GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM, GNF4_OP_MOE_COMBINE, GNF4_OP_GROUPED_DGRAD = 0, 1, 2, 3
 GNF4_MAX_TOPK = 32
 DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capacity": 0x10,
                "slot": 0x20}
@@ -37,7 +37,7 @@ DEVERR_BITS = {"sizes": 0x1, "expert": 0x2, "topk": 0x4, "timeout": 0x8, "capaci
 EXPORTED_SYMBOLS = (
     "gnf4_moe_align", "gnf4_grouped_gemm", "gnf4_dequant_debug", "gnf4_workspace_bytes",
     "gnf4_read_device_status", "gnf4_status_string", "gnf4_version",
-    "gnf4_grouped_gemm_noalloc", "gnf4_router_topk", "gnf4_moe_combine",
+    "gnf4_grouped_gemm_noalloc", "gnf4_router_topk", "gnf4_moe_combine", "gnf4_grouped_dgrad",
 )
 
 _lib = None
@@ -86,6 +86,8 @@ def load_library():
     lib.gnf4_router_topk.restype = ctypes.c_int
     lib.gnf4_moe_combine.argtypes = [P, P, P, i64, i32, i32, P, P, sz, P]
     lib.gnf4_moe_combine.restype = ctypes.c_int
+    lib.gnf4_grouped_dgrad.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, sz, P]
+    lib.gnf4_grouped_dgrad.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -227,6 +229,36 @@ def gnf4_dequant_debug(w: torch.Tensor, absmax: torch.Tensor, out_dtype: int = G
                                            _ptr(out), _stream(stream))
     _check(st, "gnf4_dequant_debug")
     return out
+
+
+def gnf4_grouped_dgrad(dy: torch.Tensor, w: torch.Tensor, absmax: torch.Tensor,
+                       sizes: torch.Tensor, expert_ids: torch.Tensor, *,
+                       dx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       blocksize: int = 64, stream=None) -> torch.Tensor:
+    """dx bf16 [M, K] = grouped dy [M, N] bf16 . W (w [E,N,K/2] uint8, absmax [E,N,K/64] fp32)."""
+    _need(dy, "dy", torch.bfloat16)
+    _need(w, "w", torch.uint8)
+    _need(absmax, "absmax", torch.float32)
+    _need(sizes, "sizes", torch.int32)
+    _need(expert_ids, "expert_ids", torch.int32)
+    M, N = dy.shape
+    E, Nw, Kh = w.shape
+    if Nw != N:
+        raise ValueError(f"w has N={Nw} but dy has N={N}")
+    K = 2 * Kh
+    G = sizes.numel()
+    if dx is None:
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dy.device)
+    else:
+        _need(dx, "dx", torch.bfloat16)
+    if workspace is None:
+        workspace = make_workspace(gnf4_workspace_bytes(GNF4_OP_GROUPED_DGRAD, M, N, K, E, G),
+                                   dy.device)
+    st = load_library().gnf4_grouped_dgrad(
+        _ptr(dy), _ptr(w), _ptr(absmax), _ptr(sizes), _ptr(expert_ids), G, M, N, K, E, blocksize,
+        _ptr(dx), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "gnf4_grouped_dgrad")
+    return dx
 
 
 def gnf4_router_topk(logits: torch.Tensor, top_k: int, *, renormalize: bool = True,

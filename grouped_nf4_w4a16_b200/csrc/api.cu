@@ -76,6 +76,7 @@ size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t
   (void)E;
   if (op == GNF4_OP_MOE_ALIGN) return kWsHeaderBytes;
   if (op == GNF4_OP_MOE_COMBINE) return M < 0 ? 0 : combine_workspace_bytes(M);
+  if (op == GNF4_OP_GROUPED_DGRAD) return kWsHeaderBytes;
   if (op != GNF4_OP_GROUPED_GEMM || M < 0 || N < 1 || K < 1 || G < 1) return 0;
   const size_t d = decode_workspace_bytes(M, N, K, G, 1);
   const size_t d2 = decode_workspace_bytes(M, N, K, G, 0);
@@ -173,6 +174,31 @@ gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t ro
   if (!aligned(w, 16) || !aligned(out, 16) || !aligned(absmax, 4)) return GNF4_ERR_MISALIGNED;
   return from_cuda(launch_dequant(w, absmax, rows, K, out_dtype == GNF4_OUT_BF16 ? 1 : 0, out,
                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gnf4_status gnf4_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float *absmax,
+                               const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                               int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                               uint16_t *dx, void *workspace, size_t ws_bytes,
+                               gnf4_stream_t stream) {
+  if (!dy || !w || !absmax || !sizes || !expert_ids || !dx || !workspace)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS || M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (K / 256 + 1 > 65535) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < kWsHeaderBytes) return GNF4_ERR_WORKSPACE_TOO_SMALL;
+  if (M == 0) return GNF4_OK;
+  if (!is_device_pointer(dy) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
+      !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(dx) ||
+      !is_device_pointer(workspace))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(dy, 2) || !aligned(dx, 2) || !aligned(absmax, 4) || !aligned(sizes, 4) ||
+      !aligned(expert_ids, 4) || !aligned(workspace, 16))
+    return GNF4_ERR_MISALIGNED;
+  return from_cuda(launch_grouped_dgrad(dy, w, absmax, sizes, expert_ids, G, M, N, K, E, dx,
+                                        static_cast<WsHeader *>(workspace),
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 gnf4_status gnf4_router_topk(const float *logits, int64_t T, int32_t E, int32_t top_k,

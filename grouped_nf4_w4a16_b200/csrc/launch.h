@@ -57,6 +57,12 @@ cudaError_t launch_moe_combine(const uint16_t *y, const int32_t *sorted_idx, con
                                int64_t T, int32_t k, int32_t H, uint16_t *out, void *workspace,
                                cudaStream_t stream);
 
+// ---- grouped dgrad (dgrad.cu)
+cudaError_t launch_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float *absmax,
+                                 const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                                 int64_t M, int32_t N, int32_t K, int32_t E, uint16_t *dx,
+                                 WsHeader *hdr, cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

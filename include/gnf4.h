@@ -76,7 +76,12 @@ typedef enum {
 typedef enum { GNF4_EPI_NONE = 0, GNF4_EPI_SWIGLU = 1 } gnf4_epilogue;
 typedef enum { GNF4_MODE_AUTO = 0, GNF4_MODE_DECODE = 1, GNF4_MODE_PREFILL = 2 } gnf4_mode;
 typedef enum { GNF4_OUT_F32 = 0, GNF4_OUT_BF16 = 1 } gnf4_out_dtype;
-typedef enum { GNF4_OP_MOE_ALIGN = 0, GNF4_OP_GROUPED_GEMM = 1, GNF4_OP_MOE_COMBINE = 2 } gnf4_op;
+typedef enum {
+    GNF4_OP_MOE_ALIGN = 0,
+    GNF4_OP_GROUPED_GEMM = 1,
+    GNF4_OP_MOE_COMBINE = 2,
+    GNF4_OP_GROUPED_DGRAD = 3
+} gnf4_op;
 
 /* Bits of the device error word (gnf4_read_device_status). */
 #define GNF4_DEVERR_SIZES 0x1u      /* a size < 0, or sum(sizes) != M */
@@ -208,6 +213,33 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
                                gnf4_stream_t stream);
 
 /*
+ * gnf4_grouped_dgrad -- the gradient of the grouped GEMM with respect to its
+ * activations, over the same packed stack:
+ *   dx[m][k] = bf16( sum_n dy[m][n] * NF4[code(e,n,k)] * absmax[e][n][k/64] )
+ * with e the expert of row m's group, the weight one fp32 multiply (as in
+ * the forward kernels), the sum in fp32 over n ascending, one rounding (RNE).
+ *
+ * Passage: package page "grouped-nf4-gemm", header block ("Owns": the grouped
+ * packed GEMM and its dgrad) and "Do not use this when" (the dgrad refuses
+ * tensors that are not on the device, as the GEMM does).
+ *
+ *   dy          device bf16 [M][N] (the gradient of the GEMM's output y)
+ *   w, absmax, sizes, expert_ids, G, E, blocksize: as for gnf4_grouped_gemm
+ *   M >= 0, N >= 1, K % 64 == 0, 1 <= G, E <= GNF4_MAX_EXPERTS, M < 2^31
+ *   dx          device bf16 [M][K] (written; must not overlap dy)
+ *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_DGRAD, ...)
+ *               bytes (the 256-byte status header), zero-filled once.
+ * A metadata error (as for gnf4_grouped_gemm) sets the device error word and
+ * nothing is written. One launch of a CUDA-core kernel sized for decode
+ * batches (it is not the tensor-core path).
+ */
+GNF4_API gnf4_status gnf4_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float *absmax,
+                                        const int32_t *sizes, const int32_t *expert_ids,
+                                        int32_t G, int64_t M, int32_t N, int32_t K, int32_t E,
+                                        int32_t blocksize, uint16_t *dx, void *workspace,
+                                        size_t ws_bytes, gnf4_stream_t stream);
+
+/*
  * gnf4_router_topk -- the router's choice of experts per token, the input of
  * gnf4_moe_align.
  *
@@ -267,7 +299,8 @@ GNF4_API gnf4_status gnf4_moe_combine(const uint16_t *y, const int32_t *sorted_i
  * gnf4_workspace_bytes -- workspace size for an op and problem size (no GPU
  * work; queries the current device's SM count once). For GNF4_OP_MOE_ALIGN
  * only E matters; for GNF4_OP_GROUPED_GEMM the size covers every mode; for
- * GNF4_OP_MOE_COMBINE, M is T*top_k and nothing else matters.
+ * GNF4_OP_MOE_COMBINE, M is T*top_k and nothing else matters; for
+ * GNF4_OP_GROUPED_DGRAD it is the status header alone.
  */
 GNF4_API size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t E, int32_t G);
 

@@ -23,6 +23,10 @@ grouped_nf4_gemm 0.1.0, opening section, unless stated):
   "grouped-nf4-gemm", "Owns": the decode glue includes swiglu).
 * :func:`baseline_bf16` -- dequantise-to-bf16 then fp32-accumulated matmul,
   the fidelity comparator of the page's "The claim" section.
+* :func:`grouped_dgrad_f64` -- the gradient of the grouped GEMM with respect
+  to its activations, dx = dy . W per group, in fp64 (package page
+  "grouped-nf4-gemm", header block, "Owns": the grouped packed GEMM and its
+  dgrad).
 * :func:`router_topk` / :func:`moe_combine` -- the router's top-k with softmax
   weights, and the top-k weighted combine after the down projection (package
   page "grouped-nf4-gemm", "Use this when": router softmax and top-k and the
@@ -82,9 +86,11 @@ def _load():
         lib.oracle_baseline_bf16.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
         lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, P, P]
         lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i32, P]
+        lib.oracle_grouped_dgrad_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P]
         for name in ("oracle_quantize_nf4", "oracle_dequant_f32", "oracle_dequant_bf16",
                      "oracle_moe_align", "oracle_grouped_gemm_f64", "oracle_swiglu_f64",
-                     "oracle_baseline_bf16", "oracle_router_topk", "oracle_moe_combine"):
+                     "oracle_baseline_bf16", "oracle_router_topk", "oracle_moe_combine",
+                     "oracle_grouped_dgrad_f64"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -249,3 +255,22 @@ def moe_combine(y: np.ndarray, sorted_idx: np.ndarray, weights: np.ndarray) -> n
     out = np.empty((T, H), dtype=np.float64)
     _check(_load().oracle_moe_combine(_p(y), _p(sorted_idx), _p(weights), T, k, H, _p(out)))
     return out
+
+
+def grouped_dgrad_f64(dy: np.ndarray, w: np.ndarray, absmax: np.ndarray, sizes: np.ndarray,
+                      expert_ids: np.ndarray) -> np.ndarray:
+    """dx fp64 [M, K] from dy as bf16 bit patterns [M, N]."""
+    dy = np.ascontiguousarray(dy, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    absmax = np.ascontiguousarray(absmax, dtype=np.float32)
+    sizes = np.ascontiguousarray(sizes, dtype=np.int32)
+    expert_ids = np.ascontiguousarray(expert_ids, dtype=np.int32)
+    M, N = dy.shape
+    E, Nw, Kh = w.shape
+    if Nw != N:
+        raise OracleError("bad shape")
+    K = 2 * Kh
+    dx = np.empty((M, K), dtype=np.float64)
+    _check(_load().oracle_grouped_dgrad_f64(_p(dy), _p(w), _p(absmax), _p(sizes), _p(expert_ids),
+                                            sizes.size, M, N, K, E, _p(dx)))
+    return dx

@@ -385,3 +385,37 @@ int oracle_moe_combine(const uint16_t *y, const int32_t *sorted_idx, const float
   free(pos);
   return ORC_OK;
 }
+
+/* ------------------------------------------------ grouped dgrad (fp64) */
+/* The gradient of the grouped GEMM with respect to its activations:
+   dx[m, k] = sum_n dy[m, n] * NF4[code(e, n, k)] * absmax[e, n, k/64], e the
+   expert of row m's group, in fp64 (the same weight values as the forward
+   oracle). Package page "grouped-nf4-gemm", header block ("Owns": the grouped
+   packed GEMM and its dgrad).
+   dy: bf16 bits [M, N]; w: [E, N, K/2]; absmax: [E, N, K/64]; dx: fp64 [M, K]. */
+int oracle_grouped_dgrad_f64(const uint16_t *dy, const uint8_t *w, const float *absmax,
+                             const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                             int64_t M, int32_t N, int32_t K, int32_t E, double *dx) {
+    if (M < 0 || N <= 0 || K <= 0 || K % GNF4O_BLOCK || E <= 0 || G < 0) return ORC_BAD_SHAPE;
+    int32_t *row_expert = (int32_t *)malloc((size_t)(M > 0 ? M : 1) * sizeof(int32_t));
+    if (!row_expert) return ORC_BAD_SHAPE;
+    int st = rows_to_expert(sizes, expert_ids, G, M, E, row_expert);
+    if (st != ORC_OK) { free(row_expert); return st; }
+    const int64_t nb = K / GNF4O_BLOCK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        const int32_t e = row_expert[m];
+        double *acc = dx + m * K;
+        for (int32_t k = 0; k < K; ++k) acc[k] = 0.0;
+        for (int32_t n = 0; n < N; ++n) {
+            const double g = (double)bf16_to_f32(dy[m * N + n]);
+            const int64_t row = (int64_t)e * N + n;
+            const uint8_t *wr = w + row * (K / 2);
+            const float *ar = absmax + row * nb;
+            for (int32_t k = 0; k < K; ++k)
+                acc[k] += g * ((double)NF4_TABLE[code_at(wr, k)] * (double)ar[k / GNF4O_BLOCK]);
+        }
+    }
+    free(row_expert);
+    return ORC_OK;
+}

@@ -104,6 +104,23 @@ def test_router_topk_and_combine_host_checks():
     assert lib.gnf4_moe_combine(1, 1, 1, 4, 2, 64, 1, 1, ws - 1, None) == 4
 
 
+def test_grouped_dgrad_host_checks():
+    lib = gnf4.load_library()
+
+    def dg(**kw):
+        a = dict(dy=1, w=1, absmax=1, sizes=1, ids=1, G=2, M=8, N=16, K=128, E=2, bs=64, dx=1,
+                 ws=1, ws_bytes=256)
+        a.update(kw)
+        return lib.gnf4_grouped_dgrad(a["dy"], a["w"], a["absmax"], a["sizes"], a["ids"], a["G"],
+                                      a["M"], a["N"], a["K"], a["E"], a["bs"], a["dx"], a["ws"],
+                                      a["ws_bytes"], None)
+    assert dg(dy=None) == 1 and dg(dx=None) == 1 and dg(M=-1) == 1 and dg(G=0) == 1
+    assert dg(K=96) == 3 and dg(bs=32) == 3 and dg(E=2000) == 3
+    assert dg(ws_bytes=16) == 4
+    assert dg(M=0) == 0
+    assert gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_DGRAD, 8, 16, 128, 2, 2) == 256
+
+
 def test_host_buffers_are_refused():
     # Host memory is refused with GNF4_ERR_HOST_POINTER (no host path exists).
     buf = (ctypes.c_uint8 * (1 << 16))()
@@ -112,3 +129,5 @@ def test_host_buffers_are_refused():
     assert gnf4.load_library().gnf4_dequant_debug(p, p, 4, 64, 64, 0, p, None) == 2
     assert gnf4.load_library().gnf4_router_topk(p, 4, 8, 2, 1, p, p, None) == 2
     assert gnf4.load_library().gnf4_moe_combine(p, p, p, 4, 2, 64, p, p, 1 << 12, None) == 2
+    assert gnf4.load_library().gnf4_grouped_dgrad(p, p, p, p, p, 1, 4, 8, 64, 1, 64, p, p, 256,
+                                                  None) == 2

@@ -465,3 +465,63 @@ def test_moe_combine_special_cases():
     bad[0] = T * k
     with pytest.raises(oracle.OracleError):
         oracle.moe_combine(y, bad, w)
+
+
+# ---------------------------------------------------------------------------
+# Grouped dgrad (package page "grouped-nf4-gemm", header block, "Owns": the
+# grouped packed GEMM and its dgrad)
+
+@pytest.mark.parametrize("E,N,K,sizes,experts", [
+    (3, 48, 128, [3, 0, 5], [2, 0, 1]),
+    (2, 96, 320, [4, 4, 1], [1, 1, 0]),      # the same expert in two groups
+    (1, 8, 64, [6], [0]),
+])
+def test_grouped_dgrad_is_the_adjoint_of_the_forward(E, N, K, sizes, experts):
+    # <dy, GEMM(x)> == <dgrad(dy), x> for any x and dy, group by group: pins
+    # the dgrad to the (separately pinned) forward oracle
+    rng = np.random.default_rng(E + N + K)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    M = int(sum(sizes))
+    x = synth.activations_bf16(M, K, seed=N)
+    dy = synth.activations_bf16(M, N, seed=K)
+    y = oracle.grouped_gemm_f64(x, packed, absmax, sizes, experts)
+    dx = oracle.grouped_dgrad_f64(dy, packed, absmax, sizes, experts)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+    # per row (each row has its own expert): sum_n dy y == sum_k dx x
+    lhs, rhs = (dyf * y).sum(axis=1), (dx * xf).sum(axis=1)
+    scale = (np.abs(dyf)[:, :, None] * 0.1).sum(axis=(1, 2)) * np.abs(xf).sum(axis=1)
+    assert (np.abs(lhs - rhs) <= 1e-12 * scale + 1e-300).all()
+
+
+def test_grouped_dgrad_matches_numpy_matmul():
+    rng = np.random.default_rng(3)
+    E, N, K = 4, 40, 192
+    sizes, experts = [2, 0, 7, 3], [3, 1, 0, 3]
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    M = int(sum(sizes))
+    dy = synth.activations_bf16(M, N, seed=3)
+    dx = oracle.grouped_dgrad_f64(dy, packed, absmax, sizes, experts)
+    W = oracle.dequant_f32(packed.reshape(E * N, K // 2),
+                           absmax.reshape(E * N, K // 64)).astype(np.float64).reshape(E, N, K)
+    dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+    ref = np.zeros((M, K))
+    r = 0
+    for s, e in zip(sizes, experts):
+        ref[r:r + s] = dyf[r:r + s] @ W[e]
+        r += s
+    # the oracle multiplies in fp64, the library routine used here on the
+    # fp32-rounded dequantised weights: within fp32 rounding of each weight
+    np.testing.assert_allclose(dx, ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_grouped_dgrad_rejects_bad_metadata():
+    packed = np.zeros((2, 8, 32), np.uint8)
+    absmax = np.ones((2, 8, 1), np.float32)
+    dy = synth.activations_bf16(4, 8, seed=0)
+    with pytest.raises(oracle.OracleError):
+        oracle.grouped_dgrad_f64(dy, packed, absmax, [2, 1], [0, 1])    # sizes sum 3 != 4
+    with pytest.raises(oracle.OracleError):
+        oracle.grouped_dgrad_f64(dy, packed, absmax, [2, 2], [0, 2])    # expert 2 of 2
