@@ -376,10 +376,11 @@ def run_ours(args, rank, world, local_rank):
 
 
 def time_glue(prob, stream, reps=50):
-    """The steps either side of the GEMMs, timed outside the step: the router's
-    top-k on seeded N(0,1) logits [T, E] and the weighted combine of the last
-    GEMM's output [T*top_k, H]. CUDA events around `reps` back-to-back launches
-    after a warm-up; the inputs stay in L2 between launches (they are small)."""
+    """The entry points beside the GEMMs, timed outside the step: the router's
+    top-k on seeded N(0,1) logits [T, E], the weighted combine of the last
+    GEMM's output [T*top_k, H] and, for decode workloads, the dgrad of the last
+    GEMM with that output as dy. CUDA events around `reps` back-to-back
+    launches after a warm-up; the inputs stay in L2 between launches."""
     gnf4 = prob.gnf4
     w = prob.w
     dev = prob.topk.device
@@ -399,6 +400,15 @@ def time_glue(prob, stream, reps=50):
         "combine": (lambda: gnf4.gnf4_moe_combine(y, prob.sorted_idx, wts, out=out, workspace=ws),
                     S * H * 2 + w.T * H * 2 + S * 8),
     }
+    if not prob.prefill:
+        # the dgrad of the last GEMM (CUDA-core kernel, decode-sized batches only)
+        d = prob.gemms[-1]
+        g = d["g"]
+        dx = torch.empty((w.M, g.K), dtype=torch.bfloat16, device=dev)
+        ws_dg = gnf4.make_workspace(256, dev)
+        calls["dgrad"] = (lambda: gnf4.gnf4_grouped_dgrad(y, d["W"][0], d["A"][0], prob.sizes,
+                                                          prob.expert_ids, dx=dx, workspace=ws_dg),
+                          prob.U * g.N * g.K * 9 // 16 + w.M * g.N * 2 + w.M * g.K * 2)
     res = {}
     with torch.cuda.stream(stream):
         for name, (fn, nbytes) in calls.items():
@@ -413,7 +423,8 @@ def time_glue(prob, stream, reps=50):
             ms = a.elapsed_time(b) / reps
             res[name] = {"ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms / 1e3) / 1e9}
     res["how"] = (f"outside the timed step; {reps} back-to-back launches per entry point "
-                  f"(router: T x E fp32 logits; combine: T*top_k x {H} bf16 rows), inputs L2-resident")
+                  f"(router: T x E fp32 logits; combine: T*top_k x {H} bf16 rows; dgrad of the last "
+                  f"GEMM, decode workloads only), inputs L2-resident")
     return res
 
 
