@@ -22,7 +22,7 @@
  *  - Host-side checks run first and synchronously; on failure nothing is
  *    launched and a status != GNF4_OK is returned. Pointers that are not
  *    device memory (host or unregistered) give GNF4_ERR_HOST_POINTER.
- *  - Data that only the device knows (sizes, expert_ids, topk_ids) is checked
+ *  - Data that only the device knows (sizes, expert_ids, topk_ids, sorted_idx) is checked
  *    on the device. A violation sets a bit in the workspace's error word (see
  *    GNF4_DEVERR_*) and the kernel skips the affected work; it never traps.
  *    Read the word with gnf4_read_device_status.
@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GNF4_VERSION 100 /* 1.0.0 */
+#define GNF4_VERSION 110 /* 1.1.0: + gnf4_router_topk, gnf4_moe_combine, gnf4_grouped_dgrad */
 
 /* Exported entry points (the library is built with hidden default visibility). */
 #if defined(__GNUC__)

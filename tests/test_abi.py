@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert gnf4.gnf4_version() == 100
+    assert gnf4.gnf4_version() == 110
     assert gnf4.gnf4_status_string(0) == "GNF4_OK"
     assert "HOST_POINTER" in gnf4.gnf4_status_string(2)
     assert gnf4.gnf4_status_string(99) == "GNF4_ERR_UNKNOWN"
