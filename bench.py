@@ -7,13 +7,18 @@ One step = one pass of the whole hot path over one batch of synthetic input:
 with sizes/expert_ids handed from the sort to the GEMMs on the device.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload olmoe|tiny|qwen3_30b_a3b|gpt_oss_120b|mixtral_8x22b]
+                    [--workload mixtral_8x22b|olmoe|tiny|qwen3_30b_a3b|gpt_oss_120b]
+                    [--only]
 
-Prints ONE JSON line on rank 0. `value` is whole-job throughput (all ranks)
-of the metric: HBM GB/s for the decode workloads (algorithmic bytes: touched
-expert weights + absmax + x + y + sort I/O), TFLOP/s for the prefill workload
-(2*M*N*K per GEMM). With N > 1 every rank runs an independent replica (the
-decode path does not shard; weak scaling), the timed region is bracketed by a
+Prints ONE JSON line on rank 0. The headline workload (default: the
+Mixtral-8x22B-shaped prefill, the largest single-GPU configuration) is timed
+for exactly K steps; `value` is its whole-job throughput (all ranks) of the
+metric: TFLOP/s for the prefill workload (2*M*N*K per GEMM), HBM GB/s for the
+decode workloads (algorithmic bytes: touched expert weights + absmax + x + y +
+sort I/O). On one GPU the other four configurations follow (unless --only),
+each with its own step throughput, per-GEMM roofline and oracle baseline under
+"configs". With N > 1 every rank runs an independent replica of the headline
+(the path does not shard; weak scaling), the timed region is bracketed by a
 barrier + synchronize and its time is the max over ranks.
 
 Timing: CUDA events on the launching stream. Each step is a CUDA graph of the
@@ -47,7 +52,7 @@ import synth  # noqa: E402
 METRIC = "grouped NF4 GEMM: HBM GB/s & % roofline (decode); TFLOPS & % peak (prefill)"
 L2_BYTES = 126 * 1024 * 1024
 DEFAULT_STEPS = {"tiny": 20000, "olmoe": 20000, "qwen3_30b_a3b": 5000, "gpt_oss_120b": 500,
-                 "mixtral_8x22b": 100}
+                 "mixtral_8x22b": 150}
 
 
 # ----------------------------------------------------------------- helpers
@@ -154,6 +159,16 @@ def _cuda_driver():
     lib.cuEventElapsedTime.restype = ctypes.c_int
     lib.cuEventCreate.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
     lib.cuEventCreate.restype = ctypes.c_int
+    lib.cuGraphGetNodes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]
+    lib.cuGraphGetNodes.restype = ctypes.c_int
+    lib.cuGraphNodeGetType.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+    lib.cuGraphNodeGetType.restype = ctypes.c_int
+    lib.cuGraphKernelNodeGetParams = getattr(lib, "cuGraphKernelNodeGetParams_v2",
+                                             lib.cuGraphKernelNodeGetParams)
+    lib.cuGraphKernelNodeGetParams.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.cuGraphKernelNodeGetParams.restype = ctypes.c_int
+    lib.cuFuncGetName.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.c_void_p]
+    lib.cuFuncGetName.restype = ctypes.c_int
     return lib
 
 
@@ -188,14 +203,15 @@ def max_over_ranks(x, world, device):
 
 
 # ------------------------------------------------------------------ problem
-class Problem:
-    """Device-resident inputs for one workload (seeded, synthetic)."""
+class HostProblem:
+    """Seeded synthetic inputs of one workload as host arrays, with the
+    algorithmic work per step. Imports nothing from the product library, so
+    the reference arm (the oracle on the host cores) never loads it."""
 
-    def __init__(self, name, seed=0, replicas=None, device="cuda"):
+    def __init__(self, name, seed=0):
         self.w = synth.WORKLOADS[name]
         w = self.w
         self.name = name
-        self.device = device
         self.topk_np = synth.routing(w, seed)
         self.U = int(np.unique(self.topk_np).size)
         self.gemms = []
@@ -203,19 +219,52 @@ class Problem:
         for g in w.gemms:
             packed, absmax = synth.random_packed_stack(w.E, g.N, g.K, seed=seed, which=g.name)
             x = synth.activations_bf16(w.M, g.K, seed=seed, which=g.name)
-            self.gemms.append(dict(g=g, packed_np=packed, absmax_np=absmax, x_np=x))
+            n_out = g.N // 2 if g.swiglu else g.N
+            self.gemms.append(dict(
+                g=g, packed_np=packed, absmax_np=absmax, x_np=x, n_out=n_out,
+                bytes=self.U * g.N * g.K * 9 // 16 + w.M * g.K * 2 + w.M * n_out * 2,
+                flops=2 * w.M * g.N * g.K))
             touched_bytes += self.U * g.N * g.K * 9 // 16
-        if replicas is None:
-            replicas = 1 if touched_bytes > 2 * L2_BYTES else 1 + -(-int(1.5 * L2_BYTES) // touched_bytes)
-        self.R = replicas
+        # weight-stack replicas rotated per step so that a step never finds its
+        # weights in L2 (none needed when a step touches more than 2x L2)
+        self.R = (1 if touched_bytes > 2 * L2_BYTES
+                  else 1 + -(-int(1.5 * L2_BYTES) // touched_bytes))
+        S = w.T * w.top_k
+        self.align_bytes = S * 4 + S * 4 + 2 * w.E * 4 + 4
+        self.step_bytes = self.align_bytes + sum(d["bytes"] for d in self.gemms)
+        self.step_flops = sum(d["flops"] for d in self.gemms)
+        self.prefill = w.regime == "prefill"
+
+    def describe(self):
+        w = self.w
+        return {
+            "workload": f"{w.name}: {w.description}",
+            "E": w.E, "top_k": w.top_k, "tokens": w.T, "rows": w.M,
+            "gemms": [f"{d['g'].name} K={d['g'].K} N={d['g'].N}" + (" +SwiGLU" if d['g'].swiglu else "")
+                      for d in self.gemms],
+            "touched_experts": self.U,
+            "weights": "uniform random NF4 codes, absmax U[0.04,0.06] (values do not affect timing)",
+            "l2": (f"{self.R} weight-stack replicas rotated per step "
+                   f"(touched bytes of the other replicas > L2)" if self.R > 1 else
+                   "touched weights per step > 2x L2 (no replica needed)"),
+        }
+
+
+class Problem(HostProblem):
+    """HostProblem plus its device tensors and the step's C-ABI calls."""
+
+    def __init__(self, name, seed=0, device="cuda"):
+        super().__init__(name, seed)
+        w = self.w
+        self.device = device
+        import grouped_nf4_w4a16_b200 as gnf4
+        self.gnf4 = gnf4
         self.topk = torch.from_numpy(self.topk_np).to(device)
         S = w.T * w.top_k
         self.sorted_idx = torch.empty(S, dtype=torch.int32, device=device)
         self.sizes = torch.empty(w.E, dtype=torch.int32, device=device)
         self.expert_ids = torch.empty(w.E, dtype=torch.int32, device=device)
         self.num_groups = torch.empty(1, dtype=torch.int32, device=device)
-        import grouped_nf4_w4a16_b200 as gnf4
-        self.gnf4 = gnf4
         self.ws_align = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_MOE_ALIGN, S, E=w.E), device)
         for d in self.gemms:
             g = d["g"]
@@ -224,21 +273,10 @@ class Problem:
             d["W"] = [wd] + [wd.clone() for _ in range(self.R - 1)]
             d["A"] = [ad] + [ad.clone() for _ in range(self.R - 1)]
             d["x"] = torch.from_numpy(d["x_np"].view(np.int16)).to(device).view(torch.bfloat16)
-            n_out = g.N // 2 if g.swiglu else g.N
-            d["y"] = torch.empty((w.M, n_out), dtype=torch.bfloat16, device=device)
+            d["y"] = torch.empty((w.M, d["n_out"]), dtype=torch.bfloat16, device=device)
             d["ws"] = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(
                 gnf4.GNF4_OP_GROUPED_GEMM, w.M, g.N, g.K, w.E, w.E), device)
             d["epi"] = gnf4.GNF4_EPI_SWIGLU if g.swiglu else gnf4.GNF4_EPI_NONE
-        # algorithmic work per step
-        self.align_bytes = S * 4 + S * 4 + 2 * w.E * 4 + 4
-        for d in self.gemms:
-            g = d["g"]
-            n_out = g.N // 2 if g.swiglu else g.N
-            d["bytes"] = self.U * g.N * g.K * 9 // 16 + w.M * g.K * 2 + w.M * n_out * 2
-            d["flops"] = 2 * w.M * g.N * g.K
-        self.step_bytes = self.align_bytes + sum(d["bytes"] for d in self.gemms)
-        self.step_flops = sum(d["flops"] for d in self.gemms)
-        self.prefill = w.regime == "prefill"
 
     def launch(self, r, events=None, drv=None, stream=None):
         """Enqueue one step with weight replica r (optionally recording events)."""
@@ -260,42 +298,59 @@ class Problem:
                                    epilogue=d["epi"], y=d["y"], workspace=d["ws"])
             ev(2 + i)
 
-    def describe(self):
-        w = self.w
-        return {
-            "workload": f"{w.name}: {w.description}",
-            "E": w.E, "top_k": w.top_k, "tokens": w.T, "rows": w.M,
-            "gemms": [f"{d['g'].name} K={d['g'].K} N={d['g'].N}" + (" +SwiGLU" if d['g'].swiglu else "")
-                      for d in self.gemms],
-            "touched_experts": self.U,
-            "weights": "uniform random NF4 codes, absmax U[0.04,0.06] (values do not affect timing)",
-            "l2": (f"{self.R} weight-stack replicas rotated per step "
-                   f"(touched bytes of the other replicas > L2)" if self.R > 1 else
-                   "touched weights per step > 2x L2 (no replica needed)"),
-            "graph": "each step is one CUDA graph of the C-ABI calls",
-        }
+    def free(self):
+        for d in self.gemms:
+            for k in ("W", "A", "x", "y", "ws"):
+                d.pop(k, None)
+
+
+def graph_kernels(drv, graph):
+    """Names of the kernel nodes of a captured (kept) CUDA graph."""
+    n = ctypes.c_size_t(0)
+    h = ctypes.c_void_p(graph.raw_cuda_graph())
+    if drv.cuGraphGetNodes(h, None, ctypes.byref(n)) != 0:
+        return None
+    nodes = (ctypes.c_void_p * n.value)()
+    if drv.cuGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+        return None
+    names = []
+    for i in range(n.value):
+        t = ctypes.c_int(-1)
+        if drv.cuGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) != 0:
+            return None
+        if t.value != 0:          # CU_GRAPH_NODE_TYPE_KERNEL
+            continue
+        params = (ctypes.c_byte * 256)()   # CUDA_KERNEL_NODE_PARAMS (v2); func first
+        if drv.cuGraphKernelNodeGetParams(ctypes.c_void_p(nodes[i]), params) != 0:
+            names.append("?")
+            continue
+        func = ctypes.c_void_p.from_buffer(params).value
+        nm = ctypes.c_char_p()
+        ok = drv.cuFuncGetName(ctypes.byref(nm), ctypes.c_void_p(func)) == 0 and nm.value
+        names.append(nm.value.decode() if ok else "?")
+    return names
 
 
 # --------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    prob = Problem(args.workload, seed=0, device=dev)
-    stream = torch.cuda.Stream(device=dev)
-    drv = _cuda_driver()
+def run_ours(name, steps, warmup, world, dev, stream, drv, with_e2e=True):
+    """Capture, warm up and time `steps` steps of workload `name`. Returns a
+    dict with the Problem, the timed ms (max over ranks), per-kernel ms, the
+    clocks seen, the end-to-end timing and the kernels of one step graph."""
+    prob = Problem(name, seed=0, device=dev)
     nk = 1 + len(prob.gemms)
     # Per weight replica: a plain step graph (timed; consecutive kernels keep
     # their programmatic launch edges) and a copy with external event nodes
-    # around each kernel (per-kernel durations, replayed after the timing).
+    # around each C-ABI call (per-call durations, replayed after the timing).
     graphs, ev_graphs, evs = [], [], []
     with torch.cuda.stream(stream):
         for r in range(prob.R):      # eager warm-up (sets kernel attributes, first-call work)
             prob.launch(r)
         torch.cuda.synchronize()
         for r in range(prob.R):
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g, stream=stream):
                 prob.launch(r)
+            g.instantiate()
             graphs.append(g)
             e = [_new_event(drv) for _ in range(nk + 1)]
             ge = torch.cuda.CUDAGraph()
@@ -304,13 +359,13 @@ def run_ours(args, rank, world, local_rank):
             ev_graphs.append(ge)
             evs.append(e)
     torch.cuda.synchronize()
-    launches_per_step = nk
+    step_kernels = graph_kernels(drv, graphs[0])
 
-    clocks = Clocks(local_rank)
+    clocks = Clocks(dev.index if dev.index is not None else 0)
     clocks.start()
     time.sleep(0.3)
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
+        for i in range(warmup):
             graphs[i % prob.R].replay()
         # keep the GPU busy for ~0.5 s before timing so clocks settle
         t_end = time.time() + 0.5
@@ -326,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
     t0 = time.time()
     start.record(stream)
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
+        for i in range(steps):
             graphs[i % prob.R].replay()
     stop.record(stream)
     stop.synchronize()
@@ -348,8 +403,8 @@ def run_ours(args, rank, world, local_rank):
     t2 = time.time()
     clk = clocks.stop(t0, t2)
 
-    # per-kernel durations: external event nodes of the last of a few replays
-    # of each replica's instrumented graph (kernels serialised by the nodes)
+    # per-call durations: external event nodes of the last of a few replays
+    # of each replica's instrumented graph (calls serialised by the nodes)
     with torch.cuda.stream(stream):
         for _ in range(3):
             for ge in ev_graphs:
@@ -362,17 +417,49 @@ def run_ours(args, rank, world, local_rank):
     kern_ms = [sum(v) / len(v) for v in per_kernel]   # NaN if a timestamp was missing
 
     ms = max_over_ranks(ms, world, dev)
+    e2e = None
+    if with_e2e:
+        # host (pinned) inputs -> device, the C-ABI calls, results -> host
+        e2e = run_e2e(prob, stream, max(3, min(steps, 2000) // 10))
+        e2e = (max_over_ranks(e2e[0], world, dev),) + tuple(e2e[1:])
+    del graphs, ev_graphs
+    return dict(prob=prob, ms=ms, kern_ms=kern_ms, clocks=clk, e2e=e2e,
+                step_kernels=step_kernels, steps=steps, warmup=warmup)
 
-    # end to end: host (pinned) inputs -> device, the C-ABI calls, results -> host
-    e2e = run_e2e(prob, stream, max(3, min(args.steps, 2000) // 10))
-    e2e = (max_over_ranks(e2e[0], world, dev),) + tuple(e2e[1:])
-    # the glue entry points last: an error there is reported in the line
-    # instead of costing the step's numbers
-    try:
-        glue = time_glue(prob, stream)
-    except Exception as exc:   # noqa: BLE001
-        glue = {"error": f"{type(exc).__name__}: {exc}"}
-    return prob, ms, kern_ms, clk, e2e, launches_per_step, glue
+
+def roofline(prob, d, k_ms, pk):
+    """Roofline of one GEMM launch: algorithmic bytes (decode, HBM-bound) or
+    FLOPs (prefill, tensor-bound) per launch over its event-timed duration."""
+    kernel = "prefill_gemm_kernel" if prob.prefill else "decode_gemm_kernel"
+    if prob.prefill:
+        # timed inside seconds of back-to-back steps: the sustained bf16 figure
+        achieved = d["flops"] / (k_ms / 1e3) / 1e12
+        peak, which = pk["bf16_tflops_sustained"], "bf16_tflops_sustained"
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "frac_of_nominal_2250": achieved / 2250.0}
+    else:
+        achieved = d["bytes"] / (k_ms / 1e3) / 1e9
+        peak, which = pk["hbm_gbs"], "hbm_gbs"
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+    roof["traffic"] = traffic_for(kernel.replace("_kernel", "") if prob.prefill else kernel,
+                                  prob.name, d["g"].name)
+    roof["kernel"] = f"{kernel} ({d['g'].name} launch)"
+    roof["algorithmic_per_launch"] = d["flops"] if prob.prefill else d["bytes"]
+    roof["launch_ms"] = k_ms
+    roof["peak_source"] = (f"measured {which} (MEASURED_PEAKS.json)" if pk["source"] == "measured"
+                           else f"fallback {which}")
+    return roof
+
+
+def kernels_entry(prob, kern_ms):
+    kernels = {"moe_align": {"ms": kern_ms[0]}}
+    for i, d in enumerate(prob.gemms):
+        entry = {"ms": kern_ms[1 + i], "GB/s": d["bytes"] / (kern_ms[1 + i] / 1e3) / 1e9}
+        if prob.prefill:
+            entry["TFLOP/s"] = d["flops"] / (kern_ms[1 + i] / 1e3) / 1e12
+        kernels[d["g"].name] = entry
+    return kernels
 
 
 def time_glue(prob, stream, reps=50):
@@ -521,11 +608,11 @@ def metric_value(prob, sec_per_step, n_ranks=1):
 
 
 def run_reference(args, rank, world):
+    """The oracle (plain C, fp64) on the host cores, on our arm's workload,
+    metric and config. Host-only: the product library is never imported."""
     if rank != 0:
         return None
-    # the oracle runs on the host cores; its inputs are the same seeded arrays
-    prob = Problem(args.workload, seed=0, replicas=1,
-                   device="cuda" if torch.cuda.is_available() else "cpu")
+    prob = HostProblem(args.workload, seed=0)
     budget = max(3.0, min(60.0, 2.0 * (args.steps + args.warmup)))
     sec, sample, threads = oracle_step_sample(prob, budget)
     val, unit = metric_value(prob, sec)
@@ -537,22 +624,54 @@ def run_reference(args, rank, world):
         "cpu_baseline": {"value": val, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "timing": "the oracle on the host cores (no GPU, no graph)",
     }
-    line["config"]["graph"] = "none: the oracle runs on the host cores"
-    line["config"]["l2"] = "not applicable (host run)"
+    line["config"]["parallelism"] = "single GPU" if world <= 1 else f"replicas x{world}"
     return line
 
 
+def side_record(res, pk, cpu_budget, glue):
+    """What one non-headline workload contributes to the line: its step
+    throughput, per-call times, per-GEMM roofline, clocks and oracle baseline."""
+    prob = res["prob"]
+    sec = res["ms"] / 1e3 / res["steps"]
+    val, unit = metric_value(prob, sec)
+    rec = {"value": val, "unit": unit, "ms_per_step": res["ms"] / res["steps"],
+           "steps": res["steps"], "warmup": res["warmup"], "config": prob.describe(),
+           "kernels": kernels_entry(prob, res["kern_ms"]),
+           "roofline": {d["g"].name: roofline(prob, d, res["kern_ms"][1 + i], pk)
+                        for i, d in enumerate(prob.gemms)},
+           "step_kernels": res["step_kernels"], "clocks": res["clocks"]}
+    if glue is not None:
+        rec["glue"] = glue
+    if cpu_budget > 0:
+        sec_cpu, sample, threads = oracle_step_sample(prob, cpu_budget)
+        v, u = metric_value(prob, sec_cpu)
+        rec["cpu_baseline"] = {"value": v, "unit": u, "cores": threads, "kind": "oracle",
+                               "sample": sample}
+    return rec
+
+
 # --------------------------------------------------------------------- main
+HEADLINE = "mixtral_8x22b"
+SIDE_STEPS = {"tiny": 5000, "olmoe": 5000, "qwen3_30b_a3b": 2000, "gpt_oss_120b": 300,
+              "mixtral_8x22b": 50}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="olmoe", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=list(synth.WORKLOADS),
+                    help="the headline workload (default: the largest single-GPU config)")
+    ap.add_argument("--only", action="store_true",
+                    help="time only the headline workload (skip the other configs)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
-                    help="seconds of CPU time for the oracle baseline sample")
+                    help="seconds of CPU time for the headline's oracle baseline sample")
+    ap.add_argument("--side-cpu-budget", type=float, default=5.0,
+                    help="seconds of CPU time for each other config's oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
@@ -564,74 +683,65 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # rank 0 alone times the oracle; the other ranks exit without work
+        line = run_reference(args, rank, world)
+        if rank == 0:
+            print(json.dumps(line))
+        return
+
     if world > 1:
         timeout = __import__("datetime").timedelta(seconds=120)
         if torch.cuda.is_available():
             torch.cuda.set_device(local_rank)
             torch.distributed.init_process_group(
                 "nccl", device_id=torch.device("cuda", local_rank), timeout=timeout)
-        else:   # host-only runs (the reference arm, tests): gloo
+        else:   # host-only runs (tests): gloo
             torch.distributed.init_process_group("gloo", timeout=timeout)
-
-    if args.impl == "reference":
-        line = run_reference(args, rank, world)
-        if rank == 0:
-            print(json.dumps(line))
-        if world > 1:
-            torch.distributed.destroy_process_group()
-        return
 
     import grouped_nf4_w4a16_b200 as gnf4
     gnf4.load_library()    # fails loudly if the CUDA library is missing
-    prob, ms, kern_ms, clk, e2e, lps, glue = run_ours(args, rank, world, local_rank)
-    sec = ms / 1e3 / args.steps
-    val, unit = metric_value(prob, sec, world)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    drv = _cuda_driver()
     pk = peaks()
 
-    # roofline of the dominant kernel: the gate_up grouped GEMM launch
-    d0 = prob.gemms[0]
-    k_ms = kern_ms[1]
-    kernel = "prefill_gemm" if prob.prefill else "decode_gemm_kernel"
-    if prob.prefill:
-        # timed inside seconds of back-to-back steps: the sustained bf16 figure
-        achieved = d0["flops"] / (k_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": traffic_for(kernel, prob.name, "gate_up")}
-    else:
-        achieved = d0["bytes"] / (k_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(kernel, prob.name, "gate_up")}
-    roof["kernel"] = f"{kernel} ({d0['g'].name} launch)"
-    roof["algorithmic_per_launch"] = d0["flops"] if prob.prefill else d0["bytes"]
-    roof["launch_ms"] = k_ms
-    which = "bf16_tflops_sustained" if prob.prefill else "hbm_gbs"
-    roof["peak_source"] = (f"measured {which} (MEASURED_PEAKS.json)" if pk["source"] == "measured"
-                           else f"fallback {which}")
+    res = run_ours(args.workload, args.steps, args.warmup, world, dev, stream, drv)
+    prob = res["prob"]
+    ms, kern_ms = res["ms"], res["kern_ms"]
+    sec = ms / 1e3 / args.steps
+    val, unit = metric_value(prob, sec, world)
+    # the glue entry points after the step's numbers: an error there is
+    # reported in the line instead of costing them
+    try:
+        glue = time_glue(prob, stream)
+    except Exception as exc:   # noqa: BLE001
+        glue = {"error": f"{type(exc).__name__}: {exc}"}
 
-    kernels = {"moe_align": {"ms": kern_ms[0]}}
-    for i, d in enumerate(prob.gemms):
-        entry = {"ms": kern_ms[1 + i], "GB/s": d["bytes"] / (kern_ms[1 + i] / 1e3) / 1e9}
-        if prob.prefill:
-            entry["TFLOP/s"] = d["flops"] / (kern_ms[1 + i] / 1e3) / 1e12
-        kernels[d["g"].name] = entry
-
-    e2e_ms, h2d, d2h, e2e_steps = e2e
+    roofs = {d["g"].name: roofline(prob, d, kern_ms[1 + i], pk) for i, d in enumerate(prob.gemms)}
+    e2e_ms, h2d, d2h, e2e_steps = res["e2e"]
     e2e_val, _ = metric_value(prob, e2e_ms / 1e3, world)
+    kpl = len(res["step_kernels"]) if res["step_kernels"] is not None else None
     line = {
         "metric": METRIC, "value": val, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": prob.describe(),
-        "roofline": roof,
-        "kernels": kernels,
+        # the dominant kernel: the gate_up GEMM launch (the larger of the two)
+        "roofline": roofs[prob.gemms[0]["g"].name],
+        "roofline_per_gemm": roofs,
+        "kernels": kernels_entry(prob, kern_ms),
         "glue": glue,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "how": "eager C-ABI calls; pinned host inputs copied in and results copied out every step"},
-        "gpu_launches": lps * args.steps,
-        "clocks": clk,
+        "gpu_launches": kpl * args.steps if kpl is not None else None,
+        "step_kernels": res["step_kernels"],
+        "timing": ("each step is one CUDA graph of the C-ABI calls (moe_align, then each GEMM); "
+                   "per-call times from event nodes in a copy of the graph"),
+        "clocks": res["clocks"],
     }
     line["config"]["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -639,6 +749,32 @@ def main():
         v, u = metric_value(prob, sec_cpu)
         line["cpu_baseline"] = {"value": v, "unit": u, "cores": threads, "kind": "oracle",
                                 "sample": sample}
+    prob.free()
+    del res, prob
+    torch.cuda.empty_cache()
+
+    # the other configurations, one GPU only: each one's step throughput,
+    # per-GEMM roofline and oracle baseline under "configs"
+    if world == 1 and not args.only:
+        others = {}
+        for name in synth.WORKLOADS:
+            if name == args.workload:
+                continue
+            try:
+                r = run_ours(name, SIDE_STEPS[name], max(3, SIDE_STEPS[name] // 20), 1, dev,
+                             stream, drv, with_e2e=False)
+                try:
+                    g = time_glue(r["prob"], stream)
+                except Exception as exc:   # noqa: BLE001
+                    g = {"error": f"{type(exc).__name__}: {exc}"}
+                others[name] = side_record(r, pk, 0.0 if args.no_cpu_baseline
+                                           else args.side_cpu_budget, g)
+                r["prob"].free()
+                del r
+                torch.cuda.empty_cache()
+            except Exception as exc:   # noqa: BLE001
+                others[name] = {"error": f"{type(exc).__name__}: {exc}"}
+        line["configs"] = others
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

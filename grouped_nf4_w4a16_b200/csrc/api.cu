@@ -46,6 +46,54 @@ gnf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GNF4_OK : GNF4_
 constexpr int64_t kPrefillMeanRows = 64;
 
 }  // namespace
+
+gnf4_status check_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *absmax,
+                               const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                               int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                               int32_t epilogue, int32_t mode, uint16_t *y, GemmArgs *out,
+                               int32_t *use_out) {
+  *use_out = -1;
+  if (!x || !w || !absmax || !sizes || !expert_ids || !y) return GNF4_ERR_INVALID_ARGUMENT;
+  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (epilogue != GNF4_EPI_NONE && epilogue != GNF4_EPI_SWIGLU) return GNF4_ERR_INVALID_ARGUMENT;
+  if (mode != GNF4_MODE_AUTO && mode != GNF4_MODE_DECODE && mode != GNF4_MODE_PREFILL)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  // tensor-copy coordinates are 32-bit: every weight row index a copy can
+  // start at (up to one expert plus one box past the stack) must fit
+  if (static_cast<int64_t>(E) * N + N + 256 >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return GNF4_OK;   // nothing to launch (*use_out stays -1)
+  if (!is_device_pointer(x) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
+      !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(y))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(x, 32) || !aligned(w, 32) || !aligned(y, 32) || !aligned(absmax, 4) ||
+      !aligned(sizes, 4) || !aligned(expert_ids, 4))
+    return GNF4_ERR_MISALIGNED;
+  GemmArgs &a = *out;
+  a.x = x; a.w = w; a.absmax = absmax; a.sizes = sizes; a.expert_ids = expert_ids;
+  a.G = G; a.M = M; a.N = N; a.K = K; a.E = E; a.swiglu = (epilogue == GNF4_EPI_SWIGLU);
+  a.y = y; a.workspace = nullptr; a.ws_bytes = 0;
+  int32_t use = mode;
+  if (use == GNF4_MODE_AUTO) {
+    const int64_t groups = G < E ? G : E;
+    // the tensor-core kernel has no fused SwiGLU yet: SwiGLU stays on the decode kernel
+    use = (M > kPrefillMeanRows * groups && epilogue == GNF4_EPI_NONE) ? GNF4_MODE_PREFILL
+                                                                       : GNF4_MODE_DECODE;
+  }
+  *use_out = use;
+  return GNF4_OK;
+}
+
+gnf4_status launch_grouped_gemm(const GemmArgs &a, int32_t use, cudaStream_t s) {
+  const cudaError_t e =
+      use == GNF4_MODE_PREFILL ? launch_prefill_gemm(a, s) : launch_decode_gemm(a, s);
+  if (e == cudaErrorNotSupported) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
+}
+
 }  // namespace gnf4
 
 using namespace gnf4;
@@ -116,49 +164,21 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
                               int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
                               int32_t epilogue, int32_t mode, uint16_t *y, void *workspace,
                               size_t ws_bytes, gnf4_stream_t stream) {
-  if (!x || !w || !absmax || !sizes || !expert_ids || !y || !workspace)
-    return GNF4_ERR_INVALID_ARGUMENT;
-  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
-  if (epilogue != GNF4_EPI_NONE && epilogue != GNF4_EPI_SWIGLU) return GNF4_ERR_INVALID_ARGUMENT;
-  if (mode != GNF4_MODE_AUTO && mode != GNF4_MODE_DECODE && mode != GNF4_MODE_PREFILL)
-    return GNF4_ERR_INVALID_ARGUMENT;
-  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  // tensor-copy coordinates are 32-bit: every weight row index a copy can
-  // start at (up to one expert plus one box past the stack) must fit
-  if (static_cast<int64_t>(E) * N + N + 256 >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0) return GNF4_OK;
-  if (!is_device_pointer(x) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
-      !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(y) ||
-      !is_device_pointer(workspace))
-    return GNF4_ERR_HOST_POINTER;
-  if (!aligned(x, 32) || !aligned(w, 32) || !aligned(y, 32) || !aligned(workspace, 32) ||
-      !aligned(absmax, 4) || !aligned(sizes, 4) || !aligned(expert_ids, 4))
-    return GNF4_ERR_MISALIGNED;
+  if (!workspace) return GNF4_ERR_INVALID_ARGUMENT;
   GemmArgs a;
-  a.x = x; a.w = w; a.absmax = absmax; a.sizes = sizes; a.expert_ids = expert_ids;
-  a.G = G; a.M = M; a.N = N; a.K = K; a.E = E; a.swiglu = (epilogue == GNF4_EPI_SWIGLU);
-  a.y = y; a.workspace = workspace; a.ws_bytes = ws_bytes;
-
-  int32_t use = mode;
-  if (use == GNF4_MODE_AUTO) {
-    const int64_t groups = G < E ? G : E;
-    // the tensor-core kernel has no fused SwiGLU yet: SwiGLU stays on the decode kernel
-    use = (M > kPrefillMeanRows * groups && epilogue == GNF4_EPI_NONE) ? GNF4_MODE_PREFILL
-                                                                       : GNF4_MODE_DECODE;
-  }
+  int32_t use = 0;
+  const gnf4_status st = check_grouped_gemm(x, w, absmax, sizes, expert_ids, G, M, N, K, E,
+                                            blocksize, epilogue, mode, y, &a, &use);
+  if (st != GNF4_OK || use < 0) return st;
+  if (!is_device_pointer(workspace)) return GNF4_ERR_HOST_POINTER;
+  if (!aligned(workspace, 32)) return GNF4_ERR_MISALIGNED;
+  a.workspace = workspace;
+  a.ws_bytes = ws_bytes;
   // the workspace the chosen kernel needs (gnf4_workspace_bytes covers every mode)
-  const int32_t swg = epilogue == GNF4_EPI_SWIGLU ? 1 : 0;
-  const size_t need = use == GNF4_MODE_PREFILL ? prefill_workspace_bytes(M, N, K, G, swg)
-                                               : decode_workspace_bytes(M, N, K, G, swg);
+  const size_t need = use == GNF4_MODE_PREFILL ? prefill_workspace_bytes(M, N, K, G, a.swiglu)
+                                               : decode_workspace_bytes(M, N, K, G, a.swiglu);
   if (ws_bytes < need) return GNF4_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      use == GNF4_MODE_PREFILL ? launch_prefill_gemm(a, s) : launch_decode_gemm(a, s);
-  if (e == cudaErrorNotSupported) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  return from_cuda(e);
+  return launch_grouped_gemm(a, use, reinterpret_cast<cudaStream_t>(stream));
 }
 
 gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,

@@ -63,6 +63,18 @@ cudaError_t launch_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const flo
                                  int64_t M, int32_t N, int32_t K, int32_t E, uint16_t *dx,
                                  WsHeader *hdr, cudaStream_t stream);
 
+// ---- entry-point plumbing shared by gnf4_grouped_gemm and its no-allocation
+// variant (api.cu): every host-side check except those of the workspace, in
+// the order gnf4_grouped_gemm reports them, filling `out` (workspace unset)
+// and the kernel to run (*use_out = GNF4_MODE_DECODE or GNF4_MODE_PREFILL;
+// -1 with GNF4_OK when M == 0 and there is nothing to launch).
+gnf4_status check_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *absmax,
+                               const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                               int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
+                               int32_t epilogue, int32_t mode, uint16_t *y, GemmArgs *out,
+                               int32_t *use_out);
+gnf4_status launch_grouped_gemm(const GemmArgs &a, int32_t use, cudaStream_t s);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

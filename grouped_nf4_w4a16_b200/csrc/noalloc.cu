@@ -55,31 +55,28 @@ extern "C" gnf4_status gnf4_grouped_gemm_noalloc(const uint16_t *x, const uint8_
                                                  int32_t N, int32_t K, int32_t E,
                                                  int32_t blocksize, int32_t epilogue, uint16_t *y,
                                                  gnf4_stream_t stream) {
-  // Shape checks that decide how much scratch the call needs; every other
-  // check is made by gnf4_grouped_gemm below, unchanged.
-  if (!x || !w || !absmax || !sizes || !expert_ids || !y) return GNF4_ERR_INVALID_ARGUMENT;
-  if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
-  if (epilogue != GNF4_EPI_NONE && epilogue != GNF4_EPI_SWIGLU) return GNF4_ERR_INVALID_ARGUMENT;
-  if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (epilogue == GNF4_EPI_SWIGLU && (N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0) return GNF4_OK;
+  // Every argument check of gnf4_grouped_gemm (decode mode) comes first, so a
+  // refused call puts no work on the caller's stream.
+  GemmArgs a;
+  int32_t use = 0;
+  const gnf4_status st = check_grouped_gemm(x, w, absmax, sizes, expert_ids, G, M, N, K, E,
+                                            blocksize, epilogue, GNF4_MODE_DECODE, y, &a, &use);
+  if (st != GNF4_OK || use < 0) return st;
 
-  // the decode kernel's workspace (the 256-byte status header with the
-  // current kernel) must fit the scratch array
-  const size_t need = decode_workspace_bytes(M, N, K, G, epilogue == GNF4_EPI_SWIGLU ? 1 : 0);
+  // the decode kernel's workspace must fit the scratch array
+  const size_t need = decode_workspace_bytes(M, N, K, G, a.swiglu);
   if (need == 0 || need > GNF4_NOALLOC_SCRATCH_BYTES) return GNF4_ERR_SCRATCH_LIMIT;
 
   void *scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return GNF4_ERR_CUDA;
 
-  // The array still holds the previous call's contents: the status word must
-  // start at zero.
-  const size_t clear =
-      decode_zero_prefix_bytes(M, N, G, epilogue == GNF4_EPI_SWIGLU ? 1 : 0);
+  // The array still holds the previous call's contents: the part the kernel
+  // needs at zero (status word, counters) is cleared on the caller's stream.
+  const size_t clear = decode_zero_prefix_bytes(M, N, G, a.swiglu);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, clear, s) != cudaSuccess) return GNF4_ERR_CUDA;
 
-  return gnf4_grouped_gemm(x, w, absmax, sizes, expert_ids, G, M, N, K, E, blocksize, epilogue,
-                           GNF4_MODE_DECODE, y, scratch, GNF4_NOALLOC_SCRATCH_BYTES, stream);
+  a.workspace = scratch;
+  a.ws_bytes = GNF4_NOALLOC_SCRATCH_BYTES;
+  return launch_grouped_gemm(a, GNF4_MODE_DECODE, s);
 }

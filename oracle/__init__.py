@@ -22,7 +22,9 @@ grouped_nf4_gemm 0.1.0, opening section, unless stated):
 * :func:`swiglu_f64` -- silu(gate) * up on the gate_up output (package page
   "grouped-nf4-gemm", "Owns": the decode glue includes swiglu).
 * :func:`baseline_bf16` -- dequantise-to-bf16 then fp32-accumulated matmul,
-  the fidelity comparator of the page's "The claim" section.
+  the fidelity comparator of the page's "The claim" section;
+  :func:`baseline_swiglu_bf16` -- that baseline's SwiGLU: silu(gate) * up in
+  fp32 on its bf16 gate_up output, rounded once to bf16.
 * :func:`grouped_dgrad_f64` -- the gradient of the grouped GEMM with respect
   to its activations, dx = dy . W per group, in fp64 (package page
   "grouped-nf4-gemm", header block, "Owns": the grouped packed GEMM and its
@@ -84,13 +86,14 @@ def _load():
         lib.oracle_grouped_gemm_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
         lib.oracle_swiglu_f64.argtypes = [P, i64, i32, P]
         lib.oracle_baseline_bf16.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
+        lib.oracle_baseline_swiglu_bf16.argtypes = [P, i64, i32, P]
         lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, P, P]
         lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i32, P]
         lib.oracle_grouped_dgrad_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P]
         for name in ("oracle_quantize_nf4", "oracle_dequant_f32", "oracle_dequant_bf16",
                      "oracle_moe_align", "oracle_grouped_gemm_f64", "oracle_swiglu_f64",
-                     "oracle_baseline_bf16", "oracle_router_topk", "oracle_moe_combine",
-                     "oracle_grouped_dgrad_f64"):
+                     "oracle_baseline_bf16", "oracle_baseline_swiglu_bf16", "oracle_router_topk",
+                     "oracle_moe_combine", "oracle_grouped_dgrad_f64"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -221,6 +224,16 @@ def baseline_bf16(x: np.ndarray, w: np.ndarray, absmax: np.ndarray, sizes: np.nd
         _p(x), _p(w), _p(absmax), _p(sizes), _p(expert_ids), sizes.size, M, N, K, E,
         None if rows is None else _p(rows), nrows, _p(y)))
     return y
+
+
+def baseline_swiglu_bf16(yb: np.ndarray) -> np.ndarray:
+    """SwiGLU of the baseline's bf16 gate_up output (bf16 bits [M, N]) in fp32,
+    rounded once: bf16 bits [M, N/2]."""
+    yb = np.ascontiguousarray(yb, dtype=np.uint16)
+    M, N = yb.shape
+    out = np.empty((M, N // 2), dtype=np.uint16)
+    _check(_load().oracle_baseline_swiglu_bf16(_p(yb), M, N, _p(out)))
+    return out
 
 
 def quantized_stack(E: int, N: int, K: int, weights_fn) -> Tuple[np.ndarray, np.ndarray]:

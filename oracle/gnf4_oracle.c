@@ -310,6 +310,28 @@ int oracle_baseline_bf16(const uint16_t *x, const uint8_t *w, const float *absma
     return ORC_OK;
 }
 
+/* SwiGLU of the dequantise-then-matmul baseline, applied to its bf16 gate_up
+ * output yb [M, N] (bf16 bits): the gate and up values as the baseline
+ * materialised them (bf16, widened exactly to fp32), silu(g) = g / (1 + e^-g)
+ * and the product with up in fp32, one bf16 rounding. Output: bf16 bits
+ * [M, N/2]. This is the baseline side of the fidelity comparison for a fused
+ * SwiGLU ("grouped-nf4-gemm -- single-launch W4A16 GEMM ...", "The claim":
+ * fused error below the dequantise-then-matmul path's; the package page's
+ * "Owns" names swiglu among the glue that follows gate_up). Reading taken:
+ * the baseline rounds its GEMM output to bf16 before the activation. */
+int oracle_baseline_swiglu_bf16(const uint16_t *yb, int64_t M, int32_t N, uint16_t *out) {
+    if (M < 0 || N <= 0 || N % 2) return ORC_BAD_SHAPE;
+    const int32_t H = N / 2;
+    for (int64_t m = 0; m < M; ++m)
+        for (int32_t j = 0; j < H; ++j) {
+            const float g = bf16_to_f32(yb[m * N + j]);
+            const float u = bf16_to_f32(yb[m * N + H + j]);
+            const float silu = g / (1.0f + expf(-g));
+            out[m * H + j] = bf16_rne(silu * u);
+        }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------ router top-k */
 /* Per token: the top_k experts by logit, picked one at a time as the largest
    remaining logit (equal logits: the lower expert id; a NaN logit counts as

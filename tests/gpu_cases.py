@@ -64,3 +64,19 @@ def boundaries(sizes: Sequence[int]) -> np.ndarray:
             out += [off, off + s - 1]
         off += s
     return np.unique(np.array(out, dtype=np.int64))
+
+
+def tile_strata(sizes: Sequence[int], seed: int = 0, half: int = 128) -> np.ndarray:
+    """One seeded row in every `half`-row slice of every group (the tensor-core
+    kernel's token tiles are 256 rows of one group, split into two 128-row
+    halves, one per CTA of a pair), plus the first and last row of every
+    non-empty group."""
+    rng = np.random.default_rng(seed)
+    out = [boundaries(sizes)]
+    off = 0
+    for s in sizes:
+        for h0 in range(0, int(s), half):
+            h1 = min(int(s), h0 + half)
+            out.append(np.array([off + int(rng.integers(h0, h1))]))
+        off += int(s)
+    return np.unique(np.concatenate(out)).astype(np.int64)

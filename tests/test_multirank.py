@@ -59,3 +59,17 @@ def test_counter_key_ignores_comments_but_not_code(tmp_path):
     assert bench.source_hash(str(p)) == h0
     p.write_text(base.replace("a + 1", "a + 2"))
     assert bench.source_hash(str(p)) != h0
+
+
+def test_reference_arm_never_loads_the_product_library():
+    # The reference arm is the oracle on the host cores: its inputs are built
+    # on the host and the product package (and so libgnf4.so) is never loaded.
+    code = ("import sys, types; sys.argv = ['bench.py']; import bench; "
+            "a = types.SimpleNamespace(workload='tiny', steps=1, warmup=3); "
+            "line = bench.run_reference(a, 0, 1); "
+            "print('LOADED' if 'grouped_nf4_w4a16_b200' in sys.modules else 'CLEAN', line['impl'])")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "CLEAN reference" in r.stdout

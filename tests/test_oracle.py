@@ -332,6 +332,35 @@ def test_baseline_emulation_against_fp64_of_bf16_weights():
     assert np.all(np.abs(yb - ref_b) <= ulp + 1e-30)
 
 
+def test_baseline_swiglu_against_expit_on_its_own_bf16_values():
+    # The baseline's SwiGLU works on the bf16 gate and up values its GEMM
+    # materialised. Pin: the closed form g * expit(g) * u in fp64 on those same
+    # values, rounded once to bf16, equals the oracle's fp32 computation except
+    # where fp32 rounding crosses a bf16 rounding boundary (then one ulp).
+    rng = np.random.default_rng(12)
+    M, N = 64, 96
+    yb = oracle.f32_to_bf16((rng.standard_normal((M, N)) * 3).astype(np.float32))
+    yb[0, 0] = 0                       # g = 0 -> 0
+    yb[1, 0] = oracle.f32_to_bf16(np.array([-80.0], np.float32))[0]   # silu(-80) ~ -1.4e-33
+    yb[2, 0] = oracle.f32_to_bf16(np.array([40.0], np.float32))[0]     # silu(40) = 40 (to fp32)
+    out = synth.bf16_bits_to_f32(oracle.baseline_swiglu_bf16(yb)).astype(np.float64)
+    v = synth.bf16_bits_to_f32(yb).astype(np.float64)
+    g, u = v[:, :N // 2], v[:, N // 2:]
+    ref = g * scipy.special.expit(g) * u
+    ref_b = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    ref_b = ref_b.astype(np.float64)
+    ulp = np.abs(ref_b) * 2.0 ** -7
+    assert np.all(np.abs(out - ref_b) <= ulp + 1e-45)
+    assert np.mean(out == ref_b) > 0.99
+    assert out[0, 0] == 0.0
+    assert out[2, 0] == ref_b[2, 0]
+    # gate and up halves are not swapped: scaling the up half scales the output
+    yb2 = yb.copy()
+    yb2[:, N // 2:] = oracle.f32_to_bf16((v[:, N // 2:] * 2).astype(np.float32))
+    out2 = synth.bf16_bits_to_f32(oracle.baseline_swiglu_bf16(yb2)).astype(np.float64)
+    assert np.array_equal(out2, 2 * out)
+
+
 def test_fidelity_ordering_is_achievable():
     # The fp64 result rounded once to bf16 is closer to the reference than the
     # materialise-to-bf16 baseline, as the README's "The claim" states.
