@@ -29,6 +29,12 @@ grouped_nf4_gemm 0.1.0, opening section, unless stated):
   to its activations, dx = dy . W per group, in fp64 (package page
   "grouped-nf4-gemm", header block, "Owns": the grouped packed GEMM and its
   dgrad).
+* :func:`grouped_gemm_mxfp4_f64` / :func:`e2m1_table` -- the same GEMM over
+  native MXFP4 (e2m1 codes, e8m0 scale per 32; package page "Direct answer");
+  :func:`grouped_gemm_bf16_absmax_f64` -- NF4 with bf16 absmax (a bf16 value
+  widens to fp32 exactly); :func:`swiglu_interleaved_f64` -- the gpt-oss
+  gated activation on interleaved, clamped gate/up columns;
+  :func:`gather_rows` -- x[i] = hidden[sorted_idx[i] // top_k].
 * :func:`router_topk` / :func:`moe_combine` -- the router's top-k with softmax
   weights, and the top-k weighted combine after the down projection (package
   page "grouped-nf4-gemm", "Use this when": router softmax and top-k and the
@@ -87,13 +93,21 @@ def _load():
         lib.oracle_swiglu_f64.argtypes = [P, i64, i32, P]
         lib.oracle_baseline_bf16.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P, i64, P]
         lib.oracle_baseline_swiglu_bf16.argtypes = [P, i64, i32, P]
+        lib.oracle_e2m1_table.argtypes = [P]
+        lib.oracle_grouped_gemm_mxfp4_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P,
+                                                      i64, P]
+        lib.oracle_swiglu_interleaved_f64.argtypes = [P, i64, i32, ctypes.c_double,
+                                                      ctypes.c_double, P]
+        lib.oracle_gather_rows.argtypes = [P, i64, i32, P, i64, i32, P]
         lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, P, P]
         lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i32, P]
         lib.oracle_grouped_dgrad_f64.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, P]
         for name in ("oracle_quantize_nf4", "oracle_dequant_f32", "oracle_dequant_bf16",
                      "oracle_moe_align", "oracle_grouped_gemm_f64", "oracle_swiglu_f64",
                      "oracle_baseline_bf16", "oracle_baseline_swiglu_bf16", "oracle_router_topk",
-                     "oracle_moe_combine", "oracle_grouped_dgrad_f64"):
+                     "oracle_moe_combine", "oracle_grouped_dgrad_f64",
+                     "oracle_grouped_gemm_mxfp4_f64", "oracle_swiglu_interleaved_f64",
+                     "oracle_gather_rows"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -234,6 +248,63 @@ def baseline_swiglu_bf16(yb: np.ndarray) -> np.ndarray:
     out = np.empty((M, N // 2), dtype=np.uint16)
     _check(_load().oracle_baseline_swiglu_bf16(_p(yb), M, N, _p(out)))
     return out
+
+
+def e2m1_table() -> np.ndarray:
+    """The 16 e2m1 code values (fp64), index = 4-bit code."""
+    out = np.empty(16, dtype=np.float64)
+    _load().oracle_e2m1_table(_p(out))
+    return out
+
+
+def grouped_gemm_mxfp4_f64(x: np.ndarray, w: np.ndarray, scales: np.ndarray, sizes: np.ndarray,
+                           expert_ids: np.ndarray, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """MXFP4 grouped GEMM in fp64: w uint8 [E, N, K/2] (even k in the low
+    nibble), scales e8m0 uint8 [E, N, K/32]; x bf16 bits [M, K]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    sizes = np.ascontiguousarray(sizes, dtype=np.int32)
+    expert_ids = np.ascontiguousarray(expert_ids, dtype=np.int32)
+    M, K = x.shape
+    E, N, Kh = w.shape
+    if Kh * 2 != K or scales.shape != (E, N, K // 32):
+        raise OracleError("bad shape")
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = M if rows is None else rows.size
+    y = np.empty((nrows, N), dtype=np.float64)
+    _check(_load().oracle_grouped_gemm_mxfp4_f64(
+        _p(x), _p(w), _p(scales), _p(sizes), _p(expert_ids), sizes.size, M, N, K, E,
+        None if rows is None else _p(rows), nrows, _p(y)))
+    return y
+
+
+def swiglu_interleaved_f64(y: np.ndarray, alpha: float, limit: float) -> np.ndarray:
+    """gpt-oss gated activation on interleaved gate (even) / up (odd) columns."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    M, N = y.shape
+    out = np.empty((M, N // 2), dtype=np.float64)
+    _check(_load().oracle_swiglu_interleaved_f64(_p(y), M, N, float(alpha), float(limit), _p(out)))
+    return out
+
+
+def gather_rows(hidden: np.ndarray, sorted_idx: np.ndarray, top_k: int) -> np.ndarray:
+    """x[i] = hidden[sorted_idx[i] // top_k] (bf16 bits)."""
+    hidden = np.ascontiguousarray(hidden, dtype=np.uint16)
+    sorted_idx = np.ascontiguousarray(sorted_idx, dtype=np.int32)
+    T, K = hidden.shape
+    x = np.empty((sorted_idx.size, K), dtype=np.uint16)
+    _check(_load().oracle_gather_rows(_p(hidden), T, K, _p(sorted_idx), sorted_idx.size, top_k,
+                                      _p(x)))
+    return x
+
+
+def grouped_gemm_bf16_absmax_f64(x, w, absmax_bf16_bits, sizes, expert_ids, rows=None):
+    """The NF4 grouped GEMM with bf16 absmax (bit patterns [E, N, K/64]): the
+    scale is the bf16 value itself, which widens to fp32 exactly."""
+    wide = (np.asarray(absmax_bf16_bits, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+    return grouped_gemm_f64(x, w, wide, sizes, expert_ids, rows=rows)
 
 
 def quantized_stack(E: int, N: int, K: int, weights_fn) -> Tuple[np.ndarray, np.ndarray]:

@@ -262,6 +262,102 @@ int oracle_grouped_gemm_f64(const uint16_t *x, const uint8_t *w, const float *ab
     return ORC_OK;
 }
 
+/* ------------------------------------------------ MXFP4 grouped GEMM (fp64) */
+/* The same grouped GEMM over native MXFP4 weights ("grouped-nf4-gemm" package
+ * page, "Direct answer": e2m1 codes with e8m0 scales, multiplied as released,
+ * no requantisation). Format (OCP microscaling FP4, the layout of the
+ * released gpt-oss expert blocks): byte j of a row holds element k = 2j in the
+ * LOW nibble and k = 2j+1 in the HIGH nibble; each code is an e2m1 number
+ * (1 sign, 2 exponent bits with bias 1, 1 mantissa bit; exponent field 0 is
+ * the subnormal 0 or 0.5); scales[e][n][b] is one e8m0 byte per 32
+ * consecutive elements, the power of two 2^(s-127) (255 is NaN). The
+ * product code * scale is exact in fp64. */
+static double e2m1_value(int c) {
+    const int sgn = (c >> 3) & 1, ex = (c >> 1) & 3, man = c & 1;
+    double mag = ex == 0 ? 0.5 * man : ldexp(1.0 + 0.5 * man, ex - 1);
+    return sgn ? -mag : mag;
+}
+
+static double e8m0_value(uint8_t s) { return s == 255 ? NAN : ldexp(1.0, (int)s - 127); }
+
+void oracle_e2m1_table(double *out16) {
+    for (int c = 0; c < 16; ++c) out16[c] = e2m1_value(c);
+}
+
+int oracle_grouped_gemm_mxfp4_f64(const uint16_t *x, const uint8_t *w, const uint8_t *scales,
+                                  const int32_t *sizes, const int32_t *expert_ids, int32_t G,
+                                  int64_t M, int32_t N, int32_t K, int32_t E, const int64_t *rows,
+                                  int64_t nrows, double *y) {
+    if (M < 0 || N <= 0 || K <= 0 || K % 32 || E <= 0 || G < 0) return ORC_BAD_SHAPE;
+    int32_t *row_expert = (int32_t *)malloc((size_t)(M > 0 ? M : 1) * sizeof(int32_t));
+    if (!row_expert) return ORC_BAD_SHAPE;
+    int st = rows_to_expert(sizes, expert_ids, G, M, E, row_expert);
+    if (st != ORC_OK) { free(row_expert); return st; }
+    if (!rows) nrows = M;
+    for (int64_t i = 0; i < nrows; ++i) {
+        if (rows && (rows[i] < 0 || rows[i] >= M)) { free(row_expert); return ORC_BAD_SHAPE; }
+    }
+    const int64_t nb = K / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t m = rows ? rows[i] : i;
+        const int32_t e = row_expert[m];
+        double *xr = (double *)malloc((size_t)K * sizeof(double));
+        for (int32_t k = 0; k < K; ++k) xr[k] = (double)bf16_to_f32(x[m * K + k]);
+        for (int32_t n = 0; n < N; ++n) {
+            const int64_t row = (int64_t)e * N + n;
+            const uint8_t *wr = w + row * (K / 2);
+            const uint8_t *sr = scales + row * nb;
+            double acc = 0.0;
+            for (int32_t k = 0; k < K; ++k) {
+                const uint8_t byte = wr[k >> 1];
+                const int code = (k & 1) ? (byte >> 4) : (byte & 0x0F);
+                acc += xr[k] * (e2m1_value(code) * e8m0_value(sr[k / 32]));
+            }
+            y[i * N + n] = acc;
+        }
+        free(xr);
+    }
+    free(row_expert);
+    return ORC_OK;
+}
+
+/* -------------------------------- SwiGLU on interleaved gate/up, clamped */
+/* The gpt-oss form of the gated activation (its published model definition),
+ * listed with the absmax variants among the next steps of this path: gate =
+ * even columns, up = odd columns of the gate_up output y [M, N]; the gate is
+ * clamped from above at `limit`, the up value to [-limit, limit];
+ * out[m, j] = g * sigmoid(alpha * g) * (u + 1), in fp64. */
+int oracle_swiglu_interleaved_f64(const double *y, int64_t M, int32_t N, double alpha,
+                                  double limit, double *out) {
+    if (M < 0 || N <= 0 || N % 2) return ORC_BAD_SHAPE;
+    const int32_t H = N / 2;
+    for (int64_t m = 0; m < M; ++m)
+        for (int32_t j = 0; j < H; ++j) {
+            double g = y[m * N + 2 * j], u = y[m * N + 2 * j + 1];
+            if (g > limit) g = limit;
+            if (u > limit) u = limit;
+            if (u < -limit) u = -limit;
+            out[m * H + j] = g / (1.0 + exp(-alpha * g)) * (u + 1.0);
+        }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------ row gather */
+/* The activation rows of the sorted order: x[i] = hidden[sorted_idx[i] / top_k]
+ * (bf16 bits; the gather the token->expert sort implies, "grouped-nf4-gemm"
+ * package page, "Use this when", folded into the GEMM). */
+int oracle_gather_rows(const uint16_t *hidden, int64_t T, int32_t K, const int32_t *sorted_idx,
+                       int64_t M, int32_t top_k, uint16_t *x) {
+    if (T < 0 || K <= 0 || M < 0 || top_k < 1) return ORC_BAD_SHAPE;
+    for (int64_t i = 0; i < M; ++i) {
+        const int32_t s = sorted_idx[i];
+        if (s < 0 || (int64_t)s >= T * top_k) return ORC_BAD_SLOT;
+        memcpy(x + i * K, hidden + (int64_t)(s / top_k) * K, (size_t)K * sizeof(uint16_t));
+    }
+    return ORC_OK;
+}
+
 /* SwiGLU on an fp64 [M, N] gate_up output: out[m, j] = silu(y[m, j]) * y[m, j + N/2]. */
 int oracle_swiglu_f64(const double *y, int64_t M, int32_t N, double *out) {
     if (M < 0 || N <= 0 || N % 2) return ORC_BAD_SHAPE;

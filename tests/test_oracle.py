@@ -554,3 +554,124 @@ def test_grouped_dgrad_rejects_bad_metadata():
         oracle.grouped_dgrad_f64(dy, packed, absmax, [2, 1], [0, 1])    # sizes sum 3 != 4
     with pytest.raises(oracle.OracleError):
         oracle.grouped_dgrad_f64(dy, packed, absmax, [2, 2], [0, 2])    # expert 2 of 2
+
+
+# ------------------------------------------------------------------ MXFP4
+# The values of the FP4 (E2M1) element type as the OCP Microscaling Formats
+# (MX) v1.0 specification tabulates them: 1 sign bit, 2 exponent bits (bias
+# 1), 1 mantissa bit; exponent field 0 is subnormal.
+OCP_E2M1_POSITIVE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _mx_dequant_numpy(w, scales):
+    """Independent NumPy decode: low nibble = even k, value from the spec's
+    table above times 2^(s - 127)."""
+    table = np.array(OCP_E2M1_POSITIVE + [-v for v in OCP_E2M1_POSITIVE])
+    lo, hi = w & 0x0F, w >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(w.shape[:-1] + (w.shape[-1] * 2,))
+    vals = table[codes]
+    sc = np.ldexp(1.0, scales.astype(np.int64) - 127)
+    sc = np.where(scales == 255, np.nan, sc)
+    return vals * np.repeat(sc, 32, axis=-1)
+
+
+def test_e2m1_table_is_the_ocp_table():
+    t = oracle.e2m1_table()
+    assert t[:8].tolist() == OCP_E2M1_POSITIVE
+    assert t[8:].tolist() == [-v for v in OCP_E2M1_POSITIVE]
+    assert np.signbit(t[8])          # code 8 is -0
+
+
+@pytest.mark.parametrize("E,N,K,sizes,experts", [
+    (2, 5, 64, [3, 2], [1, 0]), (3, 7, 128, [0, 4, 1], [2, 1, 0]), (1, 3, 96, [2], [0])])
+def test_mxfp4_gemm_matches_numpy_brute_force(E, N, K, sizes, experts):
+    rng = np.random.default_rng(E * 100 + K)
+    M = sum(sizes)
+    x = synth.activations_bf16(M, K, seed=K)
+    w = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    sc = rng.integers(110, 140, size=(E, N, K // 32)).astype(np.uint8)
+    y = oracle.grouped_gemm_mxfp4_f64(x, w, sc, np.array(sizes, np.int32), np.array(experts, np.int32))
+    wd = _mx_dequant_numpy(w, sc)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    ref = np.zeros((M, N))
+    off = 0
+    for s_, e in zip(sizes, experts):
+        ref[off:off + s_] = xf[off:off + s_] @ wd[e].T
+        off += s_
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-300)
+
+
+def test_mxfp4_gemm_nibble_order_and_one_hot_read_out():
+    # byte 0x21: k = 0 takes the low nibble (code 1 = 0.5), k = 1 the high
+    # nibble (code 2 = 1.0); scale byte 127 = 2^0, 128 = 2^1
+    w = np.zeros((1, 2, 16), np.uint8)
+    w[0, 0, 0] = 0x21
+    w[0, 1, 0] = 0xF7                      # k = 0: code 7 = 6.0, k = 1: code 15 = -6.0
+    sc = np.array([[[127], [128]]], np.uint8)
+    x = np.zeros((2, 32), np.float32)
+    x[0, 0] = 1.0
+    x[1, 1] = 1.0
+    xb = oracle.f32_to_bf16(x)
+    y = oracle.grouped_gemm_mxfp4_f64(xb, w, sc, np.array([2], np.int32), np.array([0], np.int32))
+    assert y.tolist() == [[0.5, 12.0], [1.0, -12.0]]
+
+
+def test_mxfp4_e8m0_extremes():
+    w = np.full((1, 1, 16), 0x22, np.uint8)          # every element 1.0
+    x = oracle.f32_to_bf16(np.ones((1, 32), np.float32))
+    for s_, want in [(0, 32.0 * 2.0 ** -127), (254, 32.0 * 2.0 ** 127)]:
+        y = oracle.grouped_gemm_mxfp4_f64(x, w, np.array([[[s_]]], np.uint8),
+                                          np.array([1], np.int32), np.array([0], np.int32))
+        assert y[0, 0] == want
+    y = oracle.grouped_gemm_mxfp4_f64(x, w, np.array([[[255]]], np.uint8),
+                                      np.array([1], np.int32), np.array([0], np.int32))
+    assert np.isnan(y[0, 0])
+
+
+# -------------------------------------------------------- bf16 absmax
+def test_bf16_absmax_equals_fp32_absmax_of_the_same_values():
+    rng = np.random.default_rng(21)
+    E, N, K = 2, 6, 128
+    x, w, a, s, ex = _random_problem(rng, E, N, K, [3, 2], [1, 0])
+    ab = oracle.f32_to_bf16(a)
+    a_wide = synth.bf16_bits_to_f32(ab)
+    y_b = oracle.grouped_gemm_bf16_absmax_f64(x, w, ab, s, ex)
+    assert np.array_equal(y_b, oracle.grouped_gemm_f64(x, w, a_wide, s, ex))
+    # and against NumPy: the scale of block b is the bf16 value (exact)
+    table = oracle.nf4_table().astype(np.float64)
+    codes = np.stack([w >> 4, w & 0x0F], axis=-1).reshape(E, N, K)
+    wd = table[codes] * np.repeat(a_wide.astype(np.float64), 64, axis=-1)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    ref = np.concatenate([xf[:3] @ wd[1].T, xf[3:] @ wd[0].T])
+    assert np.allclose(y_b, ref, rtol=1e-12, atol=0)
+
+
+# ------------------------------------------- interleaved, clamped SwiGLU
+def test_swiglu_interleaved_closed_form_and_clamps():
+    rng = np.random.default_rng(22)
+    y = rng.standard_normal((4, 10)) * 6
+    y[0, 0], y[0, 1] = 20.0, 3.0        # gate above the limit
+    y[1, 2], y[1, 3] = 1.0, -30.0       # up below -limit
+    y[2, 4], y[2, 5] = -40.0, 2.0       # very negative gate: not clamped from below
+    alpha, limit = 1.702, 7.0
+    out = oracle.swiglu_interleaved_f64(y, alpha, limit)
+    g = np.minimum(y[:, 0::2], limit)
+    u = np.clip(y[:, 1::2], -limit, limit)
+    ref = g * scipy.special.expit(alpha * g) * (u + 1)
+    assert np.allclose(out, ref, rtol=1e-13, atol=1e-300)
+    assert out[0, 0] == pytest.approx(7.0 * scipy.special.expit(alpha * 7.0) * 4.0, rel=1e-14)
+    assert out[1, 1] == pytest.approx(1.0 * scipy.special.expit(alpha) * (-6.0), rel=1e-14)
+    assert abs(out[2, 2]) < 1e-25
+
+
+# ---------------------------------------------------------------- gather
+def test_gather_rows_is_indexing_by_token():
+    rng = np.random.default_rng(23)
+    T, k, K = 5, 3, 64
+    hidden = rng.integers(0, 65535, size=(T, K)).astype(np.uint16)
+    topk = rng.integers(0, 4, size=(T, k)).astype(np.int32)
+    sorted_idx, sizes, experts, ng = oracle.moe_align(topk, 4)
+    x = oracle.gather_rows(hidden, sorted_idx, k)
+    assert np.array_equal(x, hidden[sorted_idx // k])
+    with pytest.raises(oracle.OracleError):
+        oracle.gather_rows(hidden, np.array([T * k], np.int32), k)
