@@ -488,11 +488,12 @@ def time_glue(prob, stream, reps=50):
                     S * H * 2 + w.T * H * 2 + S * 8),
     }
     if not prob.prefill:
-        # the dgrad of the last GEMM (CUDA-core kernel, decode-sized batches only)
+        # the dgrad of the last GEMM (tensor-core kernel for decode-sized batches)
         d = prob.gemms[-1]
         g = d["g"]
         dx = torch.empty((w.M, g.K), dtype=torch.bfloat16, device=dev)
-        ws_dg = gnf4.make_workspace(256, dev)
+        ws_dg = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_DGRAD, w.M, g.N,
+                                                              g.K, w.E, w.E), dev)
         calls["dgrad"] = (lambda: gnf4.gnf4_grouped_dgrad(y, d["W"][0], d["A"][0], prob.sizes,
                                                           prob.expert_ids, dx=dx, workspace=ws_dg),
                           prob.U * g.N * g.K * 9 // 16 + w.M * g.N * 2 + w.M * g.K * 2)

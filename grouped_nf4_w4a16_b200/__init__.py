@@ -11,6 +11,13 @@ from .binding import (  # noqa: F401
     GNF4_OK,
     GNF4_EPI_NONE,
     GNF4_EPI_SWIGLU,
+    GNF4_EPI_SWIGLU_INTERLEAVED,
+    GNF4_FMT_NF4,
+    GNF4_FMT_MXFP4,
+    GNF4_SCALE_F32,
+    GNF4_SCALE_BF16,
+    GNF4_SCALE_E8M0,
+    GemmDesc,
     GNF4_MODE_AUTO,
     GNF4_MODE_DECODE,
     GNF4_MODE_PREFILL,
@@ -31,6 +38,7 @@ from .binding import (  # noqa: F401
     gnf4_moe_align,
     gnf4_grouped_gemm,
     gnf4_grouped_gemm_noalloc,
+    gnf4_grouped_gemm_ex,
     gnf4_router_topk,
     gnf4_moe_combine,
     gnf4_grouped_dgrad,

@@ -25,7 +25,9 @@ _STATUS_NAMES = {
     9: "GNF4_ERR_SCRATCH_LIMIT",
 }
 GNF4_NOALLOC_SCRATCH_BYTES = 8 << 20
-GNF4_EPI_NONE, GNF4_EPI_SWIGLU = 0, 1
+GNF4_EPI_NONE, GNF4_EPI_SWIGLU, GNF4_EPI_SWIGLU_INTERLEAVED = 0, 1, 2
+GNF4_FMT_NF4, GNF4_FMT_MXFP4 = 0, 1
+GNF4_SCALE_F32, GNF4_SCALE_BF16, GNF4_SCALE_E8M0 = 0, 1, 2
 GNF4_MODE_AUTO, GNF4_MODE_DECODE, GNF4_MODE_PREFILL = 0, 1, 2
 GNF4_OUT_F32, GNF4_OUT_BF16 = 0, 1
 GNF4_OP_MOE_ALIGN, GNF4_OP_GROUPED_GEMM, GNF4_OP_MOE_COMBINE, GNF4_OP_GROUPED_DGRAD = 0, 1, 2, 3
@@ -38,7 +40,23 @@ EXPORTED_SYMBOLS = (
     "gnf4_moe_align", "gnf4_grouped_gemm", "gnf4_dequant_debug", "gnf4_workspace_bytes",
     "gnf4_read_device_status", "gnf4_status_string", "gnf4_version",
     "gnf4_grouped_gemm_noalloc", "gnf4_router_topk", "gnf4_moe_combine", "gnf4_grouped_dgrad",
+    "gnf4_grouped_gemm_ex",
 )
+
+
+class GemmDesc(ctypes.Structure):
+    """gnf4_gemm_desc of include/gnf4.h, field for field."""
+    _fields_ = [
+        ("struct_bytes", ctypes.c_uint32), ("format", ctypes.c_int32),
+        ("scale_dtype", ctypes.c_int32), ("epilogue", ctypes.c_int32),
+        ("swiglu_alpha", ctypes.c_float), ("swiglu_limit", ctypes.c_float),
+        ("mode", ctypes.c_int32), ("top_k", ctypes.c_int32),
+        ("x", ctypes.c_void_p), ("hidden", ctypes.c_void_p), ("sorted_idx", ctypes.c_void_p),
+        ("n_tokens", ctypes.c_int64), ("w", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("sizes", ctypes.c_void_p), ("expert_ids", ctypes.c_void_p),
+        ("G", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("E", ctypes.c_int32),
+        ("M", ctypes.c_int64), ("y", ctypes.c_void_p),
+    ]
 
 _lib = None
 
@@ -88,6 +106,8 @@ def load_library():
     lib.gnf4_moe_combine.restype = ctypes.c_int
     lib.gnf4_grouped_dgrad.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, sz, P]
     lib.gnf4_grouped_dgrad.restype = ctypes.c_int
+    lib.gnf4_grouped_gemm_ex.argtypes = [ctypes.POINTER(GemmDesc), P, sz, P]
+    lib.gnf4_grouped_gemm_ex.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -179,6 +199,72 @@ def gnf4_grouped_gemm(x: torch.Tensor, w: torch.Tensor, absmax: torch.Tensor, si
         _ptr(x), _ptr(w), _ptr(absmax), _ptr(sizes), _ptr(expert_ids), G, M, N, K, E, blocksize,
         epilogue, mode, _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "gnf4_grouped_gemm")
+    return y
+
+
+def gnf4_grouped_gemm_ex(w: torch.Tensor, scales: torch.Tensor, sizes: torch.Tensor,
+                         expert_ids: torch.Tensor, *, x: Optional[torch.Tensor] = None,
+                         hidden: Optional[torch.Tensor] = None,
+                         sorted_idx: Optional[torch.Tensor] = None, top_k: int = 1,
+                         M: Optional[int] = None, fmt: int = GNF4_FMT_NF4,
+                         epilogue: int = GNF4_EPI_NONE, swiglu_alpha: float = 1.702,
+                         swiglu_limit: float = 7.0, mode: int = GNF4_MODE_AUTO,
+                         y: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """gnf4_grouped_gemm_ex: the grouped GEMM over NF4 (scales = fp32 or bf16
+    absmax [E,N,K/64]) or MXFP4 (fmt=GNF4_FMT_MXFP4, scales = e8m0 uint8
+    [E,N,K/32]), rows from x [M,K] or gathered as hidden[sorted_idx[i] //
+    top_k] (x=None; M = number of rows, default sorted_idx.numel())."""
+    _need(w, "w", torch.uint8)
+    _need(sizes, "sizes", torch.int32)
+    _need(expert_ids, "expert_ids", torch.int32)
+    if fmt == GNF4_FMT_MXFP4:
+        _need(scales, "scales", torch.uint8)
+        sdt = GNF4_SCALE_E8M0
+    elif scales.dtype == torch.bfloat16:
+        _need(scales, "scales", torch.bfloat16)
+        sdt = GNF4_SCALE_BF16
+    else:
+        _need(scales, "scales", torch.float32)
+        sdt = GNF4_SCALE_F32
+    E, N, Kh = w.shape
+    K = 2 * Kh
+    if x is not None:
+        _need(x, "x", torch.bfloat16)
+        if hidden is not None:
+            raise ValueError("pass x or hidden, not both")
+        M = x.shape[0]
+        dev = x.device
+    else:
+        if hidden is None or sorted_idx is None:
+            raise ValueError("gathering needs hidden and sorted_idx")
+        _need(hidden, "hidden", torch.bfloat16)
+        _need(sorted_idx, "sorted_idx", torch.int32)
+        M = sorted_idx.numel() if M is None else int(M)
+        dev = hidden.device
+    G = sizes.numel()
+    n_out = N // 2 if epilogue != GNF4_EPI_NONE else N
+    if y is None:
+        y = torch.empty((M, n_out), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(y, "y", torch.bfloat16)
+    if workspace is None:
+        workspace = make_workspace(gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G), dev)
+    d = GemmDesc()
+    d.struct_bytes = ctypes.sizeof(GemmDesc)
+    d.format, d.scale_dtype, d.epilogue = fmt, sdt, epilogue
+    d.swiglu_alpha, d.swiglu_limit = swiglu_alpha, swiglu_limit
+    d.mode, d.top_k = mode, top_k
+    d.x = _ptr(x)
+    d.hidden = _ptr(hidden) if x is None else None
+    d.sorted_idx = _ptr(sorted_idx) if x is None else None
+    d.n_tokens = hidden.shape[0] if x is None else 0
+    d.w, d.scales, d.sizes, d.expert_ids = _ptr(w), _ptr(scales), _ptr(sizes), _ptr(expert_ids)
+    d.G, d.N, d.K, d.E, d.M = G, N, K, E, M
+    d.y = _ptr(y)
+    st = load_library().gnf4_grouped_gemm_ex(ctypes.byref(d), _ptr(workspace), workspace.numel(),
+                                             _stream(stream))
+    _check(st, "gnf4_grouped_gemm_ex")
     return y
 
 

@@ -76,13 +76,80 @@ gnf4_status check_grouped_gemm(const uint16_t *x, const uint8_t *w, const float 
   a.x = x; a.w = w; a.absmax = absmax; a.sizes = sizes; a.expert_ids = expert_ids;
   a.G = G; a.M = M; a.N = N; a.K = K; a.E = E; a.swiglu = (epilogue == GNF4_EPI_SWIGLU);
   a.y = y; a.workspace = nullptr; a.ws_bytes = 0;
+  a.scales = absmax; a.epi = epilogue;
+  const bool pf_ok = prefill_supports(a);
   int32_t use = mode;
   if (use == GNF4_MODE_AUTO) {
     const int64_t groups = G < E ? G : E;
-    // the tensor-core kernel has no fused SwiGLU yet: SwiGLU stays on the decode kernel
-    use = (M > kPrefillMeanRows * groups && epilogue == GNF4_EPI_NONE) ? GNF4_MODE_PREFILL
-                                                                       : GNF4_MODE_DECODE;
+    use = (M > kPrefillMeanRows * groups && pf_ok) ? GNF4_MODE_PREFILL : GNF4_MODE_DECODE;
   }
+  if (use == GNF4_MODE_PREFILL && !pf_ok) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  *use_out = use;
+  return GNF4_OK;
+}
+
+gnf4_status check_grouped_gemm_ex(const gnf4_gemm_desc *d, GemmArgs *out, int32_t *use_out) {
+  *use_out = -1;
+  if (!d) return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->struct_bytes != sizeof(gnf4_gemm_desc)) return GNF4_ERR_INVALID_ARGUMENT;
+  const bool gather = d->x == nullptr;
+  if (gather ? (!d->hidden || !d->sorted_idx) : (d->hidden != nullptr))
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (!d->w || !d->scales || !d->sizes || !d->expert_ids || !d->y) return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->M < 0 || d->N < 1 || d->K < 1 || d->E < 1 || d->G < 1) return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->format != GNF4_FMT_NF4 && d->format != GNF4_FMT_MXFP4) return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->format == GNF4_FMT_NF4 ? (d->scale_dtype != GNF4_SCALE_F32 &&
+                                   d->scale_dtype != GNF4_SCALE_BF16)
+                                : d->scale_dtype != GNF4_SCALE_E8M0)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->epilogue != GNF4_EPI_NONE && d->epilogue != GNF4_EPI_SWIGLU &&
+      d->epilogue != GNF4_EPI_SWIGLU_INTERLEAVED)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->epilogue == GNF4_EPI_SWIGLU_INTERLEAVED &&
+      !(d->swiglu_limit > 0.0f && d->swiglu_limit < 3.0e38f && d->swiglu_alpha == d->swiglu_alpha))
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->mode != GNF4_MODE_AUTO && d->mode != GNF4_MODE_DECODE && d->mode != GNF4_MODE_PREFILL)
+    return GNF4_ERR_INVALID_ARGUMENT;
+  if (gather && (d->top_k < 1 || d->n_tokens < 0)) return GNF4_ERR_INVALID_ARGUMENT;
+  if (d->K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (d->E > GNF4_MAX_EXPERTS || d->G > GNF4_MAX_EXPERTS) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (d->epilogue != GNF4_EPI_NONE && (d->N % 2) != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (d->M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (gather && d->n_tokens * static_cast<int64_t>(d->top_k) >= INT_MAX)
+    return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(d->E) * d->N + d->N + 256 >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (d->M == 0) return GNF4_OK;
+  const void *xs = gather ? static_cast<const void *>(d->hidden) : static_cast<const void *>(d->x);
+  if (!is_device_pointer(xs) || !is_device_pointer(d->w) || !is_device_pointer(d->scales) ||
+      !is_device_pointer(d->sizes) || !is_device_pointer(d->expert_ids) ||
+      !is_device_pointer(d->y) || (gather && !is_device_pointer(d->sorted_idx)))
+    return GNF4_ERR_HOST_POINTER;
+  if (!aligned(xs, 32) || !aligned(d->w, 32) || !aligned(d->y, 32) || !aligned(d->scales, 4) ||
+      !aligned(d->sizes, 4) || !aligned(d->expert_ids, 4) ||
+      (gather && !aligned(d->sorted_idx, 4)))
+    return GNF4_ERR_MISALIGNED;
+  GemmArgs &a = *out;
+  a.x = d->x; a.w = d->w;
+  a.absmax = (d->format == GNF4_FMT_NF4 && d->scale_dtype == GNF4_SCALE_F32)
+                 ? static_cast<const float *>(d->scales) : nullptr;
+  a.scales = d->scales;
+  a.fmt = d->format; a.scale_dtype = d->scale_dtype; a.epi = d->epilogue;
+  a.alpha = d->swiglu_alpha; a.limit = d->swiglu_limit;
+  a.hidden = gather ? d->hidden : nullptr;
+  a.sorted_idx = gather ? d->sorted_idx : nullptr;
+  a.n_tokens = gather ? d->n_tokens : 0;
+  a.top_k = gather ? d->top_k : 1;
+  a.sizes = d->sizes; a.expert_ids = d->expert_ids;
+  a.G = d->G; a.M = d->M; a.N = d->N; a.K = d->K; a.E = d->E;
+  a.swiglu = d->epilogue != GNF4_EPI_NONE;
+  a.y = d->y; a.workspace = nullptr; a.ws_bytes = 0;
+  const bool pf_ok = prefill_supports(a);
+  int32_t use = d->mode;
+  if (use == GNF4_MODE_AUTO) {
+    const int64_t groups = d->G < d->E ? d->G : d->E;
+    use = (d->M > kPrefillMeanRows * groups && pf_ok) ? GNF4_MODE_PREFILL : GNF4_MODE_DECODE;
+  }
+  if (use == GNF4_MODE_PREFILL && !pf_ok) return GNF4_ERR_UNSUPPORTED_SHAPE;
   *use_out = use;
   return GNF4_OK;
 }
@@ -124,7 +191,7 @@ size_t gnf4_workspace_bytes(int32_t op, int64_t M, int32_t N, int32_t K, int32_t
   (void)E;
   if (op == GNF4_OP_MOE_ALIGN) return kWsHeaderBytes;
   if (op == GNF4_OP_MOE_COMBINE) return M < 0 ? 0 : combine_workspace_bytes(M);
-  if (op == GNF4_OP_GROUPED_DGRAD) return kWsHeaderBytes;
+  if (op == GNF4_OP_GROUPED_DGRAD) return dgrad_workspace_bytes();
   if (op != GNF4_OP_GROUPED_GEMM || M < 0 || N < 1 || K < 1 || G < 1) return 0;
   const size_t d = decode_workspace_bytes(M, N, K, G, 1);
   const size_t d2 = decode_workspace_bytes(M, N, K, G, 0);
@@ -181,6 +248,24 @@ gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, const float *
   return launch_grouped_gemm(a, use, reinterpret_cast<cudaStream_t>(stream));
 }
 
+gnf4_status gnf4_grouped_gemm_ex(const gnf4_gemm_desc *desc, void *workspace, size_t ws_bytes,
+                                 gnf4_stream_t stream) {
+  if (!workspace) return GNF4_ERR_INVALID_ARGUMENT;
+  GemmArgs a;
+  int32_t use = 0;
+  const gnf4_status st = check_grouped_gemm_ex(desc, &a, &use);
+  if (st != GNF4_OK || use < 0) return st;
+  if (!is_device_pointer(workspace)) return GNF4_ERR_HOST_POINTER;
+  if (!aligned(workspace, 32)) return GNF4_ERR_MISALIGNED;
+  a.workspace = workspace;
+  a.ws_bytes = ws_bytes;
+  const size_t need = use == GNF4_MODE_PREFILL
+                          ? prefill_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu)
+                          : decode_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu);
+  if (ws_bytes < need) return GNF4_ERR_WORKSPACE_TOO_SMALL;
+  return launch_grouped_gemm(a, use, reinterpret_cast<cudaStream_t>(stream));
+}
+
 gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, int64_t rows, int32_t K,
                                int32_t blocksize, int32_t out_dtype, void *out,
                                gnf4_stream_t stream) {
@@ -206,15 +291,15 @@ gnf4_status gnf4_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float
   if (M < 0 || N < 1 || K < 1 || E < 1 || G < 1) return GNF4_ERR_INVALID_ARGUMENT;
   if (blocksize != GNF4_BLOCKSIZE || K % GNF4_BLOCKSIZE != 0) return GNF4_ERR_UNSUPPORTED_SHAPE;
   if (E > GNF4_MAX_EXPERTS || G > GNF4_MAX_EXPERTS || M >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (K / 256 + 1 > 65535) return GNF4_ERR_UNSUPPORTED_SHAPE;
-  if (ws_bytes < kWsHeaderBytes) return GNF4_ERR_WORKSPACE_TOO_SMALL;
+  if (N % 8 != 0 || static_cast<int64_t>(E) * N + 256 >= INT_MAX) return GNF4_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < dgrad_workspace_bytes()) return GNF4_ERR_WORKSPACE_TOO_SMALL;
   if (M == 0) return GNF4_OK;
   if (!is_device_pointer(dy) || !is_device_pointer(w) || !is_device_pointer(absmax) ||
       !is_device_pointer(sizes) || !is_device_pointer(expert_ids) || !is_device_pointer(dx) ||
       !is_device_pointer(workspace))
     return GNF4_ERR_HOST_POINTER;
-  if (!aligned(dy, 2) || !aligned(dx, 2) || !aligned(absmax, 4) || !aligned(sizes, 4) ||
-      !aligned(expert_ids, 4) || !aligned(workspace, 16))
+  if (!aligned(dy, 16) || !aligned(w, 16) || !aligned(dx, 2) || !aligned(absmax, 4) ||
+      !aligned(sizes, 4) || !aligned(expert_ids, 4) || !aligned(workspace, 16))
     return GNF4_ERR_MISALIGNED;
   return from_cuda(launch_grouped_dgrad(dy, w, absmax, sizes, expert_ids, G, M, N, K, E, dx,
                                         static_cast<WsHeader *>(workspace),

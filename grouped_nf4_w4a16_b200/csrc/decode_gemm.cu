@@ -1,79 +1,86 @@
-// decode_gemm.cu -- decode-regime grouped NF4 GEMM (few activation rows per expert).
+// decode_gemm.cu -- decode-regime grouped 4-bit GEMM (few activation rows per expert).
 //
 // Passage: "grouped-nf4-gemm -- single-launch W4A16 GEMM over fused NF4 MoE
 // expert stacks", opening section (one launch for all active experts, LUT
 // decode of the packed codes, blockwise fp32 absmax, fp32 accumulation, bf16
-// epilogue, no bf16 weight copy). At a handful of activation rows per expert
-// this GEMM reads every touched weight byte exactly once and is bound by HBM
-// bandwidth, so the kernel is built around keeping HBM busy: a TMA producer
-// keeps up to six 22 KB stages of packed weights in flight per SM.
+// epilogue, no bf16 weight copy) and "Status / roadmap" (split-K for starved
+// grids); package page "grouped-nf4-gemm", "Direct answer" (the same grouped
+// GEMM over native MXFP4, e2m1 codes with e8m0 scales) and "Use this when"
+// (the token gather folded into the GEMM's launch). At a handful of activation
+// rows per expert this GEMM reads every touched weight byte once and is bound
+// by HBM bandwidth, so the kernel is built around keeping HBM busy: a TMA
+// producer keeps up to six 16 KB stages of packed weights in flight per SM.
 //
-// Work decomposition (no split-K, no cross-CTA reduction)
+// Work decomposition
 //   batch  = up to 8 consecutive activation rows of one group (the MMA's N).
-//   unit   = 16 weight rows of the group's expert for one batch, over the
-//            whole of K: two row groups of 8 (with SwiGLU: 8 gate rows j..j+7
-//            and the matching 8 up rows N/2+j..). A unit's output is final
-//            when its K loop ends.
-//   The units of all groups are laid end to end (group by group, batch by
-//   batch, row by row) and every CTA (one per SM) takes an equal contiguous
-//   range, so every SM streams the same number of weight bytes. The unit
-//   list is derived on the device from (sizes, expert_ids): the host never
-//   learns which experts are active (no sync, graph-capturable).
-//   tile   = up to 8 consecutive units of one batch.
+//   unit   = 16 weight rows of the group's expert for one batch: two row
+//            groups of 8 (with SwiGLU: 8 gate rows and the matching 8 up rows).
+//   tile   = up to 8 consecutive units of one batch; a tile-stage is 256
+//            K-elements of a tile. The tiles of all groups are laid end to end
+//            (group by group, batch by batch) on the device from (sizes,
+//            expert_ids): the host never learns which experts are active.
+//   Stream-K split: the W = tiles x stages tile-stages are cut into one equal
+//   contiguous range per CTA (one CTA per SM), so every SM streams the same
+//   number of weight bytes whatever the tile count. A tile that lies inside
+//   one CTA's range is finished by it; a tile cut by range boundaries is
+//   computed in pieces: each piece leaves its fp32 partial sums in the
+//   workspace and counts itself in that tile's counter, and the piece that
+//   counts last adds the partials in piece order (deterministic), writes y and
+//   resets the counter. When tiles outnumber SMs only the few tiles at range
+//   boundaries are cut; when SMs outnumber tiles (starved grids) every tile is
+//   split across several SMs.
 //
-// Numerics: each code value is an fp16 part hi plus the fp16 of the
-// remainder times 2^13 (both round to nearest even), together within 1e-7
-// relative of the fp32 value. Activations
-// are staged as bf16 and rewritten in place as fp16 times a power of two
-// per (row, 64-element block), which the block sum divides out in fp32.
+// Formats and numerics (per stage, each consumer lane decodes packed bytes
+// through a byte-indexed table replicated per lane, so no lookup conflicts)
+//   NF4:   code value NF4[c] carried as its fp16 rounding hi; with a fused
+//          SwiGLU also the fp16 of the remainder times 2^13 (two MMAs), which
+//          together are within 1e-7 relative of the fp32 value (SwiGLU
+//          multiplies a gate error by the up value, so the gate_up GEMM of a
+//          SwiGLU layer keeps both parts). The scale is the fp32 (or bf16)
+//          absmax of the 64-element block, applied to the block's fp32 sum.
+//   MXFP4: e2m1 code values are exact in fp16 (one MMA); the e8m0 scale of
+//          each 32-element half-block is applied to its fp32 sum.
+//   Activations are staged as bf16 and rewritten in place as fp16 times a
+//   power of two per (row, 64-element block), which the block sum divides out.
 //
-// Inside a CTA (warp 16 = tensor copies, warp 17 = absmax copies, warp 18 =
-// activation conversion, warps 0-15 = consumers)
-//   Stage = 256 K-elements of a tile: the tile's weight rows as a few TMA
-//   boxes of 128 packed bytes per row (128-byte swizzle), the batch's
-//   activations as one box of 4 blocks x 8 rows x 64 bf16, and the 8 x 4
-//   absmax values of each row group (cp.async, 4 bytes each: absmax rows
-//   need not be 16-byte aligned).
+// Inside a CTA (warp 16 = tensor copies, warp 17 = scale copies and, when the
+// activations are gathered, their row copies, warp 18 = activation conversion,
+// warps 0-15 = consumers)
 //   Consumer warp w takes 64-element block w / 4 of every stage for the two
-//   units 2 (w % 4), 2 (w % 4) + 1, so one set of activation fragments
-//   serves both. Per unit, two m16n8k16 fp16 MMAs per 16 K-elements (hi,
-//   remainder) cover all 16 weight rows: A rows g and g + 8 are the unit's
-//   row groups (with SwiGLU a gate row and its up row, which the epilogue
-//   combines in registers). For each packed byte (two codes) one byte
-//   permute forms the address of a 256-byte table row replicated per lane
-//   (no bank conflicts) holding the hi pair and, 128 bytes on, the
-//   remainder pair. The block's fp32 result is scaled by absmax(row, block)
-//   and the activations' 2^-S and accumulated in fp32; when a tile's K loop
-//   ends, the pair's four block warps sum their partial results through
-//   shared memory (fixed order) and the block-0 warp writes y.
-// Every wait is bounded (2 s); on expiry the kernel records
-// GNF4_DEVERR_TIMEOUT, lets the producer's copies land and returns.
+//   units 2 (w % 4), 2 (w % 4) + 1; when a tile piece ends, the four block
+//   warps of a unit pair sum their partial results through shared memory
+//   (fixed order) and the block-0 warp writes y or the piece's partial.
+// Every wait is bounded (2 s unless the workspace header asks for less); on
+// expiry the kernel records GNF4_DEVERR_TIMEOUT, lets the producer's copies
+// land and returns.
 #include <climits>
 
 #include <cuda_fp16.h>
 
 #include "launch.h"
-#include "sm100.cuh"
+#include "lut_mma.cuh"
 
 namespace gnf4 {
 namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kTmaWarp = kConsumerWarps;          // issues the tensor copies
-constexpr int kScaleWarp = kConsumerWarps + 1;    // copies the absmax values
+constexpr int kScaleWarp = kConsumerWarps + 1;    // copies scales (and gathered activations)
 constexpr int kXWarp = kConsumerWarps + 2;        // converts the staged activations to fp16
 constexpr int kThreads = (kConsumerWarps + 3) * 32;
 constexpr int kTileUnits = 8;                 // units per tile (2 row groups each)
 constexpr int kStages = 6;
 constexpr int kBatch = 8;                     // activation rows per batch (MMA N)
 constexpr int kBoxBytes = 1024;               // 8 rows x 128 bytes
-constexpr int kStageBlocks = 4;               // absmax blocks per stage (256 K-elements)
+constexpr int kStageBlocks = 4;               // 64-element blocks per stage (256 K-elements)
 constexpr int kWStage = kTileUnits * 2 * kBoxBytes;              // 16 KB
 constexpr int kXStage = kStageBlocks * kBoxBytes;                // 4 KB
 constexpr int kXsStage = kStageBlocks * kBatch * 4;              // 128 B: 2^-S per (block, row)
-constexpr int kAStage = kTileUnits * 2 * 8 * kStageBlocks * 4;   // 2 KB
+constexpr int kAStage = kTileUnits * 2 * 8 * kStageBlocks * 4;   // 2 KB of scale words
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
 constexpr float kLoInv = 1.0f / 8192.0f;      // remainders are carried times 2^13
+constexpr int kPairs = kTileUnits / 2;        // unit pairs per tile
+constexpr int kPartialSlot = 2 * 32;          // float4 per (pair) partial: 2 units x 32 lanes
 
 // Shared memory layout, as absolute shared-window addresses. The window
 // starts with memory the driver reserves and the static tables below; the
@@ -98,143 +105,88 @@ constexpr int kLutOff = 131072;
 constexpr int kLutBytes = 256 * 256;
 constexpr int kAOff = kLutOff + kLutBytes;
 constexpr int kXchgOff = kAOff + kStages * kAStage;           // float4 [4 pairs][3][2 units][32]
-constexpr int kXchgBytes = (kTileUnits / 2) * 3 * 2 * 32 * 16;
-constexpr int kUnitStartOff = kXchgOff + kXchgBytes;          // int64 [kMaxG + 1]
-constexpr int kGExpOff = kUnitStartOff + (kMaxG + 1) * 8;     // uint16 [kMaxG]
-constexpr int kSmemEnd = kGExpOff + kMaxG * 2;
+constexpr int kXchgBytes = kPairs * 3 * 2 * 32 * 16;
+constexpr int kGExpOff = kXchgOff + kXchgBytes;               // uint16 [kMaxG]
+constexpr int kBatchOff = kGExpOff + kMaxG * 2;               // int32 [kMaxG + 1]: first batch per group
+constexpr int kSmemEnd = kBatchOff + (kMaxG + 1) * 4;
 // dynamic bytes requested: the window reaches kSmemEnd from any start >= kMinDyn
 constexpr int kSmemBytes = kSmemEnd - kMinDyn;
 static_assert(kMiscOff + 8 * 4 <= kLutOff, "low region overlaps the table");
 static_assert(kBarOff % 8 == 0 && kXOff % 1024 == 0 && kLutOff % 65536 == 0, "alignment");
 static_assert(kSmemBytes + kDynBase - kMinDyn <= 227 * 1024, "fits one CTA per SM");
 
-// ------------------------------------------------------------------ PTX
+// Scale encodings of the stack (GemmArgs::scale_kind).
+constexpr int kScaleF32 = 0;    // NF4 absmax, fp32
+constexpr int kScaleBf16 = 1;   // NF4 absmax, bf16
+constexpr int kScaleE8m0 = 2;   // MXFP4: two e8m0 bytes per 64-element block
 
-// Not volatile: the compiler may interleave independent accumulation chains.
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+// e2m1 code value (OCP microscaling FP4: sign, 2 exponent bits, 1 mantissa
+// bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), exact in fp16.
+__device__ __forceinline__ float e2m1_value(int c) {
+  const int m = c & 7;
+  const float mag = m < 2 ? 0.5f * m : static_cast<float>(2 + (m & 1)) * exp2f(static_cast<float>((m >> 1) - 2));
+  return (c & 8) ? -mag : mag;
 }
 
-// D = A.B with a zero accumulator in.
-__device__ __forceinline__ void mma_f16_z(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
-// prmt.b32 in its default mode: result byte i = byte (sel nibble i & 7) of
-// {b, a} (the selectors used here never set bit 3 of a nibble).
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-// hi and lo fp16 pairs of the 4 packed bytes of `word` (pair p: byte p),
-// from this lane's slots of the table: lutlane = shared address of the table
-// (a multiple of 65536) + lane * 4, so one byte permute forms the whole
-// address table + byte * 256 + lane * 4; the lo pair sits 128 bytes on.
-__device__ __forceinline__ void decode_word(uint32_t lutlane, uint32_t word, uint32_t (&hi)[4],
-                                            uint32_t (&lo)[4]) {
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const uint32_t a = prmt(word, lutlane, 0x7604u | (p << 4));
-    asm("ld.shared.b32 %0, [%2];\n\tld.shared.b32 %1, [%2+128];"
-        : "=r"(hi[p]), "=r"(lo[p])
-        : "r"(a));
-  }
-}
-
-// Bounded wait by every lane of the warp (no divergent branch); the lanes
-// agree on the answer by vote.
-__device__ __forceinline__ bool warp_wait_all(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, WsHeader *hdr) {
-  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr));
-}
-
-// One arrival on `bar` for the whole (converged) warp, by an elected lane.
-__device__ __forceinline__ void mbar_arrive_elect(uint64_t *bar) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
-      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
-
-__device__ __forceinline__ uint16_t bf16_bits(float v) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(v);
-  return *reinterpret_cast<const uint16_t *>(&b);
-}
-
-// hi[c]: fp16 bits of the code value (round to nearest even).
-__device__ __forceinline__ uint32_t code_hi(int c) {
-  const __half h = __float2half_rn(nf4_value(c));
-  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&h));
-}
-
-// lo[c]: fp16 bits of (NF4[c] - hi[c]) * 2^13 (round to nearest even). The
-// remainder is exact in fp32 and at most 2^-12 in magnitude, so the scaled
-// value stays below 2; hi + lo * 2^-13 is within 1e-7 relative of NF4[c].
-__device__ __forceinline__ uint32_t code_lo(int c) {
-  const __half h = __float2half_rn(nf4_value(c));
-  const __half l = __float2half_rn((nf4_value(c) - __half2float(h)) * 8192.0f);
-  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(&l));
+// 2^(s - 127) for an e8m0 byte (0xFF encodes NaN).
+__device__ __forceinline__ float e8m0_value(uint32_t s) {
+  if (s == 255u) return __uint_as_float(0x7FC00000u);
+  return s == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(s << 23);
 }
 
 struct Problem {
-  int32_t N, K, E, G, swiglu;
+  int32_t N, K, E, G;
+  int32_t epi;      // 0 none, 1 SwiGLU on the two halves, 2 SwiGLU on interleaved rows, clamped
   int32_t KB;       // 64-element blocks per row
-  int32_t KC;       // stages per unit
-  int64_t upb;      // units per batch
+  int32_t KC;       // stages per tile
+  int32_t upb;      // units per batch
+  int32_t tpb;      // tiles per batch
 };
 
 struct Tile {
   int64_t row0;     // first activation row of the batch
-  int64_t j0;       // unit index within the batch of the tile's first unit
+  int32_t j0;       // unit index within the batch of the tile's first unit
   int32_t nunits;   // 1..kTileUnits
   int32_t mrows;    // activation rows in the batch (1..8)
   int32_t e;        // expert
 };
 
-// The tile that starts at unit u (never past u_hi or the end of u's batch).
-__device__ __forceinline__ Tile make_tile(int64_t u, int64_t u_hi, const Problem &p,
-                                          const int64_t *unit_start, const int *row_off,
-                                          const uint16_t *gexp) {
-  int lo = 0, hi = p.G;   // invariant: unit_start[lo] <= u < unit_start[hi]
+// Tile t: batch t / tpb, the (t % tpb)-th run of up to 8 units of it.
+__device__ __forceinline__ Tile make_tile(int64_t t, const Problem &p, const int *batch_start,
+                                          const int *row_off, const uint16_t *gexp) {
+  const int64_t bt = t / p.tpb;
+  const int32_t jt = static_cast<int32_t>(t - bt * p.tpb);
+  int lo = 0, hi = p.G;   // invariant: batch_start[lo] <= bt < batch_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (unit_start[mid] <= u) lo = mid; else hi = mid;
+    if (batch_start[mid] <= bt) lo = mid; else hi = mid;
   }
-  const int64_t local = u - unit_start[lo];
-  const int64_t batch = local < (int64_t{1} << 31)
-                            ? static_cast<int64_t>(static_cast<uint32_t>(local) /
-                                                   static_cast<uint32_t>(p.upb))
-                            : local / p.upb;
-  const int64_t run_end = unit_start[lo] + (batch + 1) * p.upb;
-  int64_t end = u + kTileUnits;
-  if (end > u_hi) end = u_hi;
-  if (end > run_end) end = run_end;
-  Tile t;
-  t.row0 = static_cast<int64_t>(row_off[lo]) + batch * kBatch;
-  t.j0 = local - batch * p.upb;
-  t.nunits = static_cast<int32_t>(end - u);
-  t.mrows = min(kBatch, row_off[lo + 1] - row_off[lo] - static_cast<int32_t>(batch) * kBatch);
-  t.e = gexp[lo];
-  return t;
+  const int32_t lb = static_cast<int32_t>(bt) - batch_start[lo];
+  Tile tl;
+  tl.row0 = static_cast<int64_t>(row_off[lo]) + static_cast<int64_t>(lb) * kBatch;
+  tl.j0 = jt * kTileUnits;
+  tl.nunits = min(kTileUnits, p.upb - tl.j0);
+  tl.mrows = min(kBatch, row_off[lo + 1] - row_off[lo] - lb * kBatch);
+  tl.e = gexp[lo];
+  return tl;
 }
 
-// Packed-weight tensor maps with boxes of 8, 16, 32, 64 and 128 rows x 128
-// bytes: a tile's contiguous rows are fetched with a few large copies.
+// Where piece (tile t, CTA c) keeps its partial sums: slot 0 if t is the
+// first tile c touches, slot 1 if it is the last one (a cut tile is always
+// one of the two for every CTA that holds a piece of it).
+__device__ __forceinline__ int64_t piece_slot(int64_t W, int64_t P, int64_t KC, int64_t t,
+                                              int64_t c) {
+  return c * 2 + (range_lo(W, P, c) / KC == t ? 0 : 1);
+}
+
+// Packed-weight tensor maps: boxes of 8, 16, 32, 64 and 128 rows x 128 bytes
+// over [E*N rows][K/2 bytes] (2-D), and for interleaved gate/up rows, boxes
+// of 8, 16, 32 and 64 rows of one parity over [E*N/2 pairs][2][K/2] (3-D).
 constexpr int kNumWMaps = 5;
+constexpr int kNumIMaps = 4;
 struct WeightMaps {
   CUtensorMap m[kNumWMaps];   // m[i]: boxes of (8 << i) rows
+  CUtensorMap im[kNumIMaps];  // im[i]: boxes of (8 << i) rows of one parity (epilogue 2 only)
 };
 
 // Copies `nrows` (a multiple of 8) consecutive weight rows, 128 bytes of
@@ -252,13 +204,100 @@ __device__ __forceinline__ void load_weight_rows(char *dst, const WeightMaps &wm
   }
 }
 
+// Copies rows 2 (pair0 + i) + parity, i < npairs (a multiple of 8), as
+// consecutive 128-byte rows.
+__device__ __forceinline__ void load_parity_rows(char *dst, const WeightMaps &wm, int c0,
+                                                 int64_t pair0, int parity, int npairs,
+                                                 uint64_t *bar) {
+  int done = 0;
+#pragma unroll
+  for (int i = kNumIMaps - 1; i >= 0; --i) {
+    const int h = 8 << i;
+    while (npairs - done >= h) {
+      tma_load_3d(dst + done * 128, &wm.im[i], c0, parity, static_cast<int>(pair0 + done), bar);
+      done += h;
+    }
+  }
+}
+
+struct DecodeParams {
+  const void *scales;          // fp32 / bf16 absmax [E][N][K/64], or e8m0 [E][N][K/32]
+  const int32_t *sizes;
+  const int32_t *expert_ids;
+  const uint16_t *hidden;      // gathered activations [T][K] (nullptr: x through the tensor map)
+  const int32_t *sorted_idx;   // [M] slot of each row (gather)
+  int64_t n_slots;             // T * top_k (gather)
+  int32_t top_k;               // (gather)
+  int32_t G;
+  int64_t M;
+  int32_t N, K, E;
+  int32_t scale_kind;
+  int32_t epi;
+  float alpha, limit;          // epilogue 2
+  uint16_t *y;
+  WsHeader *hdr;
+  uint32_t *counters;          // [P][kPairs]
+  float4 *partials;            // [P][2][kPairs][kPartialSlot]
+};
+
+// The output of one unit pair (acc[uu][*], C-fragment order) for tile tl.
+__device__ __forceinline__ void store_outputs(uint16_t *y, float alpha, float limit,
+                                              const Problem &p, const Tile &tl, int up, int g,
+                                              int q, const float (&acc)[2][4], bool act1) {
+  const int64_t ncols = p.epi ? p.N / 2 : p.N;
+#pragma unroll
+  for (int uu = 0; uu < 2; ++uu) {
+    if (uu == 1 && !act1) break;
+    const int64_t j = tl.j0 + 2 * up + uu;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int m = 2 * q + i;
+      if (m >= tl.mrows) continue;
+      uint16_t *yr = y + (tl.row0 + m) * ncols;
+      const float a0 = acc[uu][i], a1 = acc[uu][2 + i];
+      if (p.epi == 0) {
+        const int64_t c0 = 16 * j + g, c1 = 16 * j + 8 + g;
+        if (c0 < p.N) yr[c0] = bf16_bits(a0);
+        if (c1 < p.N) yr[c1] = bf16_bits(a1);
+      } else {
+        const int64_t c = 8 * j + g;
+        if (c >= ncols) continue;
+        float o;
+        if (p.epi == 1) {
+          o = silu(a0) * a1;
+        } else {   // clamped gate and up, gate * sigmoid(alpha * gate) * (up + 1)
+          const float gt = fminf(a0, limit);
+          const float u = fminf(fmaxf(a1, -limit), limit);
+          o = gt / (1.0f + expf(-alpha * gt)) * (u + 1.0f);
+        }
+        yr[c] = bf16_bits(o);
+      }
+    }
+  }
+}
+
+// PARTS: fp16 parts per NF4 code value (1 or 2). SK: the scale encoding
+// (kScaleF32, kScaleBf16, or kScaleE8m0 for MXFP4, which is one part).
+template <int PARTS, int SK>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gemm_kernel(const __grid_constant__ WeightMaps wmaps,
-                       const __grid_constant__ CUtensorMap xmap, const float *__restrict__ absmax,
-                       const int32_t *__restrict__ sizes, const int32_t *__restrict__ expert_ids,
-                       int32_t G, int64_t M, int32_t N, int32_t K, int32_t E, int32_t swiglu,
-                       uint16_t *__restrict__ y, WsHeader *hdr) {
+                       const __grid_constant__ CUtensorMap xmap,
+                       const __grid_constant__ DecodeParams a) {
+  constexpr bool MX = SK == kScaleE8m0;
   extern __shared__ __align__(1024) char smem_raw[];
+  // The parameters the loops use, as locals: the parameter block's address
+  // is never taken, so every use is a constant-bank operand, not a load that
+  // the asm statements' memory clobbers would force to repeat.
+  WsHeader *hdr = a.hdr;
+  const void *const scales = a.scales;
+  constexpr int scale_kind = SK;
+  const uint16_t *const hidden = a.hidden;
+  const int32_t *const sorted_idx = a.sorted_idx;
+  const int32_t top_k = a.top_k;
+  uint16_t *const yout = a.y;
+  const float alpha = a.alpha, limit = a.limit;
+  float4 *const partials = a.partials;
+  uint32_t *const counters = a.counters;
   // generic pointer of shared-window address 0: smem + kXxxOff is region kXxx
   const uint32_t dyn0 = smem_u32(smem_raw);
   char *smem = smem_raw - dyn0;
@@ -273,26 +312,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return;
   }
-  int64_t *unit_start = reinterpret_cast<int64_t *>(smem + kUnitStartOff);
   int *row_off = reinterpret_cast<int *>(smem + kRowOffOff);
+  int *batch_start = reinterpret_cast<int *>(smem + kBatchOff);
   uint16_t *gexp = reinterpret_cast<uint16_t *>(smem + kGExpOff);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
   uint64_t *empty = full + kStages;
   uint64_t *xready = empty + kStages;
-  uint64_t *xfull = xready + kStages;          // [kTileUnits / 2]
-  uint64_t *xempty = xfull + kTileUnits / 2;   // [kTileUnits / 2]
+  uint64_t *xfull = xready + kStages;          // [kPairs]
+  uint64_t *xempty = xfull + kPairs;           // [kPairs]
   int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort
   volatile int *abort_flag = &misc[1];
-  __shared__ int64_t s_tot;   // total units (written by warp 0 with the group table)
+  __shared__ int s_tot;       // total batches (written by warp 0 with the group table)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();
 
   Problem p;
-  p.N = N; p.K = K; p.E = E; p.G = G; p.swiglu = swiglu;
-  p.KB = K / 64;
+  p.N = a.N; p.K = a.K; p.E = a.E; p.G = a.G; p.epi = a.epi;
+  p.KB = a.K / 64;
   p.KC = (p.KB + kStageBlocks - 1) / kStageBlocks;
-  p.upb = swiglu ? (N / 2 + 7) / 8 : (N + 15) / 16;
+  p.upb = a.epi ? (a.N / 2 + 7) / 8 : (a.N + 15) / 16;
+  p.tpb = (p.upb + kTileUnits - 1) / kTileUnits;
+  const bool gather = hidden != nullptr;
 
   if (tid == 0) {
     misc[0] = 0;
@@ -302,106 +343,104 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], kConsumerWarps);
       mbar_init(&xready[s], 1);
     }
-    for (int i = 0; i < kTileUnits / 2; ++i) {
+    for (int i = 0; i < kPairs; ++i) {
       mbar_init(&xfull[i], 3);
       mbar_init(&xempty[i], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int i = 0; i < kNumWMaps; ++i) prefetch_tensormap(&wmaps.m[i]);
-    prefetch_tensormap(&xmap);
+    if (a.epi == 2)
+      for (int i = 0; i < kNumIMaps; ++i) prefetch_tensormap(&wmaps.im[i]);
+    if (!gather) prefetch_tensormap(&xmap);
   }
 
-  // ---- decode table: row b, lane slot l: the fp16 pair (hi[b >> 4],
-  //      hi[b & 15]) at l * 4 and the pair of remainders at 128 + l * 4 (low
-  //      half = even k = high nibble)
-  if (tid < 256) {
-    const uint32_t hp = code_hi(tid >> 4) | (code_hi(tid & 15) << 16);
-    const uint32_t lp = code_lo(tid >> 4) | (code_lo(tid & 15) << 16);
-    uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + tid * 256);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      dst[i] = make_uint4(hp, hp, hp, hp);
-      dst[8 + i] = make_uint4(lp, lp, lp, lp);
+  // ---- decode table: row b, lane slot l: the fp16 pair of byte b's two code
+  //      values (low half = even k) at l * 4 and (NF4 with two parts) the pair
+  //      of remainders at 128 + l * 4. NF4 puts even k in the high nibble,
+  //      MXFP4 in the low nibble.
+  for (int i = tid; i < 256 * 8; i += kThreads) {
+    const int b = i >> 3, part = i & 7;
+    uint32_t hp, lp = 0u;
+    if (MX) {
+      hp = half_bits(e2m1_value(b & 15)) | (half_bits(e2m1_value(b >> 4)) << 16);
+    } else {
+      hp = code_hi(b >> 4) | (code_hi(b & 15) << 16);
+      if (PARTS == 2) lp = code_lo(b >> 4) | (code_lo(b & 15) << 16);
     }
+    uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + b * 256);
+    dst[part] = make_uint4(hp, hp, hp, hp);
+    if (PARTS == 2) dst[8 + part] = make_uint4(lp, lp, lp, lp);
   }
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
+  // bounded waits give up after the header's limit when it sets one
+  const uint64_t limit_ns = hdr->reserved[0] ? static_cast<uint64_t>(hdr->reserved[0]) : kTimeoutNs;
 
   // ---- group table from (sizes, expert_ids), validated on the device: built
   //      by warp 0 alone (its lanes' loads in flight together, one warp scan),
-  //      then one block barrier publishes it with the barrier set-up.
+  //      then one block barrier publishes it with the barrier set-up. With a
+  //      gather, every row's slot is checked too, before any work.
   if (warp == 0) {
-    const int per = (G + 31) / 32;
-    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
-    int64_t my_rows = 0, my_units = 0;
+    const int per = (p.G + 31) / 32;
+    const int g0 = min(p.G, lane * per), g1 = min(p.G, g0 + per);
+    int64_t my_rows = 0, my_batches = 0;
     int bad = 0;
     for (int g = g0; g < g1; ++g) {
-      const int sz = sizes[g];
-      const int e = expert_ids[g];
+      const int sz = a.sizes[g];
+      const int e = a.expert_ids[g];
       if (sz < 0) bad |= GNF4_DEVERR_SIZES;
-      if (sz > 0 && (e < 0 || e >= E)) bad |= GNF4_DEVERR_EXPERT;
+      if (sz > 0 && (e < 0 || e >= p.E)) bad |= GNF4_DEVERR_EXPERT;
       gexp[g] = static_cast<uint16_t>(e);
       row_off[g] = sz;   // kept here until the offsets are known
       my_rows += max(sz, 0);
-      my_units += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
+      my_batches += sz > 0 ? (sz + kBatch - 1) / kBatch : 0;
     }
-    int64_t vr = my_rows, vu = my_units;   // inclusive scan over the lanes
+    int64_t vr = my_rows, vb = my_batches;   // inclusive scan over the lanes
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int64_t a = __shfl_up_sync(0xffffffffu, vr, o);
-      const int64_t b = __shfl_up_sync(0xffffffffu, vu, o);
-      if (lane >= o) { vr += a; vu += b; }
+      const int64_t x0 = __shfl_up_sync(0xffffffffu, vr, o);
+      const int64_t x1 = __shfl_up_sync(0xffffffffu, vb, o);
+      if (lane >= o) { vr += x0; vb += x1; }
     }
     const int64_t tot_r = __shfl_sync(0xffffffffu, vr, 31);
-    const int64_t tot_u = __shfl_sync(0xffffffffu, vu, 31);
-    int64_t r = vr - my_rows, c = vu - my_units;
+    const int64_t tot_b = __shfl_sync(0xffffffffu, vb, 31);
+    int64_t r = vr - my_rows, c = vb - my_batches;
     for (int g = g0; g < g1; ++g) {
       const int sz = max(row_off[g], 0);
       row_off[g] = static_cast<int>(r);
-      unit_start[g] = c;
+      batch_start[g] = static_cast<int>(c);
       r += sz;
-      c += sz > 0 ? ((sz + kBatch - 1) / kBatch) * p.upb : 0;
+      c += sz > 0 ? (sz + kBatch - 1) / kBatch : 0;
+    }
+    if (tot_r == a.M && gather) {
+      for (int64_t i = lane; i < a.M; i += 32) {
+        const int32_t sl = sorted_idx[i];
+        if (sl < 0 || sl >= a.n_slots) bad |= GNF4_DEVERR_SLOT;
+      }
     }
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (lane == 0) {
-      unit_start[G] = tot_u;
-      row_off[G] = static_cast<int>(tot_r);
-      if (tot_r != M) bad |= GNF4_DEVERR_SIZES;
-      s_tot = tot_u;
+      batch_start[p.G] = static_cast<int>(tot_b);
+      row_off[p.G] = static_cast<int>(tot_r);
+      if (tot_r != a.M) bad |= GNF4_DEVERR_SIZES;
+      s_tot = static_cast<int>(tot_b);
       misc[0] = bad;
     }
   }
   __syncthreads();   // group table, barrier set-up and misc visible
-  const int64_t tot_u = s_tot;
   const int errbits = misc[0];
   if (errbits) {
     if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
     return;
   }
-  // Whole tiles, not units, are split across CTAs: a tile costs KC stages
-  // whatever its unit count, so a unit range cutting through a batch's tiles
-  // would cost its CTA an extra tile (twice the stages when every CTA holds
-  // about one tile). Each batch has upb units in tpb = ceil(upb / 8) tiles;
-  // this CTA takes tiles [T b / P, T (b + 1) / P) of the T = B tpb, B =
-  // tot_u / upb batches (32-bit arithmetic when T fits: q P + r gives
-  // q b + r b / P).
-  const int64_t tpb = (p.upb + kTileUnits - 1) / kTileUnits;
-  const int64_t T = (tot_u / p.upb) * tpb;
-  const int64_t P = gridDim.x;
-  int64_t u_lo, u_hi;
-  if (T < (int64_t{1} << 31) && p.upb < (int64_t{1} << 31)) {
-    const uint32_t tt = static_cast<uint32_t>(T), Pu = gridDim.x, bu = blockIdx.x;
-    const uint32_t q = tt / Pu, rr = tt - q * Pu;
-    const uint32_t t_lo = q * bu + rr * bu / Pu, t_hi = q * (bu + 1) + rr * (bu + 1) / Pu;
-    const uint32_t tp = static_cast<uint32_t>(tpb);
-    u_lo = static_cast<int64_t>(t_lo / tp) * p.upb + static_cast<int64_t>(t_lo % tp) * kTileUnits;
-    u_hi = static_cast<int64_t>(t_hi / tp) * p.upb + static_cast<int64_t>(t_hi % tp) * kTileUnits;
-  } else {
-    const int64_t t_lo = T * blockIdx.x / P, t_hi = T * (blockIdx.x + 1) / P;
-    u_lo = (t_lo / tpb) * p.upb + (t_lo % tpb) * kTileUnits;
-    u_hi = (t_hi / tpb) * p.upb + (t_hi % tpb) * kTileUnits;
-  }
-  if (u_lo >= u_hi) return;
+  const int64_t T = static_cast<int64_t>(s_tot) * p.tpb;   // tiles
+  const int64_t KC = p.KC;
+  const int64_t W = T * KC;                                 // tile-stages
+  // CTAs beyond the tile-stage count take nothing, so every range is non-empty
+  // and the pieces of a cut tile are exactly the CTAs cta_of() names
+  const int64_t P = min(static_cast<int64_t>(gridDim.x), W);
+  if (static_cast<int64_t>(blockIdx.x) >= P) return;
+  const int64_t s_lo = range_lo(W, P, blockIdx.x), s_hi = range_lo(W, P, blockIdx.x + 1);
 
   if (warp == kXWarp) {
     // ------------------------------------------------ activation conversion
@@ -412,15 +451,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the stage's scale table for the consumers' block sums.
     const int b = lane >> 3, r = lane & 7;
     uint32_t it = 0;
-    for (int64_t u = u_lo; u < u_hi;) {
-      const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
-      for (int kc = 0; kc < p.KC; ++kc, ++it) {
-        const int s = static_cast<int>(it % kStages);
+    for (int64_t s = s_lo; s < s_hi;) {
+      const int64_t t = s / KC;
+      const int k0 = static_cast<int>(s - t * KC);
+      const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
+      const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
+      for (int kc = k0; kc < k1; ++kc, ++it) {
+        const int st = static_cast<int>(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
-        if (!warp_wait_bar(&full[s], ph, abort_flag, hdr)) return;
+        if (!warp_wait_one(&full[st], ph, abort_flag, hdr, limit_ns)) return;
         // rows past the batch feed only outputs that are never stored: skipped
-        if (r < t.mrows) {
-          char *row = smem + kXOff + s * kXStage + b * kBoxBytes + r * 128;
+        if (r < tl.mrows) {
+          char *row = smem + kXOff + st * kXStage + b * kBoxBytes + r * 128;
           uint4 v[8];
           // bf16 magnitudes compare as integers, two per word; four
           // independent chains keep the reduction short
@@ -452,13 +494,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             *reinterpret_cast<uint4 *>(row + ((c ^ r) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
           }
-          reinterpret_cast<float *>(smem + kXsOff + s * kXsStage)[lane] =
+          reinterpret_cast<float *>(smem + kXsOff + st * kXsStage)[lane] =
               __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&xready[s]);
+        if (lane == 0) mbar_arrive(&xready[st]);
       }
-      u += t.nunits;
+      s += k1 - k0;
     }
     return;
   }
@@ -466,65 +508,121 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= kTmaWarp) {
     // ------------------------------------------------------------ producers
     // Two warps fill each stage: the copy warp issues the tensor copies (one
-    // byte-count arrival), the scale warp the 4-byte absmax copies (one
-    // arrival per lane when its copies land). Split so that neither issue
-    // stream waits behind the other.
+    // byte-count arrival), the scale warp the 4-byte scale copies and, with a
+    // gather, the activation rows as 16-byte copies (one arrival per lane
+    // when its copies land). Split so that neither issue stream waits behind
+    // the other.
     const bool scale_warp = warp == kScaleWarp;
     const int r = lane >> 2, blk = lane & 3;
-    const int64_t total_rows = static_cast<int64_t>(E) * N;
-    const int64_t di = swiglu ? 8 : 16;            // rows from one unit to the next
-    const int64_t dr = swiglu ? N / 2 : 8;         // rows from row group 0 to row group 1
+    const int64_t total_rows = static_cast<int64_t>(p.E) * p.N;
+    // scale bytes of the whole stack (2-byte encodings: the last word read
+    // must stay inside it)
+    const int64_t scale_bytes = total_rows * p.KB * 2;
+    // gathered activations: lane copies row gr = lane % 8 of block gb = lane / 8
+    const int gr = lane & 7, gb = lane >> 3;
     uint32_t it = 0;
     bool ok = true;
-    for (int64_t u = u_lo; u < u_hi && ok;) {
-      const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
-      const int64_t row0 = static_cast<int64_t>(t.e) * N + di * t.j0;   // first weight row
-      // absmax source of this lane (row r, block blk) for each row group slot
-      const int64_t arow = row0 + r;
-      uint32_t vmask = 0;   // bit 2i+rgi: that row exists in the stack
+    for (int64_t s = s_lo; s < s_hi && ok;) {
+      const int64_t t = s / KC;
+      const int k0 = static_cast<int>(s - t * KC);
+      const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
+      const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
+      const int64_t ebase = static_cast<int64_t>(tl.e) * p.N;
+      // weight row of unit i, row group rgi, row r within the group
+      auto wrow = [&](int i, int rgi, int rr) -> int64_t {
+        const int64_t j = tl.j0 + i;
+        if (p.epi == 0) return ebase + 16 * j + 8 * rgi + rr;
+        if (p.epi == 1) return ebase + 8 * j + rr + rgi * (p.N / 2);
+        return ebase + 2 * (8 * j + rr) + rgi;
+      };
+      uint32_t vmask = 0;   // bit 2i+rgi: row r of that row group exists in the stack
+      const uint16_t *hrow = nullptr;
+      // scale elements: of row r of unit 0 / row group 0 at block blk, and
+      // the steps from one unit and from one row group to the next
+      const int64_t e00 = wrow(0, 0, r) * p.KB + blk;
+      const int64_t du = (wrow(1, 0, r) - wrow(0, 0, r)) * p.KB;
+      const int64_t dg = (wrow(0, 1, r) - wrow(0, 0, r)) * p.KB;
       if (scale_warp) {
-        for (int i = 0; i < t.nunits; ++i)
+        for (int i = 0; i < tl.nunits; ++i)
 #pragma unroll
           for (int rgi = 0; rgi < 2; ++rgi)
-            if (arow + i * di + rgi * dr < total_rows) vmask |= 1u << (2 * i + rgi);
+            if (wrow(i, rgi, r) < ebase + p.N) vmask |= 1u << (2 * i + rgi);
+        if (gather && gr < tl.mrows) {
+          const int32_t slot = sorted_idx[tl.row0 + gr];   // checked in range up front
+          hrow = hidden + static_cast<int64_t>(slot / top_k) * p.K;
+        }
       }
-      const float *abase = absmax + arow * p.KB + blk;
-      for (int kc = 0; kc < p.KC; ++kc, ++it) {
-        const int s = static_cast<int>(it % kStages);
+      for (int kc = k0; kc < k1; ++kc, ++it) {
+        const int st = static_cast<int>(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
-        if (!warp_wait_bar(&empty[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
+        if (!warp_wait_one(&empty[st], ph ^ 1u, abort_flag, hdr, limit_ns)) { ok = false; break; }
         if (scale_warp) {
-          // stage layout [unit][block][row][row group]: a consumer lane reads
-          // both row groups of its row in one 8-byte load
-          char *as = smem + kAOff + s * kAStage + (blk * 8 + r) * 8;
+          // stage layout [unit][block][row][row group], one 4-byte word each:
+          // a consumer lane reads both row groups of its row in one 8-byte load
+          const uint32_t as = smem_u32(smem + kAOff + st * kAStage + (blk * 8 + r) * 8);
           const bool kok = kc * kStageBlocks + blk < p.KB;
-          for (int i = 0; i < t.nunits; ++i) {
+          const int64_t ek = e00 + kc * kStageBlocks;   // element of unit 0, row group 0
+          if (scale_kind == kScaleF32) {
+            const float *fk = static_cast<const float *>(scales) + ek;
+            for (int i = 0; i < tl.nunits; ++i) {
 #pragma unroll
-            for (int rgi = 0; rgi < 2; ++rgi) {
-              const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
-              const float *src = abase + ((i * di + rgi * dr) * p.KB + kc * kStageBlocks);
-              cp_async4(smem_u32(as + i * 256 + rgi * 4), v ? src : absmax, v ? 4u : 0u);
+              for (int rgi = 0; rgi < 2; ++rgi) {
+                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
+                cp_async4(as + i * 256 + rgi * 4, v ? fk + i * du + rgi * dg : scales, v ? 4u : 0u);
+              }
+            }
+          } else {
+            // the 4-byte word that holds the (row, block)'s 2 bytes (the last
+            // word of the stack is read only as far as the stack goes)
+            const char *cb = static_cast<const char *>(scales);
+            for (int i = 0; i < tl.nunits; ++i) {
+#pragma unroll
+              for (int rgi = 0; rgi < 2; ++rgi) {
+                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
+                const int64_t wb = ((ek + i * du + rgi * dg) * 2) & ~int64_t{3};
+                cp_async4(as + i * 256 + rgi * 4, v ? cb + wb : scales,
+                          v ? (wb + 4 <= scale_bytes ? 4u : 2u) : 0u);
+              }
             }
           }
-          cp_async_arrive_noinc(&full[s]);
+          if (gather) {
+            // the batch's rows of x for this stage's 4 blocks, through
+            // sorted_idx, into the layout the tensor copy gives (128-byte
+            // swizzle: chunk c of row r at chunk c ^ r); rows past the batch
+            // and blocks past K are zero-filled
+            const int kbx = kc * kStageBlocks + gb;
+            const bool v = hrow != nullptr && kbx < p.KB;
+            const uint32_t dst = smem_u32(smem + kXOff + st * kXStage + gb * kBoxBytes + gr * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              cp_async16(dst + ((c ^ gr) << 4), v ? hrow + kbx * 64 + c * 8 : hidden,
+                         v ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(&full[st]);
         } else if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s],
-                                static_cast<uint32_t>(t.nunits * 16 * 128 + kXStage));
-          char *ws = smem + kWOff + s * kWStage;
-          if (!swiglu) {
-            load_weight_rows(ws, wmaps, kc * 128, row0, t.nunits * 16, &full[s]);
-          } else {   // gate rows, then the matching up rows 8 KB further
-            load_weight_rows(ws, wmaps, kc * 128, row0, t.nunits * 8, &full[s]);
-            load_weight_rows(ws + kTileUnits * kBoxBytes, wmaps, kc * 128, row0 + N / 2,
-                             t.nunits * 8, &full[s]);
+          mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(tl.nunits * 16 * 128 +
+                                                                 (gather ? 0 : kXStage)));
+          char *ws = smem + kWOff + st * kWStage;
+          if (p.epi == 0) {
+            load_weight_rows(ws, wmaps, kc * 128, wrow(0, 0, 0), tl.nunits * 16, &full[st]);
+          } else if (p.epi == 1) {   // gate rows, then the matching up rows 8 KB further
+            load_weight_rows(ws, wmaps, kc * 128, wrow(0, 0, 0), tl.nunits * 8, &full[st]);
+            load_weight_rows(ws + kTileUnits * kBoxBytes, wmaps, kc * 128, wrow(0, 1, 0),
+                             tl.nunits * 8, &full[st]);
+          } else {                   // interleaved: even rows (gate), then odd rows (up)
+            const int64_t pair0 = (ebase >> 1) + 8 * static_cast<int64_t>(tl.j0);
+            load_parity_rows(ws, wmaps, kc * 128, pair0, 0, tl.nunits * 8, &full[st]);
+            load_parity_rows(ws + kTileUnits * kBoxBytes, wmaps, kc * 128, pair0, 1,
+                             tl.nunits * 8, &full[st]);
           }
           // the batch's activations for the stage's 4 blocks in one copy (a
           // block past K is zero-filled by the copy engine)
-          tma_load_3d(smem + kXOff + s * kXStage, &xmap, 0, static_cast<int>(t.row0),
-                      kc * kStageBlocks, &full[s]);
+          if (!gather)
+            tma_load_3d(smem + kXOff + st * kXStage, &xmap, 0, static_cast<int>(tl.row0),
+                        kc * kStageBlocks, &full[st]);
         }
       }
-      u += t.nunits;
+      s += k1 - k0;
     }
     if (scale_warp) {
       cp_async_wait_all();
@@ -542,102 +640,153 @@ __global__ void __launch_bounds__(kThreads, 1)
   // --------------------------------------------------------------- consumers
   // Warp w takes 64-element block w / 4 of every stage for units 2 (w % 4)
   // and 2 (w % 4) + 1 of the tile; the four block warps of a unit pair sum
-  // their partial results when the tile's K loop ends.
+  // their partial results when the tile piece ends.
   const int g = lane >> 2, q = lane & 3;
   const int up = warp & 3;                  // unit pair
   const int blk = warp >> 2;                // block of the stage
-  // This lane's K-elements of a block: the 8 of 16-byte activation chunk f
-  // and the 8 of chunk f ^ 4 (packed bytes 4 f .. 4 f + 3 and 4 (f ^ 4) ..),
-  // f = 0, 5, 2, 7 for q = 0..3. With the 128-byte swizzle (chunk ^ row):
-  // f & 3 takes every value, so a warp's 4-byte packed-word reads hit 32
-  // distinct banks; and no two values of f differ only in bit 0, so the 8
-  // lanes (rows g, g + 1) that share a 16-byte activation read's wavefront
-  // hit 8 distinct chunks. Both reads run free of bank conflicts.
+  // This lane's K-elements of a block: the 8 of 16-byte activation chunk cA
+  // = q and the 8 of chunk cB = q + 4 (packed bytes 4 cA .. 4 cA + 3 of the
+  // block, and 16 bytes on). The first two MMAs of a block take chunks 0..3
+  // (the block's first 32 elements), the last two chunks 4..7, which MXFP4's
+  // per-32 scales need. With the 128-byte swizzle (chunk ^ row) the packed
+  // words of chunk q of rows g = 0..7 fall in 32 distinct banks. The
+  // activation chunks are read in the order f, f ^ 4 with f = 0, 5, 2, 7 for
+  // q = 0..3 (f is cA or cB): no two values of f differ only in bit 0, so the
+  // 8 lanes (rows g, g + 1) that share a 16-byte read's wavefront hit 8
+  // distinct chunks; lanes with odd q swap the two reads back afterwards.
+  // Both reads run free of bank conflicts.
+  // (NF4 sums all four MMAs of a block into one value, so its lanes simply
+  // take chunk f for the first two MMAs and f ^ 4 for the last two: no swap.)
   const int f = (q & 2) | ((q & 1) ? 5 : 0);
-  const int offA = g * 128 + (((2 * blk + (f >> 2)) ^ g) << 4) + 4 * (f & 3);
-  const int offB = g * 128 + (((2 * blk + 1 - (f >> 2)) ^ g) << 4) + 4 * (f & 3);
-  const int xoffA = blk * kBoxBytes + g * 128 + ((f ^ g) << 4);
-  const int xoffB = blk * kBoxBytes + g * 128 + ((f ^ 4 ^ g) << 4);
+  const int cA = MX ? q : f, cB = MX ? (q | 4) : (f ^ 4);
+  const int offA = g * 128 + (((2 * blk + (cA >> 2)) ^ g) << 4) + 4 * (cA & 3);
+  const int offB = g * 128 + (((2 * blk + (cB >> 2)) ^ g) << 4) + 4 * (cB & 3);
+  const int xoffF = blk * kBoxBytes + g * 128 + ((f ^ g) << 4);
+  const int xoffG = blk * kBoxBytes + g * 128 + ((f ^ 4 ^ g) << 4);
+  const bool xswap = MX && (q & 1) != 0;
   const uint32_t lutlane = static_cast<uint32_t>(kLutOff) | (static_cast<uint32_t>(lane) * 4u);
-  const int64_t ncols = swiglu ? N / 2 : N;
+  constexpr bool two_byte = SK != kScaleF32;
   // partial sums of block warp b (1..3) for unit uu of the pair
   auto xchg_at = [&](int b, int uu) -> float4 * {
     return reinterpret_cast<float4 *>(smem + kXchgOff) + ((up * 3 + (b - 1)) * 2 + uu) * 32 + lane;
   };
   uint32_t it = 0, ep = 0;
-  for (int64_t u = u_lo; u < u_hi;) {
-    const Tile t = make_tile(u, u_hi, p, unit_start, row_off, gexp);
-    const bool act0 = 2 * up < t.nunits, act1 = 2 * up + 1 < t.nunits;
+  for (int64_t s = s_lo; s < s_hi;) {
+    const int64_t t = s / KC;
+    const int k0 = static_cast<int>(s - t * KC);
+    const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
+    const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
+    const bool act0 = 2 * up < tl.nunits, act1 = 2 * up + 1 < tl.nunits;
+    const int64_t ebase = static_cast<int64_t>(tl.e) * p.N;
     // C fragment: [0] weight row g, activation row 2q; [1] row g, 2q + 1;
     // [2] row g + 8 (SwiGLU: the matching up row), 2q; [3] row g + 8, 2q + 1
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    for (int kc = 0; kc < p.KC; ++kc, ++it) {
-      const int s = static_cast<int>(it % kStages);
+    for (int kc = k0; kc < k1; ++kc, ++it) {
+      const int st = static_cast<int>(it % kStages);
       const uint32_t ph = (it / kStages) & 1u;
       // the activation warp arrives on xready only after it has observed
       // this stage's copies complete (full), so this one wait also orders
-      // the copied weights and absmax before the reads below
-      if (!warp_wait_all(&xready[s], ph, abort_flag, hdr)) return;
+      // the copied weights and scales before the reads below
+      if (!warp_wait_all(&xready[st], ph, abort_flag, hdr, limit_ns)) return;
       if (act0) {
-        // A block past K reads zero-filled activations and absmax: it adds 0.
-        const char *wst = smem + kWOff + s * kWStage;
+        // A block past K reads zero-filled activations and scales: it adds 0.
+        const char *wst = smem + kWOff + st * kWStage;
         // 2^-S of activation rows 2q and 2q + 1 in this block
-        const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + s * kXsStage)[blk * 4 + q];
-        const char *ast = smem + kAOff + s * kAStage + (blk * 8 + g) * 8;
+        const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + st * kXsStage)[blk * 4 + q];
+        const char *ast = smem + kAOff + st * kAStage + (blk * 8 + g) * 8;
         // (rows past the batch feed only outputs that are never stored)
-        const char *xst = smem + kXOff + s * kXStage;
-        const uint4 xa = *reinterpret_cast<const uint4 *>(xst + xoffA);
-        const uint4 xb = *reinterpret_cast<const uint4 *>(xst + xoffB);
+        const char *xst = smem + kXOff + st * kXStage;
+        const uint4 xf = *reinterpret_cast<const uint4 *>(xst + xoffF);
+        const uint4 xg = *reinterpret_cast<const uint4 *>(xst + xoffG);
+        const uint4 xa = xswap ? xg : xf;   // chunk cA
+        const uint4 xb = xswap ? xf : xg;   // chunk cB
+        const int kb = kc * kStageBlocks + blk;
 #pragma unroll
         for (int uu = 0; uu < 2; ++uu) {
           if (uu == 1 && !act1) break;
           const int ui = 2 * up + uu;
           // weight rows g and g + 8 of the unit (1 KB boxes of 8 rows)
-          const char *r0 = wst + (swiglu ? ui : 2 * ui) * kBoxBytes;
-          const char *r1 = wst + (swiglu ? kTileUnits + ui : 2 * ui + 1) * kBoxBytes;
+          const char *r0 = wst + (p.epi ? ui : 2 * ui) * kBoxBytes;
+          const char *r1 = wst + (p.epi ? kTileUnits + ui : 2 * ui + 1) * kBoxBytes;
           const uint32_t wa0 = *reinterpret_cast<const uint32_t *>(r0 + offA);
           const uint32_t wb0 = *reinterpret_cast<const uint32_t *>(r0 + offB);
           const uint32_t wa1 = *reinterpret_cast<const uint32_t *>(r1 + offA);
           const uint32_t wb1 = *reinterpret_cast<const uint32_t *>(r1 + offB);
-          const float2 amv = *reinterpret_cast<const float2 *>(ast + ui * 256);
-          const float am0 = amv.x, am1 = amv.y;   // rows g and g + 8
+          const uint2 sw = *reinterpret_cast<const uint2 *>(ast + ui * 256);   // rows g, g + 8
+          // the 2 scale bytes of (row, block) sit in the low or the high half
+          // of the copied 4-byte word, as the element index is even or odd
+          uint32_t s0 = sw.x, s1 = sw.y;
+          if (two_byte) {
+            const int64_t j = tl.j0 + ui;
+            const int64_t w0 = p.epi == 0 ? ebase + 16 * j + g
+                               : (p.epi == 1 ? ebase + 8 * j + g : ebase + 2 * (8 * j + g));
+            const int64_t w1 = p.epi == 0 ? w0 + 8 : (p.epi == 1 ? w0 + p.N / 2 : w0 + 1);
+            const uint32_t h0 = static_cast<uint32_t>((w0 * p.KB + kb) & 1);
+            const uint32_t h1 = static_cast<uint32_t>((w1 * p.KB + kb) & 1);
+            s0 = (s0 >> (16 * h0)) & 0xFFFFu;
+            s1 = (s1 >> (16 * h1)) & 0xFFFFu;
+          }
           // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
           // then (2, 3) of each word; activation registers in the same order.
           uint32_t ha0[4], la0[4], ha1[4], la1[4], hb0[4], lb0[4], hb1[4], lb1[4];
-          decode_word(lutlane, wa0, ha0, la0);
-          decode_word(lutlane, wa1, ha1, la1);
-          decode_word(lutlane, wb0, hb0, lb0);
-          decode_word(lutlane, wb1, hb1, lb1);
-          float ch[4], cl[4];
-          mma_f16_z(ch, ha0[0], ha1[0], ha0[1], ha1[1], xa.x, xa.y);
-          mma_f16(ch, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);
-          mma_f16(ch, hb0[0], hb1[0], hb0[1], hb1[1], xb.x, xb.y);
-          mma_f16(ch, hb0[2], hb1[2], hb0[3], hb1[3], xb.z, xb.w);
-          mma_f16_z(cl, la0[0], la1[0], la0[1], la1[1], xa.x, xa.y);
-          mma_f16(cl, la0[2], la1[2], la0[3], la1[3], xa.z, xa.w);
-          mma_f16(cl, lb0[0], lb1[0], lb0[1], lb1[1], xb.x, xb.y);
-          mma_f16(cl, lb0[2], lb1[2], lb0[3], lb1[3], xb.z, xb.w);
-          // block sum times absmax(row) and the activation rows' 2^-S
-          acc[uu][0] = fmaf(fmaf(cl[0], kLoInv, ch[0]), am0 * xs.x, acc[uu][0]);
-          acc[uu][1] = fmaf(fmaf(cl[1], kLoInv, ch[1]), am0 * xs.y, acc[uu][1]);
-          acc[uu][2] = fmaf(fmaf(cl[2], kLoInv, ch[2]), am1 * xs.x, acc[uu][2]);
-          acc[uu][3] = fmaf(fmaf(cl[3], kLoInv, ch[3]), am1 * xs.y, acc[uu][3]);
+          decode_word<PARTS>(lutlane, wa0, ha0, la0);
+          decode_word<PARTS>(lutlane, wa1, ha1, la1);
+          decode_word<PARTS>(lutlane, wb0, hb0, lb0);
+          decode_word<PARTS>(lutlane, wb1, hb1, lb1);
+          if (MX) {
+            // the two 32-element halves separately, each times its e8m0
+            // scale (byte 0 of the pair: first half, byte 1: second half)
+            float c0[4], c1[4];
+            mma_f16_z(c0, ha0[0], ha1[0], ha0[1], ha1[1], xa.x, xa.y);
+            mma_f16(c0, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);
+            mma_f16_z(c1, hb0[0], hb1[0], hb0[1], hb1[1], xb.x, xb.y);
+            mma_f16(c1, hb0[2], hb1[2], hb0[3], hb1[3], xb.z, xb.w);
+            const float e00 = e8m0_value(s0 & 0xFFu), e01 = e8m0_value(s0 >> 8);
+            const float e10 = e8m0_value(s1 & 0xFFu), e11 = e8m0_value(s1 >> 8);
+            acc[uu][0] = fmaf(fmaf(c1[0], e01, c0[0] * e00), xs.x, acc[uu][0]);
+            acc[uu][1] = fmaf(fmaf(c1[1], e01, c0[1] * e00), xs.y, acc[uu][1]);
+            acc[uu][2] = fmaf(fmaf(c1[2], e11, c0[2] * e10), xs.x, acc[uu][2]);
+            acc[uu][3] = fmaf(fmaf(c1[3], e11, c0[3] * e10), xs.y, acc[uu][3]);
+          } else {
+            float ch[4];
+            mma_f16_z(ch, ha0[0], ha1[0], ha0[1], ha1[1], xa.x, xa.y);
+            mma_f16(ch, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);
+            mma_f16(ch, hb0[0], hb1[0], hb0[1], hb1[1], xb.x, xb.y);
+            mma_f16(ch, hb0[2], hb1[2], hb0[3], hb1[3], xb.z, xb.w);
+            if (PARTS == 2) {
+              float cl[4];
+              mma_f16_z(cl, la0[0], la1[0], la0[1], la1[1], xa.x, xa.y);
+              mma_f16(cl, la0[2], la1[2], la0[3], la1[3], xa.z, xa.w);
+              mma_f16(cl, lb0[0], lb1[0], lb0[1], lb1[1], xb.x, xb.y);
+              mma_f16(cl, lb0[2], lb1[2], lb0[3], lb1[3], xb.z, xb.w);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) ch[i] = fmaf(cl[i], kLoInv, ch[i]);
+            }
+            // absmax of rows g and g + 8 (fp32, or bf16 widened exactly)
+            const float am0 = __uint_as_float(two_byte ? s0 << 16 : s0);
+            const float am1 = __uint_as_float(two_byte ? s1 << 16 : s1);
+            // block sum times absmax(row) and the activation rows' 2^-S
+            acc[uu][0] = fmaf(ch[0], am0 * xs.x, acc[uu][0]);
+            acc[uu][1] = fmaf(ch[1], am0 * xs.y, acc[uu][1]);
+            acc[uu][2] = fmaf(ch[2], am1 * xs.x, acc[uu][2]);
+            acc[uu][3] = fmaf(ch[3], am1 * xs.y, acc[uu][3]);
+          }
         }
       }
       __syncwarp();
-      mbar_arrive_elect(&empty[s]);
+      mbar_arrive_elect(&empty[st]);
     }
     if (act0) {
       if (blk != 0) {
         // hand the partial sums to the pair's block-0 warp
-        if (ep > 0 && !warp_wait_bar(&xempty[up], (ep - 1) & 1u, abort_flag, hdr)) return;
+        if (ep > 0 && !warp_wait_one(&xempty[up], (ep - 1) & 1u, abort_flag, hdr, limit_ns)) return;
 #pragma unroll
         for (int uu = 0; uu < 2; ++uu)
           *xchg_at(blk, uu) = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&xfull[up]);
       } else {
-        if (!warp_wait_bar(&xfull[up], ep & 1u, abort_flag, hdr)) return;
+        if (!warp_wait_one(&xfull[up], ep & 1u, abort_flag, hdr, limit_ns)) return;
 #pragma unroll
         for (int b = 1; b < 4; ++b) {
 #pragma unroll
@@ -651,30 +800,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&xempty[up]);
+        const int64_t b_first = cta_of(W, P, t * KC), b_last = cta_of(W, P, t * KC + KC - 1);
+        if (b_first == b_last) {
+          store_outputs(yout, alpha, limit, p, tl, up, g, q, acc, act1);
+        } else {
+          // a piece of a cut tile: leave the partial sums, count the piece;
+          // the piece that counts last adds all pieces in order and stores
+          float4 *mine = partials + (piece_slot(W, P, KC, t, blockIdx.x) * kPairs + up) * kPartialSlot;
 #pragma unroll
-        for (int uu = 0; uu < 2; ++uu) {
-          if (uu == 1 && !act1) break;
-          const int64_t j = t.j0 + 2 * up + uu;
+          for (int uu = 0; uu < 2; ++uu)
+            mine[uu * 32 + lane] = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
+          __syncwarp();
+          uint32_t old = 0;
+          uint32_t *cnt = counters + b_first * kPairs + up;
+          if (lane == 0) {
+            __threadfence();
+            old = atomic_add_acq_rel(cnt, 1u);
+          }
+          old = __shfl_sync(0xffffffffu, old, 0);
+          if (old == static_cast<uint32_t>(b_last - b_first)) {
+            __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int m = 2 * q + i;
-            if (m >= t.mrows) continue;
-            uint16_t *yr = y + (t.row0 + m) * ncols;
-            const float a0 = acc[uu][i], a1 = acc[uu][2 + i];
-            if (!swiglu) {
-              const int64_t c0 = 16 * j + g, c1 = 16 * j + 8 + g;
-              if (c0 < N) yr[c0] = bf16_bits(a0);
-              if (c1 < N) yr[c1] = bf16_bits(a1);
-            } else {
-              const int64_t c = 8 * j + g;
-              if (c < ncols) yr[c] = bf16_bits(silu(a0) * a1);
+            for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc[uu][i] = 0.0f;
+            for (int64_t c = b_first; c <= b_last; ++c) {
+              const float4 *pc = partials + (piece_slot(W, P, KC, t, c) * kPairs + up) * kPartialSlot;
+#pragma unroll
+              for (int uu = 0; uu < 2; ++uu) {
+                const float4 v = __ldcg(pc + uu * 32 + lane);
+                acc[uu][0] += v.x;
+                acc[uu][1] += v.y;
+                acc[uu][2] += v.z;
+                acc[uu][3] += v.w;
+              }
             }
+            store_outputs(yout, alpha, limit, p, tl, up, g, q, acc, act1);
+            if (lane == 0) *cnt = 0u;   // reusable by the next launch
           }
         }
       }
       ++ep;
     }
-    u += t.nunits;
+    s += k1 - k0;
   }
 }
 
@@ -682,17 +850,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t decode_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu) {
   (void)M; (void)N; (void)K; (void)G; (void)swiglu;
-  return kWsHeaderBytes;
+  const size_t P = static_cast<size_t>(device_sm_count());
+  const size_t counters = (P * kPairs * 4 + 255) / 256 * 256;
+  return kWsHeaderBytes + counters + P * 2 * kPairs * kPartialSlot * sizeof(float4);
 }
 
 size_t decode_zero_prefix_bytes(int64_t M, int32_t N, int32_t G, int32_t swiglu) {
   (void)M; (void)N; (void)G; (void)swiglu;
-  return kWsHeaderBytes;
+  const size_t P = static_cast<size_t>(device_sm_count());
+  return kWsHeaderBytes + (P * kPairs * 4 + 255) / 256 * 256;
 }
 
 cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (static_cast<int64_t>(a.E) * a.N + a.N + 256 >= INT_MAX) return cudaErrorNotSupported;
+  const bool mx = a.fmt == GNF4_FMT_MXFP4;
+  const int parts = (!mx && a.epi != GNF4_EPI_NONE) ? 2 : 1;
   WeightMaps wm;
+  std::memset(&wm, 0, sizeof(wm));
   // packed weights as [E*N rows][K/2 bytes], boxes of (8 << i) rows x 128 bytes
   for (int i = 0; i < kNumWMaps; ++i) {
     if (!encode_tensor_map_2d(&wm.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w,
@@ -702,10 +876,23 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
                               CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
+  if (a.epi == GNF4_EPI_SWIGLU_INTERLEAVED) {
+    // the same bytes as [E*N/2 pairs][2 parities][K/2]: boxes of one parity
+    for (int i = 0; i < kNumIMaps; ++i) {
+      const uint64_t dims[3] = {static_cast<uint64_t>(a.K / 2), 2,
+                                static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N) / 2};
+      const uint64_t pitches[2] = {static_cast<uint64_t>(a.K / 2), static_cast<uint64_t>(a.K)};
+      const uint32_t box[3] = {128, 1, 8u << i};
+      if (!encode_tensor_map(&wm.im[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.w, dims, pitches, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    }
+  }
   // activations viewed as [K/64 blocks][M rows][64 bf16]: one box = 4 blocks x
   // 8 rows x 64 elements, laid out in shared memory as 4 swizzled 1 KB tiles
   CUtensorMap xmap;
-  {
+  std::memset(&xmap, 0, sizeof(xmap));
+  if (a.hidden == nullptr) {
     const uint64_t dims[3] = {64, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K / 64)};
     const uint64_t pitches[2] = {static_cast<uint64_t>(a.K) * 2, 128};
     const uint32_t box[3] = {64, kBatch, kStageBlocks};
@@ -714,19 +901,44 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
 
-  static bool configured[64] = {false};
+  const int P = device_sm_count();
+  DecodeParams d;
+  d.scales = a.scales;
+  d.sizes = a.sizes;
+  d.expert_ids = a.expert_ids;
+  d.hidden = a.hidden;
+  d.sorted_idx = a.sorted_idx;
+  d.n_slots = a.n_tokens * a.top_k;
+  d.top_k = a.top_k;
+  d.G = a.G; d.M = a.M; d.N = a.N; d.K = a.K; d.E = a.E;
+  d.scale_kind = mx ? kScaleE8m0 : (a.scale_dtype == GNF4_SCALE_BF16 ? kScaleBf16 : kScaleF32);
+  d.epi = a.epi;
+  d.alpha = a.alpha;
+  d.limit = a.limit;
+  d.y = a.y;
+  d.hdr = static_cast<WsHeader *>(a.workspace);
+  char *ws = static_cast<char *>(a.workspace);
+  d.counters = reinterpret_cast<uint32_t *>(ws + kWsHeaderBytes);
+  d.partials = reinterpret_cast<float4 *>(ws + decode_zero_prefix_bytes(a.M, a.N, a.G, a.swiglu));
+
+  const bool bf = !mx && a.scale_dtype == GNF4_SCALE_BF16;
+  auto kernel = mx ? decode_gemm_kernel<1, kScaleE8m0>
+                   : (parts == 2 ? (bf ? decode_gemm_kernel<2, kScaleBf16>
+                                       : decode_gemm_kernel<2, kScaleF32>)
+                                 : (bf ? decode_gemm_kernel<1, kScaleBf16>
+                                       : decode_gemm_kernel<1, kScaleF32>));
+  const int ki = mx ? 4 : (parts - 1) * 2 + (bf ? 1 : 0);
+  static bool configured[64][5] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
-    cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (dev < 0 || dev >= 64 || !configured[dev][ki]) {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
     if (err != cudaSuccess) return err;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    if (dev >= 0 && dev < 64) configured[dev][ki] = true;
   }
-  return launch_pdl(decode_gemm_kernel, dim3(device_sm_count()), dim3(kThreads),
-                    static_cast<size_t>(kSmemBytes), stream, wm, xmap, a.absmax, a.sizes,
-                    a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.swiglu, a.y,
-                    static_cast<WsHeader *>(a.workspace));
+  return launch_pdl(kernel, dim3(P), dim3(kThreads), static_cast<size_t>(kSmemBytes), stream, wm,
+                    xmap, d);
 }
 
 }  // namespace gnf4

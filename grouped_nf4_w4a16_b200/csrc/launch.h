@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstddef>
+#include <cstring>
 #include <cstdint>
 #include <utility>
 #include <cuda_runtime.h>
@@ -12,9 +13,18 @@ namespace gnf4 {
 
 // Grouped GEMM problem as seen by the kernels (all pointers device memory).
 struct GemmArgs {
-  const uint16_t *x;        // bf16 [M][K]
+  const uint16_t *x;        // bf16 [M][K] (nullptr when the rows are gathered)
   const uint8_t *w;         // [E][N][K/2]
-  const float *absmax;      // [E][N][K/64]
+  const float *absmax;      // [E][N][K/64] fp32 (NF4 with fp32 absmax; else nullptr)
+  const void *scales;       // the block scales in their own encoding (== absmax for fp32)
+  int32_t fmt = GNF4_FMT_NF4;           // gnf4_format
+  int32_t scale_dtype = GNF4_SCALE_F32; // gnf4_scale_dtype
+  int32_t epi = GNF4_EPI_NONE;          // gnf4_epilogue
+  float alpha = 0.0f, limit = 0.0f;     // GNF4_EPI_SWIGLU_INTERLEAVED
+  const uint16_t *hidden = nullptr;     // gather: [n_tokens][K]; row i = hidden[sorted_idx[i] / top_k]
+  const int32_t *sorted_idx = nullptr;
+  int64_t n_tokens = 0;
+  int32_t top_k = 1;
   const int32_t *sizes;     // [G]
   const int32_t *expert_ids;// [G]
   int32_t G;
@@ -47,6 +57,9 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream);
 
 // ---- prefill-regime grouped GEMM (prefill_gemm.cu)
 size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32_t swiglu);
+// Whether the tensor-core kernel runs this combination of format, scales,
+// epilogue and gather.
+bool prefill_supports(const GemmArgs &a);
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream);
 
 // ---- router top-k and weighted combine (router.cu)
@@ -58,6 +71,8 @@ cudaError_t launch_moe_combine(const uint16_t *y, const int32_t *sorted_idx, con
                                cudaStream_t stream);
 
 // ---- grouped dgrad (dgrad.cu)
+size_t dgrad_workspace_bytes();
+size_t dgrad_zero_prefix_bytes();
 cudaError_t launch_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float *absmax,
                                  const int32_t *sizes, const int32_t *expert_ids, int32_t G,
                                  int64_t M, int32_t N, int32_t K, int32_t E, uint16_t *dx,
@@ -74,6 +89,8 @@ gnf4_status check_grouped_gemm(const uint16_t *x, const uint8_t *w, const float 
                                int32_t epilogue, int32_t mode, uint16_t *y, GemmArgs *out,
                                int32_t *use_out);
 gnf4_status launch_grouped_gemm(const GemmArgs &a, int32_t use, cudaStream_t s);
+// The same for gnf4_grouped_gemm_ex's descriptor.
+gnf4_status check_grouped_gemm_ex(const gnf4_gemm_desc *d, GemmArgs *out, int32_t *use_out);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

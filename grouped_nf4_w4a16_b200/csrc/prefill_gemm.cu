@@ -289,7 +289,7 @@ constexpr uint32_t kIdescF8 = (1u << 4) | (0u << 7) | (1u << 10) |
 struct TileInfo {
   int64_t row0;     // first activation row of the pair tile
   int32_t rows;     // valid activation rows (1..256)
-  int32_t n0;       // first weight row (within the expert) of the pair tile
+  int32_t n0;       // first output column of the pair tile (256 per tile; 128 with SwiGLU)
   int32_t e;        // expert
 };
 
@@ -297,7 +297,7 @@ struct TileInfo {
 // token tile i inner (pairs running at the same time share weight tiles).
 __device__ __forceinline__ TileInfo tile_info(int t, int G, const int *tile_start,
                                               const int *row_off, const int *gsize,
-                                              const int *gexp) {
+                                              const int *gexp, int ncols_tile) {
   int lo = 0, hi = G;   // tile_start[lo] <= t < tile_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -309,9 +309,70 @@ __device__ __forceinline__ TileInfo tile_info(int t, int G, const int *tile_star
   TileInfo ti;
   ti.row0 = static_cast<int64_t>(row_off[lo]) + static_cast<int64_t>(i) * kBN;
   ti.rows = min(kBN, gsize[lo] - i * kBN);
-  ti.n0 = j * kPairM;
+  ti.n0 = j * ncols_tile;
   ti.e = gexp[lo];
   return ti;
+}
+
+// Scale encodings (PrefillParams::scale_kind).
+constexpr int kScaleF32 = 0;    // NF4 absmax, fp32
+constexpr int kScaleBf16 = 1;   // NF4 absmax, bf16
+constexpr int kScaleE8m0 = 2;   // MXFP4: one e8m0 byte per 32 elements (a pair per K-step)
+
+struct PrefillParams {
+  const uint8_t *w;
+  const void *scales;           // fp32 / bf16 absmax [E][N][K/64] or e8m0 [E][N][K/32]
+  const float *tok_inv;         // 2^-s per activation row (written by the prep kernel)
+  const int32_t *sizes;
+  const int32_t *expert_ids;
+  const int32_t *sorted_idx;    // gather: every entry must lie in [0, n_slots) (checked)
+  int64_t n_slots;
+  int32_t G;
+  int64_t M;
+  int32_t N, K, E;
+  int32_t scale_kind;
+  int32_t epi;                  // 0 none, 1 SwiGLU on halves, 2 SwiGLU on interleaved rows
+  float alpha, limit;
+  uint16_t *y;
+  int32_t bulk_out;
+  WsHeader *hdr;
+};
+
+// Weight row (within the expert) of local row rl (0..127) of CTA `rank` in
+// a pair tile whose first output column is n0. Without SwiGLU rows are the
+// output columns. With SwiGLU a warp's 32 TMEM lanes hold 16 gate rows and
+// their 16 up rows: halves layout (epilogue 1): lanes 0-15 gate rows j..j+15,
+// lanes 16-31 up rows N/2 + j..; interleaved layout (epilogue 2): lane l row
+// 2 j + l (gate rows even, up rows odd), so the 128 rows are contiguous.
+// *col: the output column of the row's pair; *valid: the row exists.
+__device__ __forceinline__ int64_t weight_row(const PrefillParams &p, int n0, uint32_t rank,
+                                              int rl, bool *valid) {
+  if (p.epi == 0) {
+    const int64_t n = n0 + kBM * static_cast<int64_t>(rank) + rl;
+    *valid = n < p.N;
+    return n;
+  }
+  const int qq = rl >> 5, l = rl & 31;
+  if (p.epi == 1) {
+    const int64_t j = n0 + 64 * static_cast<int64_t>(rank) + 16 * qq + (l & 15);
+    *valid = j < p.N / 2;
+    return l < 16 ? j : p.N / 2 + j;
+  }
+  const int64_t j = n0 + 64 * static_cast<int64_t>(rank) + 16 * qq + (l >> 1);
+  *valid = j < p.N / 2;
+  return 2 * j + (l & 1);
+}
+
+// One scale value (block scale times nothing else) as fp32: element idx of
+// the stack's scale array; for e8m0 the larger of the pair at 2-byte element
+// idx (row maxima only need the larger).
+__device__ __forceinline__ float scale_max_at(const PrefillParams &p, int64_t idx) {
+  if (p.scale_kind == kScaleF32) return fabsf(__ldg(static_cast<const float *>(p.scales) + idx));
+  const uint32_t v = __ldg(static_cast<const unsigned short *>(p.scales) + idx);
+  if (p.scale_kind == kScaleBf16) return fabsf(__uint_as_float(v << 16));
+  const uint32_t m = max(v & 0xFFu, v >> 8);
+  return m == 255u ? __uint_as_float(0x7FC00000u)
+                   : (m == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(m << 23));
 }
 
 // Warp-uniform bounded wait with cluster-scope acquire: lane 0 waits, every
@@ -323,16 +384,36 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t *bar, uint32_t parity
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// SK: the scale encoding (kScaleE8m0 = MXFP4, one bf16 pass); SWIGLU: the
+// epilogue pairs gate and up rows (the halves or the interleaved layout,
+// chosen at run time).
+template <int SK, bool SWIGLU>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                         const __grid_constant__ CUtensorMap x8map,
                         const __grid_constant__ CUtensorMap wmap,
-                        const __grid_constant__ CUtensorMap ymap, const uint8_t *__restrict__ w,
-                        const float *__restrict__ absmax, const float *__restrict__ tok_inv,
-                        const int32_t *__restrict__ sizes,
-                        const int32_t *__restrict__ expert_ids, int32_t G, int64_t M, int32_t N,
-                        int32_t K, int32_t E, uint16_t *__restrict__ y, int32_t bulk_out,
-                        WsHeader *hdr) {
+                        const __grid_constant__ CUtensorMap w4map,
+                        const __grid_constant__ CUtensorMap ymap,
+                        const PrefillParams pin) {
+  // A local copy that the helpers take by reference: after inlining it lives
+  // in registers; the parameter block's own address is never taken (a use
+  // through such an address would be a memory load that every asm memory
+  // clobber forces to repeat).
+  constexpr bool MX = SK == kScaleE8m0;
+  PrefillParams p = pin;
+  p.scale_kind = SK;             // compile-time from here on
+  if (!SWIGLU) p.epi = 0;
+  const float *__restrict__ tok_inv = p.tok_inv;
+  const int32_t *__restrict__ sizes = p.sizes;
+  const int32_t *__restrict__ expert_ids = p.expert_ids;
+  const int32_t G = p.G, N = p.N, K = p.K, E = p.E;
+  const int64_t M = p.M;
+  uint16_t *__restrict__ y = p.y;
+  const int32_t bulk_out = p.bulk_out;
+  WsHeader *hdr = p.hdr;
+  // output columns per pair tile, and of y
+  const int ncols_tile = p.epi ? kPairM / 2 : kPairM;
+  const int64_t ncols = p.epi ? N / 2 : N;
   extern __shared__ char smem_raw[];
   char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) &
                                         ~static_cast<uintptr_t>(2047));
@@ -362,8 +443,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
 
   // ---- set-up: decode table, barriers, TMEM (no global memory yet)
-  for (int i = tid; i < 16 * 32; i += kThreads)
-    reinterpret_cast<float *>(smem + kLutOff)[i] = nf4_value(i >> 5);
+  for (int i = tid; i < 16 * 32; i += kThreads) {
+    const int c = i >> 5;
+    float v = nf4_value(c);
+    if (MX) {   // e2m1: sign, 2 exponent bits (bias 1), 1 mantissa bit
+      const int m = c & 7;
+      const float mag = m < 2 ? 0.5f * m : static_cast<float>(2 + (m & 1)) * exp2f(static_cast<float>((m >> 1) - 2));
+      v = (c & 8) ? -mag : mag;
+    }
+    reinterpret_cast<float *>(smem + kLutOff)[i] = v;
+  }
   if (tid == 0) {
     misc[0] = 0;
     misc[1] = 0;
@@ -385,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&xmap);
     prefetch_tensormap(&x8map);
-    prefetch_tensormap(&wmap);
+    prefetch_tensormap(p.epi == 1 ? &w4map : &wmap);
     if (bulk_out) prefetch_tensormap(&ymap);
   }
   if (warp == 2) {
@@ -400,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- group table (validated; both CTAs compute the same one)
   __shared__ int s_wsum[2][kThreads / 32];
-  const int NJ = (N + kPairM - 1) / kPairM;
+  const int NJ = static_cast<int>((ncols + ncols_tile - 1) / ncols_tile);
   const int per = (G + kThreads - 1) / kThreads;
   const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
   int my_rows = 0, my_tiles = 0, bad = 0;
@@ -443,6 +532,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) tile_start[G] = tot_t;
   }
   if (tid == 0 && static_cast<int64_t>(tot_r) != M) atomicOr(&misc[0], GNF4_DEVERR_SIZES);
+  if (p.sorted_idx != nullptr) {   // gathered rows: every slot in range before any work
+    int badslot = 0;
+    for (int64_t i = tid; i < M; i += kThreads) {
+      const int32_t sl = __ldg(p.sorted_idx + i);
+      if (sl < 0 || sl >= p.n_slots) badslot = 1;
+    }
+    if (__syncthreads_or(badslot) && tid == 0) atomicOr(&misc[0], GNF4_DEVERR_SLOT);
+  }
   // both CTAs: barriers initialised and TMEM allocated before any remote access
   tc_fence_before();
   cluster_sync();
@@ -458,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         uint32_t g = 0;   // stage ring counter
         for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
-          const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
+          const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp, ncols_tile);
           const int xrow = static_cast<int>(ti.row0) + kBNh * static_cast<int>(rank);
           bool ok = true;
           for (int kb = 0; kb < KB; ++kb, ++g) {
@@ -505,11 +602,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kBK / 16; ++kk)
               mma_pair_f16(tmem + kAccCol, a_hi + 8u * kk, sw128_desc(xaddr + kk * 32), kIdesc,
                            (kb > 0 || kk > 0) ? 1u : 0u);
-            // lo pass: e4m3 remainders x e5m2 activations, 2 x K=32
+            // lo pass: e4m3 remainders x e5m2 activations, 2 x K=32 (an MXFP4
+            // weight is exact in bf16: no remainder)
+            if (!MX) {
 #pragma unroll
-            for (int kk = 0; kk < kBK / 32; ++kk)
-              mma_pair_f8(tmem + kAccCol, a_lo + 8u * kk, sw64_desc(x8addr + kk * 32), kIdescF8,
-                          1u);
+              for (int kk = 0; kk < kBK / 32; ++kk)
+                mma_pair_f8(tmem + kAccCol, a_lo + 8u * kk, sw64_desc(x8addr + kk * 32), kIdescF8,
+                            1u);
+            }
             mma_commit_pair(&x_free[s], 0x3);
             mma_commit_pair(&a_free[sa], 0x3);
           }
@@ -529,31 +629,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t gq = 0;   // slot ring counter
       bool ok = true;
       for (int t = pair; t < tiles && ok && !*abort_flag; t += npairs) {
-        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
-        const int nbase = ti.n0 + kBM * static_cast<int>(rank);   // first row within the expert
-        const int64_t row0 = static_cast<int64_t>(ti.e) * N + nbase;
+        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp, ncols_tile);
+        const int64_t ebase = static_cast<int64_t>(ti.e) * N;
+        // this lane's 4 rows (rr = lane + 32 i): scale element of the row's
+        // first block, and whether the row exists
+        int64_t rb[4];
+        bool rv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          rb[i] = (ebase + weight_row(p, ti.n0, rank, lane + 32 * i, &rv[i])) * KB;
         for (int qd = 0; qd < nquads; ++qd, ++gq) {
           const int slot = static_cast<int>(gq % kWQuads);
           const uint32_t ph = (gq / kWQuads) & 1u;
           if (!warp_wait_cluster(&w_free[slot], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
-          char *as = smem + kAbsOff + slot * kASlotBytes;
+          const uint32_t as = smem_u32(smem + kAbsOff + slot * kASlotBytes) + lane * 4;
+          if (p.scale_kind == kScaleF32) {
+            const float *fb = static_cast<const float *>(p.scales) + 4 * qd;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int rr = lane + 32 * i;
-            const bool rv = nbase + rr < N;     // a row of this expert (else zeros)
+            for (int i = 0; i < 4; ++i) {
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-              const int kb = 4 * qd + blk;
-              const bool v = rv && kb < KB;
-              const float *src = v ? absmax + (row0 + rr) * KB + kb : absmax;
-              cp_async4(smem_u32(as + blk * (kBM * 4) + rr * 4), src, v ? 4u : 0u);
+              for (int blk = 0; blk < 4; ++blk) {
+                const bool v = rv[i] && 4 * qd + blk < KB;
+                cp_async4(as + blk * (kBM * 4) + i * 128, v ? fb + rb[i] + blk : p.scales,
+                          v ? 4u : 0u);
+              }
+            }
+          } else {   // the 4-byte word holding this (row, K-step)'s 2 bytes
+            const char *cb = static_cast<const char *>(p.scales);
+            const int64_t total = static_cast<int64_t>(E) * N * KB * 2;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int blk = 0; blk < 4; ++blk) {
+                const bool v = rv[i] && 4 * qd + blk < KB;
+                const int64_t wb = ((rb[i] + 4 * qd + blk) * 2) & ~int64_t{3};
+                cp_async4(as + blk * (kBM * 4) + i * 128, v ? cb + wb : p.scales,
+                          v ? (wb + 4 <= total ? 4u : 2u) : 0u);
+              }
             }
           }
           cp_async_arrive_noinc(&w_full[slot]);
           if (lane == 0) {
             mbar_arrive_expect_tx(&w_full[slot], kWSlotBytes);
-            tma_load_2d(smem + kWOff + slot * kWSlotBytes, &wmap, qd * 128,
-                        static_cast<int>(row0), &w_full[slot]);
+            char *wdst = smem + kWOff + slot * kWSlotBytes;
+            if (p.epi == 1) {   // per TMEM lane quarter: 16 gate rows, then their 16 up rows
+#pragma unroll
+              for (int qq = 0; qq < 4; ++qq)
+                tma_load_4d(wdst + qq * 4096, &w4map, qd * 128,
+                            ti.n0 + 64 * static_cast<int>(rank) + 16 * qq, 0, ti.e, &w_full[slot]);
+            } else {            // 128 consecutive rows
+              bool unused;
+              const int64_t row0 = ebase + weight_row(p, ti.n0, rank, 0, &unused);
+              tma_load_2d(wdst, &wmap, qd * 128, static_cast<int>(row0), &w_full[slot]);
+            }
           }
         }
       }
@@ -570,44 +698,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int quarter = warp & 3;          // TMEM lane quarter
       const int half = dw >> 2;              // K half of the stage / token half of the tile
       const int rl = quarter * 32 + lane;                      // row within this CTA's half
-      const int r = kBM * static_cast<int>(rank) + rl;         // row within the pair tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       // shared address of this lane's table slot (bits 7..10 clear): the
       // entry of code c is at lut_lane | c * 128
       const uint32_t lut_lane = smem_u32(smem + kLutOff) + static_cast<uint32_t>(lane) * 4u;
       // absmax row of this thread's weight row in pair tile t (nullptr: no such row)
-      auto row_absmax = [&](int t) -> const float * {
-        if (t >= tiles) return nullptr;
-        const TileInfo tn = tile_info(t, G, tile_start, row_off, gsize, gexp);
-        const int nn = tn.n0 + r;
-        return nn < N ? absmax + (static_cast<int64_t>(tn.e) * N + nn) * KB : nullptr;
+      // scale-array element index of this thread's weight row in pair tile t
+      // (its first block; -1: no such row)
+      auto row_scales = [&](int t) -> int64_t {
+        if (t >= tiles) return -1;
+        const TileInfo tn = tile_info(t, G, tile_start, row_off, gsize, gexp, ncols_tile);
+        bool v;
+        const int64_t nn = weight_row(p, tn.n0, rank, rl, &v);
+        return v ? (static_cast<int64_t>(tn.e) * N + nn) * KB : -1;
       };
-      // Row maximum of absmax for the row scale: for the first tile read here,
-      // for every later tile gathered one block per K-step of the tile before.
+      // Row maximum of the block scales for the row scale: for the first
+      // tile read here, for every later tile gathered one block per K-step of
+      // the tile before.
       float mx = 0.0f;
-      if (const float *a0 = row_absmax(pair)) {
-        float m[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-        int b = 0;
-        for (; b + 8 <= KB; b += 8) {   // 8 independent loads in flight
+      {
+        const int64_t a0 = row_scales(pair);
+        if (a0 >= 0) {
+          float m[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+          int b = 0;
+          for (; b + 8 <= KB; b += 8) {   // 8 independent loads in flight
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(__ldg(a0 + b + i)));
+            for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], scale_max_at(p, a0 + b + i));
+          }
+          for (; b < KB; ++b) m[0] = fmaxf(m[0], scale_max_at(p, a0 + b));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx = fmaxf(mx, m[i]);
         }
-        for (; b < KB; ++b) m[0] = fmaxf(m[0], fabsf(__ldg(a0 + b)));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, m[i]);
       }
       uint32_t g = 0;    // decoded-weight stage counter
       uint32_t gq = 0;   // packed-weight slot counter
       uint32_t ntile = 0;
       for (int t = pair; t < tiles && !*abort_flag; t += npairs, ++ntile) {
-        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp);
-        const float *ap_next = row_absmax(t + npairs);
+        const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp, ncols_tile);
+        const int64_t ap_next = row_scales(t + npairs);
         float mx_next = 0.0f;
-        float nxq[4];   // next tile's absmax values, folded 4 K-steps after their load
+        float nxq[4];   // next tile's block scales, folded 4 K-steps after their load
 #pragma unroll
         for (int j = 0; j < 4; ++j) nxq[j] = 0.0f;
-        const int n = ti.n0 + r;
-        const bool rok = n < N;
+        bool rok;
+        const int64_t n = weight_row(p, ti.n0, rank, rl, &rok);
+        // scale-array element index of this row's blocks (for the 2-byte
+        // encodings: which half of each copied word holds them)
+        const int64_t sbase = (static_cast<int64_t>(ti.e) * N + n) * KB;
         // Row scale 2^S, S = beta + 14 with 2^beta * max(absmax of the row) in
         // [1, 2): scaled weights stay below 2^15 and their bf16 remainders
         // below 64, inside the e4m3 range, whatever the row's magnitude.
@@ -634,10 +771,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kb >= KB) break;
             const uint4 pk =
                 *reinterpret_cast<const uint4 *>(wsm + (((2 * sub + half) ^ (rl & 7)) << 4));
-            const float am = asm4[sub * kBM] * rscale;
-            // next tile's absmax, first used 4 K-steps after its load (no wait here)
-            mx_next = fmaxf(mx_next, fabsf(nxq[sub]));
-            nxq[sub] = ap_next != nullptr ? __ldg(ap_next + kb) : 0.0f;
+            float am;
+            if (p.scale_kind == kScaleF32) {
+              am = asm4[sub * kBM];
+            } else {
+              const uint32_t wv = __float_as_uint(asm4[sub * kBM]);
+              const uint32_t v16 = (wv >> (16 * static_cast<uint32_t>((sbase + kb) & 1))) & 0xFFFFu;
+              if (MX) {   // e8m0 of this warp's 32-element half of the K-step
+                const uint32_t e = half ? (v16 >> 8) : (v16 & 0xFFu);
+                am = e == 255u ? __uint_as_float(0x7FC00000u)
+                               : (e == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23));
+              } else {
+                am = __uint_as_float(v16 << 16);
+              }
+            }
+            am *= rscale;
+            // next tile's block scales, first used 4 K-steps after their load (no wait here)
+            mx_next = fmaxf(mx_next, nxq[sub]);
+            nxq[sub] = ap_next >= 0 ? scale_max_at(p, ap_next + kb) : 0.0f;
             const int s = g % kAStages;
             const uint32_t ph = (g / kAStages) & 1u;
             // hi[i]: bf16 pair of k = 32 half + 2i, 2i+1; lo[i]: e4m3 of k = 32 half + 4i .. +3
@@ -646,34 +797,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
-              for (int p = 0; p < 4; ++p) {
-                // codes of byte p: high nibble = even k, low nibble = odd k;
-                // each moved straight to bits 7..10 of its table address
+              for (int pb = 0; pb < 4; ++pb) {
+                // codes of byte pb (NF4: high nibble = even k; MXFP4: low
+                // nibble = even k), each moved straight to bits 7..10 of its
+                // table address
                 const uint32_t w = words[q];
-                const uint32_t s0 = p == 0 ? (w << 3) : (w >> (8 * p - 3));
-                const uint32_t s1 = p == 0 ? (w << 7) : (w >> (8 * p - 7));
+                const uint32_t sh = pb == 0 ? (w << 3) : (w >> (8 * pb - 3));   // high nibble
+                const uint32_t sl = pb == 0 ? (w << 7) : (w >> (8 * pb - 7));   // low nibble
+                const uint32_t s0 = MX ? sl : sh, s1 = MX ? sh : sl;
                 float v0, v1;
                 asm("ld.shared.f32 %0, [%1];" : "=f"(v0) : "r"(lut_lane | (s0 & 0x780u)));
                 asm("ld.shared.f32 %0, [%1];" : "=f"(v1) : "r"(lut_lane | (s1 & 0x780u)));
                 const float w0 = __fmul_rn(v0, am), w1 = __fmul_rn(v1, am);
                 const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
                 const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
-                const float h0 = __uint_as_float(hb << 16), h1 = __uint_as_float(hb & 0xFFFF0000u);
-                // remainders (exact in fp32, below 64 in magnitude) to e4m3, RNE
-                const uint32_t l8 = __nv_cvt_float2_to_fp8x2(make_float2(w0 - h0, w1 - h1),
-                                                             __NV_SATFINITE, __NV_E4M3);
-                hi[q * 4 + p] = hb;
-                if (p & 1)
-                  lo[q * 2 + (p >> 1)] = __byte_perm(lo_even, l8, 0x5410u);
-                else
-                  lo_even = l8;
+                hi[q * 4 + pb] = hb;
+                if (!MX) {
+                  const float h0 = __uint_as_float(hb << 16), h1 = __uint_as_float(hb & 0xFFFF0000u);
+                  // remainders (exact in fp32, below 64 in magnitude) to e4m3, RNE
+                  const uint32_t l8 = __nv_cvt_float2_to_fp8x2(make_float2(w0 - h0, w1 - h1),
+                                                               __NV_SATFINITE, __NV_E4M3);
+                  if (pb & 1)
+                    lo[q * 2 + (pb >> 1)] = __byte_perm(lo_even, l8, 0x5410u);
+                  else
+                    lo_even = l8;
+                }
               }
             }
             if (!warp_wait_cluster(&a_free[s], ph ^ 1u, abort_flag, hdr)) { ok = false; break; }
             tc_fence_after();
             const uint32_t col = kACol + kAStageCols * s;
             tmem_st16(tmem + lane_base + col + 16u * half, hi);
-            tmem_st8(tmem + lane_base + col + 32u + 8u * half, lo);
+            if (!MX) tmem_st8(tmem + lane_base + col + 32u + 8u * half, lo);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -686,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, fabsf(nxq[j]));
+        for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, nxq[j]);
         mx = mx_next;
         // ---- epilogue: accumulator -> bf16 y (this CTA's 128 weight rows).
         // Chunks of 32 tokens: scaled and rounded into a shared-memory box
@@ -710,6 +865,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // lane c holds 2^-s of activation row c0 + c of the tile
           const float tinv = c0 + lane < ti.rows ? __ldg(tok_inv + ti.row0 + c0 + lane) : 0.0f;
+          if (p.epi != 0) {
+            // SwiGLU: the gate lane of each row pair takes its up value from
+            // the partner lane and writes one output column of 32 tokens
+            const bool halves = p.epi == 1;
+            const int partner = halves ? (lane ^ 16) : (lane ^ 1);
+            const bool gate_lane = halves ? lane < 16 : (lane & 1) == 0;
+            const int jl = halves ? (lane & 15) : (lane >> 1);
+            const int64_t jbox = static_cast<int64_t>(ti.n0) + 64 * static_cast<int64_t>(rank) +
+                                 16 * quarter;   // first output column of this warp
+            const bool use_box = bulk_out && c0 + 32 <= ti.rows;
+            if (use_box && jbox >= ncols) continue;   // none of this warp's columns exists
+            uint16_t *box = reinterpret_cast<uint16_t *>(smem + kOutOff) + dw * 1024;
+            if (use_box) {
+              if (lane == 0) bulk_wait_read_0();   // the previous chunk's store has read the box
+              __syncwarp();
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float tc = __shfl_sync(0xffffffffu, tinv, c);
+              const float v = __uint_as_float(acc[c]) * rinv * tc;
+              const float u = __shfl_sync(0xffffffffu, v, partner);
+              if (gate_lane) {
+                float o;
+                if (halves) {
+                  o = v / (1.0f + expf(-v)) * u;
+                } else {
+                  const float gt = fminf(v, p.limit);
+                  const float uc = fminf(fmaxf(u, -p.limit), p.limit);
+                  o = gt / (1.0f + expf(-p.alpha * gt)) * (uc + 1.0f);
+                }
+                const __nv_bfloat16 b = __float2bfloat16_rn(o);
+                const uint16_t bits = *reinterpret_cast<const uint16_t *>(&b);
+                if (use_box) {
+                  box[c * 16 + jl] = bits;
+                } else if (rok && c0 + c < ti.rows) {
+                  y[(ti.row0 + c0 + c) * ncols + jbox + jl] = bits;
+                }
+              }
+            }
+            if (use_box) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&ymap, box, static_cast<int>(jbox), static_cast<int>(ti.row0) + c0);
+                bulk_commit();
+              }
+            }
+            continue;
+          }
           if (bulk_out && c0 + 32 <= ti.rows) {
             if (nbox >= N) continue;   // none of this warp's rows exists (nor does its box)
             uint16_t *box = reinterpret_cast<uint16_t *>(smem + kOutOff) + dw * 1024;
@@ -794,10 +998,14 @@ __device__ __forceinline__ void scale_chunk(const uint4 v, float f, uint4 *dst, 
   *dst8 = make_uint2(o8[0] | (o8[1] << 16), o8[2] | (o8[3] << 16));
 }
 
+// With a gather (hidden != nullptr) row m of x is hidden[sorted_idx[m] /
+// top_k]; a slot outside [0, n_slots) reads as a row of zeros (the GEMM
+// kernel refuses the call on such a slot and writes nothing).
 __global__ void __launch_bounds__(kPrepThreads)
-    prefill_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
-                        uint8_t *__restrict__ x8, float *__restrict__ tok_inv, int64_t M,
-                        int32_t K) {
+    prefill_prep_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ hidden,
+                        const int32_t *__restrict__ sorted_idx, int32_t top_k, int64_t n_slots,
+                        uint16_t *__restrict__ xs, uint8_t *__restrict__ x8,
+                        float *__restrict__ tok_inv, int64_t M, int32_t K) {
   __shared__ float s_max[kPrepThreads / 32];
   pdl_trigger();
   pdl_wait();
@@ -805,21 +1013,29 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int c8 = K / 8;   // 8-element chunks per row
   const bool in_regs = c8 <= kPrepThreads * kPrepChunks;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
+    const uint16_t *row = x + m * K;
+    bool zero_row = false;
+    if (hidden != nullptr) {
+      const int32_t sl = __ldg(sorted_idx + m);
+      zero_row = sl < 0 || sl >= n_slots;
+      row = hidden + static_cast<int64_t>(zero_row ? 0 : sl / top_k) * K;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(row);
     uint4 v[kPrepChunks];
     float mx = 0.0f;
+    const int c8r = zero_row ? 0 : c8;   // chunks read from memory (a zero row reads none)
     if (in_regs) {
 #pragma unroll
       for (int u = 0; u < kPrepChunks; ++u) {
         const int i = tid + u * kPrepThreads;
-        v[u] = i < c8 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        v[u] = i < c8r ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < kPrepChunks; ++u)
         mx = fmaxf(mx, fmaxf(fmaxf(bf16_abs_max2(v[u].x), bf16_abs_max2(v[u].y)),
                              fmaxf(bf16_abs_max2(v[u].z), bf16_abs_max2(v[u].w))));
     } else {
-      for (int i = tid; i < c8; i += kPrepThreads) {
+      for (int i = tid; i < c8r; i += kPrepThreads) {
         const uint4 a = __ldg(src + i);
         mx = fmaxf(mx, fmaxf(fmaxf(bf16_abs_max2(a.x), bf16_abs_max2(a.y)),
                              fmaxf(bf16_abs_max2(a.z), bf16_abs_max2(a.w))));
@@ -850,7 +1066,8 @@ __global__ void __launch_bounds__(kPrepThreads)
         if (i < c8) scale_chunk(v[u], f, dst + i, dst8 + i);
       }
     } else {
-      for (int i = tid; i < c8; i += kPrepThreads) scale_chunk(__ldg(src + i), f, dst + i, dst8 + i);
+      for (int i = tid; i < c8; i += kPrepThreads)
+        scale_chunk(i < c8r ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u), f, dst + i, dst8 + i);
     }
   }
 }
@@ -870,10 +1087,19 @@ size_t prefill_workspace_bytes(int64_t M, int32_t N, int32_t K, int32_t G, int32
   return kWsHeaderBytes + 3 * x8_bytes(M, K) + tok_bytes(M);
 }
 
+bool prefill_supports(const GemmArgs &a) {
+  const bool nf4 = a.fmt == GNF4_FMT_NF4 &&
+                   (a.scale_dtype == GNF4_SCALE_F32 || a.scale_dtype == GNF4_SCALE_BF16);
+  const bool mx = a.fmt == GNF4_FMT_MXFP4 && a.scale_dtype == GNF4_SCALE_E8M0;
+  return nf4 || mx;
+}
+
 cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
-  if (a.swiglu) return cudaErrorNotSupported;   // fused SwiGLU is decode-only for now
+  if (!prefill_supports(a)) return cudaErrorNotSupported;
   if (a.ws_bytes < prefill_workspace_bytes(a.M, a.N, a.K, a.G, a.swiglu)) return cudaErrorInvalidValue;
-  CUtensorMap xmap, x8map, wmap, ymap;
+  const bool mx = a.fmt == GNF4_FMT_MXFP4;
+  CUtensorMap xmap, x8map, wmap, w4map, ymap;
+  std::memset(&w4map, 0, sizeof(w4map));
   // the row-scaled operands live in the workspace after the header
   uint8_t *x8 = static_cast<uint8_t *>(a.workspace) + kWsHeaderBytes;
   uint16_t *xs = reinterpret_cast<uint16_t *>(x8 + x8_bytes(a.M, a.K));
@@ -889,15 +1115,17 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
                             static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kBK, kBNh,
                             CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  // output as [M rows][N bf16], boxes of 32 rows x 32 elements, for the
-  // epilogue's bulk stores; they need rows of a multiple of 16 bytes
-  // (otherwise every output is stored element by element and the map is a
-  // placeholder the kernel does not touch)
-  const int32_t bulk_out = a.N % 8 == 0 ? 1 : 0;
+  // output as [M rows][ncols bf16], boxes of 32 rows x 32 elements (16 with
+  // SwiGLU), for the epilogue's bulk stores; they need rows of a multiple of
+  // 16 bytes (otherwise every output is stored element by element and the map
+  // is a placeholder the kernel does not touch)
+  const int64_t ncols = a.swiglu ? a.N / 2 : a.N;
+  const int32_t bulk_out = ncols % 8 == 0 ? 1 : 0;
   if (bulk_out) {
     if (!encode_tensor_map_2d(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y,
-                              static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
-                              static_cast<uint64_t>(a.N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+                              static_cast<uint64_t>(ncols), static_cast<uint64_t>(a.M),
+                              static_cast<uint64_t>(ncols) * 2, a.swiglu ? 16 : 32, 32,
+                              CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   // packed weights as [E*N rows][K/2 bytes], boxes of 128 rows x 128 bytes
@@ -907,23 +1135,62 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
                             static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N),
                             static_cast<uint64_t>(a.K) / 2, 128, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  if (a.epi == GNF4_EPI_SWIGLU) {
+    // the same bytes as [E][2 halves][N/2 rows][K/2]: a box holds 16 rows of
+    // the gate half, then the 16 matching rows of the up half
+    const uint64_t kh = static_cast<uint64_t>(a.K) / 2, nh = static_cast<uint64_t>(a.N) / 2;
+    const uint64_t dims[4] = {kh, nh, 2, static_cast<uint64_t>(a.E)};
+    const uint64_t pitches[3] = {kh, nh * kh, 2 * nh * kh};
+    const uint32_t box[4] = {128, 16, 2, 1};
+    if (!encode_tensor_map(&w4map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, a.w, dims, pitches, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   if (!bulk_out) ymap = wmap;
+  if (a.epi != GNF4_EPI_SWIGLU) w4map = wmap;
 
-  static bool configured[64] = {false};
+  const int sk = mx ? kScaleE8m0 : (a.scale_dtype == GNF4_SCALE_BF16 ? kScaleBf16 : kScaleF32);
+  using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                            PrefillParams);
+  static const KernelFn kernels[3][2] = {
+      {prefill_gemm_kernel<kScaleF32, false>, prefill_gemm_kernel<kScaleF32, true>},
+      {prefill_gemm_kernel<kScaleBf16, false>, prefill_gemm_kernel<kScaleBf16, true>},
+      {prefill_gemm_kernel<kScaleE8m0, false>, prefill_gemm_kernel<kScaleE8m0, true>}};
+  const int ks = a.swiglu ? 1 : 0;
+  const KernelFn kernel = kernels[sk][ks];
+  static bool configured[64][3][2] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
-    cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (dev < 0 || dev >= 64 || !configured[dev][sk][ks]) {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
     if (err != cudaSuccess) return err;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    if (dev >= 0 && dev < 64) configured[dev][sk][ks] = true;
   }
   // one block per activation row (rows strided over the grid)
   const int64_t want = a.M;   // 4 blocks of 256 threads fit an SM at 64 registers
   const int xblocks = static_cast<int>(want < 4 * device_sm_count() ? want : 4 * device_sm_count());
   cudaError_t err = launch_pdl(prefill_prep_kernel, dim3(xblocks), dim3(kPrepThreads), 0, stream,
-                               static_cast<const uint16_t *>(a.x), xs, x8, tok_inv, a.M, a.K);
+                               static_cast<const uint16_t *>(a.x), a.hidden, a.sorted_idx,
+                               a.top_k, a.n_tokens * a.top_k, xs, x8, tok_inv, a.M, a.K);
   if (err != cudaSuccess) return err;
+
+  PrefillParams pp;
+  pp.w = a.w;
+  pp.scales = a.scales;
+  pp.tok_inv = tok_inv;
+  pp.sizes = a.sizes;
+  pp.expert_ids = a.expert_ids;
+  pp.sorted_idx = a.hidden != nullptr ? a.sorted_idx : nullptr;
+  pp.n_slots = a.n_tokens * a.top_k;
+  pp.G = a.G; pp.M = a.M; pp.N = a.N; pp.K = a.K; pp.E = a.E;
+  pp.scale_kind = mx ? kScaleE8m0 : (a.scale_dtype == GNF4_SCALE_BF16 ? kScaleBf16 : kScaleF32);
+  pp.epi = a.epi;
+  pp.alpha = a.alpha;
+  pp.limit = a.limit;
+  pp.y = a.y;
+  pp.bulk_out = bulk_out;
+  pp.hdr = static_cast<WsHeader *>(a.workspace);
 
   // one CTA per SM, in pairs (clusters of 2) for the 2-SM MMA
   const int grid = device_sm_count() & ~1;
@@ -941,10 +1208,7 @@ cudaError_t launch_prefill_gemm(const GemmArgs &a, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, xmap, x8map, wmap, ymap, a.w, a.absmax, tok_inv,
-                            a.sizes,
-                            a.expert_ids, a.G, a.M, a.N, a.K, a.E, a.y, bulk_out,
-                            static_cast<WsHeader *>(a.workspace));
+  return cudaLaunchKernelEx(&cfg, kernel, xmap, x8map, wmap, w4map, ymap, pp);
 }
 
 }  // namespace gnf4

@@ -56,6 +56,24 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   }
 }
 
+// As wait_bar, with the time limit given (a kernel may shorten it on request).
+__device__ __forceinline__ bool wait_bar_lim(uint64_t *bar, uint32_t parity,
+                                             volatile int *abort_flag, WsHeader *hdr,
+                                             uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  const uint32_t hint = limit_ns < kWaitHintNs ? static_cast<uint32_t>(limit_ns) : kWaitHintNs;
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (*abort_flag) return false;
+    if (global_timer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform bounded wait: lane 0 waits, every lane gets the same answer,
 // so warp-collective instructions after it are never reached by part of a warp.
 __device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity,
@@ -97,6 +115,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
       : "memory");
 }
 
+// 4-D tiled tensor copy (c0 innermost; same alignment rule).
+__device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, int c3, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 4-byte asynchronous copy global -> shared (src_bytes 0: writes zeros, reads nothing).
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
@@ -119,7 +148,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 }
 
 // ------------------------------------------------------------ host side
-// Encodes a tiled tensor map of rank 2 or 3: dims[0] is the contiguous
+// Encodes a tiled tensor map of rank 2 to 5: dims[0] is the contiguous
 // dimension, pitches[i] the byte stride of dims[i + 1]. Returns false if the
 // driver refuses it.
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,

@@ -24,9 +24,9 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, co
                        const uint64_t *dims, const uint64_t *pitches, const uint32_t *box,
                        CUtensorMapSwizzle swizzle) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
-  if (encode == nullptr || rank < 2 || rank > 3) return false;
-  cuuint64_t d[3], st[2];
-  cuuint32_t b[3], es[3];
+  if (encode == nullptr || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
   for (int i = 0; i < rank; ++i) {
     d[i] = static_cast<cuuint64_t>(dims[i]);
     b[i] = static_cast<cuuint32_t>(box[i]);

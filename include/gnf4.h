@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GNF4_VERSION 110 /* 1.1.0: + gnf4_router_topk, gnf4_moe_combine, gnf4_grouped_dgrad */
+#define GNF4_VERSION 120 /* 1.2.0: + gnf4_grouped_gemm_ex (MXFP4, bf16 absmax, gather, gpt-oss SwiGLU) */
 
 /* Exported entry points (the library is built with hidden default visibility). */
 #if defined(__GNUC__)
@@ -73,7 +73,21 @@ typedef enum {
                                          gnf4_grouped_gemm_noalloc */
 } gnf4_status;
 
-typedef enum { GNF4_EPI_NONE = 0, GNF4_EPI_SWIGLU = 1 } gnf4_epilogue;
+typedef enum {
+    GNF4_EPI_NONE = 0,
+    GNF4_EPI_SWIGLU = 1,              /* silu(gate) * up, gate = columns [0, N/2), up = [N/2, N) */
+    GNF4_EPI_SWIGLU_INTERLEAVED = 2   /* gate = even columns, up = odd columns, clamped; see
+                                         gnf4_grouped_gemm_ex */
+} gnf4_epilogue;
+typedef enum {
+    GNF4_FMT_NF4 = 0,                 /* NF4 codes (bitsandbytes layout) + absmax per 64 */
+    GNF4_FMT_MXFP4 = 1                /* e2m1 codes + e8m0 scale per 32 (OCP microscaling) */
+} gnf4_format;
+typedef enum {
+    GNF4_SCALE_F32 = 0,               /* NF4 absmax as fp32 */
+    GNF4_SCALE_BF16 = 1,              /* NF4 absmax as bf16 */
+    GNF4_SCALE_E8M0 = 2               /* MXFP4 scales: one byte 2^(s-127) per 32 elements */
+} gnf4_scale_dtype;
 typedef enum { GNF4_MODE_AUTO = 0, GNF4_MODE_DECODE = 1, GNF4_MODE_PREFILL = 2 } gnf4_mode;
 typedef enum { GNF4_OUT_F32 = 0, GNF4_OUT_BF16 = 1 } gnf4_out_dtype;
 typedef enum {
@@ -155,29 +169,40 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *   blocksize   must be 64
  *   epilogue    gnf4_epilogue
  *   mode        gnf4_mode: AUTO picks DECODE when the mean rows per possible
- *               group, M / min(G, E), is at most 64 or when SwiGLU is fused,
- *               else PREFILL. Both modes accept any group sizes; the mode only
- *               selects the kernel. PREFILL with SWIGLU is refused with
- *               GNF4_ERR_UNSUPPORTED_SHAPE (the tensor-core kernel has no
- *               fused SwiGLU).
+ *               group, M / min(G, E), is at most 64, else PREFILL. Both modes
+ *               accept any group sizes and both epilogues; the mode only
+ *               selects the kernel.
  *   y           device bf16 [M][N] or [M][N/2]; fully overwritten; must not
  *               overlap x, w, absmax or the workspace.
  *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G)
  *               bytes (which covers every mode; the call itself only checks
  *               the need of the kernel it runs and refuses less with
  *               GNF4_ERR_WORKSPACE_TOO_SMALL). Its first 256 bytes are the
- *               device status word: zero it once before the first use. The
- *               DECODE kernel needs nothing more; PREFILL also writes, after
- *               the header, the row-scaled operands of x: an e5m2 copy (M*K
- *               bytes, rounded up to 256), a bf16 copy (twice that) and one
- *               fp32 factor per row (M*4 bytes, rounded up to 256).
- *               Two calls that may run concurrently need separate workspaces.
+ *               device status header: zero the whole workspace once before
+ *               the first use. Word 2 of the header (bytes 8..11), when not
+ *               zero, shortens every bounded wait of the DECODE kernel to
+ *               that many nanoseconds (a test hook; 0 = the 2 s default).
+ *               DECODE then uses, after the header, one counter per
+ *               (SM, unit pair) (zero between calls: each call leaves them
+ *               at zero) and the fp32 partial sums of the tiles its stream-K
+ *               split cuts (8 KB per SM). PREFILL writes, after the header,
+ *               the row-scaled operands of x: an e5m2 copy (M*K bytes,
+ *               rounded up to 256), a bf16 copy (twice that) and one fp32
+ *               factor per row (M*4 bytes, rounded up to 256). After a call
+ *               that ran out of time (GNF4_ERR_TIMEOUT) zero the workspace
+ *               again before reusing it. Two calls that may run
+ *               concurrently need separate workspaces.
  * Numerics: every product enters an fp32 accumulator. DECODE carries each
- *   code value as an fp16 part plus an fp16 remainder (scaled by 2^13),
- *   together within 1e-7 relative of the fp32 table value, and
- *   x per row and 64-element block scaled by a power of two into fp16 (exact
- *   for every element above 2^-28 of that block's largest magnitude); each
- *   block sum is scaled by absmax and the power of two in fp32.
+ *   code value as its fp16 rounding (relative error at most 2^-12; the
+ *   elementwise tolerance above holds with margin on the shapes in scope)
+ *   and, with a fused SwiGLU (which multiplies a gate error by the up
+ *   value), also the fp16 of the remainder (scaled by 2^13), together
+ *   within 1e-7 relative of the fp32 table value; x per row and 64-element
+ *   block is scaled by a power of two into fp16 (exact for every element
+ *   above 2^-28 of that block's largest magnitude); each block sum is
+ *   scaled by absmax and the power of two in fp32. DECODE's stream-K split
+ *   adds the fp32 partial sums of a cut tile in a fixed order: results are
+ *   deterministic for a given GPU (SM count).
  *   PREFILL scales each weight row and each row of x by a power of two,
  *   multiplies the bf16 rounding of the fp32 weight NF4[code] * absmax by the
  *   scaled x (exact in bf16), adds the e4m3 rounding of what that rounding
@@ -192,6 +217,81 @@ GNF4_API gnf4_status gnf4_grouped_gemm(const uint16_t *x, const uint8_t *w, cons
                               int64_t M, int32_t N, int32_t K, int32_t E, int32_t blocksize,
                               int32_t epilogue, int32_t mode, uint16_t *y, void *workspace,
                               size_t ws_bytes, gnf4_stream_t stream);
+
+/*
+ * gnf4_grouped_gemm_ex -- the grouped GEMM with its options in a descriptor:
+ * the weight format (NF4 or native MXFP4), the scale encoding, the epilogue
+ * (none, SwiGLU on halves, SwiGLU on interleaved clamped rows) and the
+ * activation gather through the sort's permutation.
+ *
+ * Passages: README opening section (the operation); package page
+ * "grouped-nf4-gemm", "Direct answer" and header block ("Owns": the grouped
+ * packed GEMM over NF4 and native MXFP4, e2m1 + e8m0, computed on the
+ * released bytes with no requantisation and no bf16 copy); "Use this when"
+ * (the small launches around the expert GEMM, the token gather among them,
+ * folded into one); the streaming page's bake options (absmax stored as fp32
+ * or bf16).
+ *
+ * For every row m of group g (expert e) and output column n:
+ *   NF4:   acc = sum_k x[m][k] * NF4[code(e,n,k)] * absmax[e][n][k/64]
+ *          (absmax fp32, or bf16 widened exactly to fp32)
+ *   MXFP4: acc = sum_k x[m][k] * E2M1[code(e,n,k)] * 2^(scale[e][n][k/32]-127)
+ *          code(e,n,k) = low nibble of w[e][n][k/2] for even k, high for odd
+ *          k (the OCP microscaling FP4 packing of the released gpt-oss
+ *          blocks); E2M1 = 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives;
+ *          scale 255 is NaN.
+ *   epilogue NONE / SWIGLU: as gnf4_grouped_gemm.
+ *   epilogue SWIGLU_INTERLEAVED (the gpt-oss form): gate = acc of even
+ *          column 2j, up = acc of odd column 2j+1; g = min(gate, limit),
+ *          u = min(max(up, -limit), limit);
+ *          y[m][j] = bf16_rne(g * sigmoid(alpha * g) * (u + 1)), y is [M][N/2].
+ *   gather: with x == NULL the rows are taken through the sort's permutation,
+ *          row m = hidden[sorted_idx[m] / top_k]: no sorted copy of the
+ *          activations is written. sorted_idx comes from gnf4_moe_align (its
+ *          first M entries); an entry outside [0, n_tokens*top_k) sets
+ *          GNF4_DEVERR_SLOT and nothing is written.
+ *
+ * Descriptor fields (struct_bytes = sizeof(gnf4_gemm_desc)):
+ *   x or (hidden, sorted_idx, n_tokens, top_k): exactly one of x and hidden
+ *   is non-NULL; hidden is [n_tokens][K] bf16, n_tokens*top_k < 2^31.
+ *   w, scales, sizes, expert_ids, G, M, N, K, E, y, mode: as for
+ *   gnf4_grouped_gemm (K % 64 == 0 for both formats; N even for both SwiGLU
+ *   forms; swiglu_limit > 0 for the interleaved form).
+ *   scale_dtype: GNF4_SCALE_F32 or GNF4_SCALE_BF16 with NF4,
+ *   GNF4_SCALE_E8M0 with MXFP4.
+ * Kernels: DECODE runs every combination. PREFILL (and AUTO's prefill
+ * choice) runs NF4 with fp32 or bf16 absmax, MXFP4, gathered or sorted rows
+ * and every epilogue; anything else is refused with
+ * GNF4_ERR_UNSUPPORTED_SHAPE. Numerics as gnf4_grouped_gemm; an MXFP4 code
+ * value is exact in fp16 and bf16 and enters the MMA whole.
+ * Workspace: gnf4_workspace_bytes(GNF4_OP_GROUPED_GEMM, M, N, K, E, G).
+ * Alignment: x, hidden, w, y and the workspace 32-byte aligned; scales,
+ * sizes, expert_ids and sorted_idx 4-byte aligned.
+ */
+typedef struct gnf4_gemm_desc {
+    uint32_t struct_bytes;      /* sizeof(gnf4_gemm_desc) */
+    int32_t format;             /* gnf4_format */
+    int32_t scale_dtype;        /* gnf4_scale_dtype */
+    int32_t epilogue;           /* gnf4_epilogue */
+    float swiglu_alpha;         /* SWIGLU_INTERLEAVED: alpha (gpt-oss: 1.702) */
+    float swiglu_limit;         /* SWIGLU_INTERLEAVED: limit (gpt-oss: 7.0) */
+    int32_t mode;               /* gnf4_mode */
+    int32_t top_k;              /* gather: slots per token */
+    const uint16_t *x;          /* [M][K] bf16 rows in sorted order, or NULL to gather */
+    const uint16_t *hidden;     /* gather: [n_tokens][K] bf16 */
+    const int32_t *sorted_idx;  /* gather: [M] slot t*top_k+j of each row */
+    int64_t n_tokens;           /* gather: rows of hidden */
+    const uint8_t *w;           /* [E][N][K/2] packed codes */
+    const void *scales;         /* NF4: absmax [E][N][K/64]; MXFP4: e8m0 [E][N][K/32] */
+    const int32_t *sizes;       /* [G] */
+    const int32_t *expert_ids;  /* [G] */
+    int32_t G, N, K, E;
+    int64_t M;
+    uint16_t *y;                /* [M][N] or [M][N/2] bf16 */
+} gnf4_gemm_desc;
+
+GNF4_API gnf4_status gnf4_grouped_gemm_ex(const gnf4_gemm_desc *desc, void *workspace,
+                                          size_t ws_bytes, gnf4_stream_t stream);
 
 /*
  * gnf4_dequant_debug -- materialise NF4[code] * absmax for inspection/tests.
@@ -225,13 +325,23 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
  *
  *   dy          device bf16 [M][N] (the gradient of the GEMM's output y)
  *   w, absmax, sizes, expert_ids, G, E, blocksize: as for gnf4_grouped_gemm
- *   M >= 0, N >= 1, K % 64 == 0, 1 <= G, E <= GNF4_MAX_EXPERTS, M < 2^31
+ *   M >= 0, N >= 8 with N % 8 == 0, K % 64 == 0, 1 <= G, E <= GNF4_MAX_EXPERTS,
+ *   M < 2^31
  *   dx          device bf16 [M][K] (written; must not overlap dy)
  *   workspace   device, >= gnf4_workspace_bytes(GNF4_OP_GROUPED_DGRAD, ...)
- *               bytes (the 256-byte status header), zero-filled once.
+ *               bytes: the 256-byte status header, one counter per (SM,
+ *               value) and the fp32 partials of the tiles the stream-K split
+ *               cuts (4 KB per SM); zero it once (each call leaves the
+ *               counters at zero).
+ * One launch of a tensor-core kernel (mma.sync, fp32 accumulation) over
+ * batches of up to 8 rows and 64-element blocks of k, split over the SMs by
+ * tile-stages of 256 weight rows. Numerics: the weight carried as two fp16
+ * parts (within 1e-7 relative of NF4[code]); dy * absmax, exact in fp32,
+ * scaled by a power of two per (row, 16 weight rows) and carried as two fp16
+ * parts; fp32 sums, a fixed summation order (deterministic for a given GPU).
+ * Alignment: dy and w 16-byte aligned, absmax 4, dx 2, workspace 16.
  * A metadata error (as for gnf4_grouped_gemm) sets the device error word and
- * nothing is written. One launch of a CUDA-core kernel sized for decode
- * batches (it is not the tensor-core path).
+ * nothing is written.
  */
 GNF4_API gnf4_status gnf4_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const float *absmax,
                                         const int32_t *sizes, const int32_t *expert_ids,

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert gnf4.gnf4_version() == 110
+    assert gnf4.gnf4_version() == 120
     assert gnf4.gnf4_status_string(0) == "GNF4_OK"
     assert "HOST_POINTER" in gnf4.gnf4_status_string(2)
     assert gnf4.gnf4_status_string(99) == "GNF4_ERR_UNKNOWN"
@@ -117,8 +117,11 @@ def test_grouped_dgrad_host_checks():
     assert dg(dy=None) == 1 and dg(dx=None) == 1 and dg(M=-1) == 1 and dg(G=0) == 1
     assert dg(K=96) == 3 and dg(bs=32) == 3 and dg(E=2000) == 3
     assert dg(ws_bytes=16) == 4
-    assert dg(M=0) == 0
-    assert gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_DGRAD, 8, 16, 128, 2, 2) == 256
+    assert dg(N=12) == 3                                 # the tensor-core dgrad needs N % 8 == 0
+    need = gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_DGRAD, 8, 16, 128, 2, 2)
+    assert need > 256                                    # header + split counters and partials
+    assert dg(ws_bytes=need - 1) == 4
+    assert dg(M=0, ws_bytes=need) == 0
 
 
 def test_host_buffers_are_refused():
@@ -129,5 +132,41 @@ def test_host_buffers_are_refused():
     assert gnf4.load_library().gnf4_dequant_debug(p, p, 4, 64, 64, 0, p, None) == 2
     assert gnf4.load_library().gnf4_router_topk(p, 4, 8, 2, 1, p, p, None) == 2
     assert gnf4.load_library().gnf4_moe_combine(p, p, p, 4, 2, 64, p, p, 1 << 12, None) == 2
-    assert gnf4.load_library().gnf4_grouped_dgrad(p, p, p, p, p, 1, 4, 8, 64, 1, 64, p, p, 256,
-                                                  None) == 2
+    assert gnf4.load_library().gnf4_grouped_dgrad(p, p, p, p, p, 1, 4, 8, 64, 1, 64, p, p,
+                                                  1 << 30, None) == 2
+
+
+def test_grouped_gemm_ex_host_checks():
+    # The descriptor entry point refuses bad descriptors before any launch
+    # (fake device pointers: every case fails before they are dereferenced).
+    import ctypes
+    lib = gnf4.load_library()
+
+    def desc(**kw):
+        d = gnf4.GemmDesc()
+        d.struct_bytes = ctypes.sizeof(gnf4.GemmDesc)
+        d.format, d.scale_dtype, d.epilogue = gnf4.GNF4_FMT_NF4, gnf4.GNF4_SCALE_F32, 0
+        d.swiglu_alpha, d.swiglu_limit, d.mode, d.top_k = 1.702, 7.0, 0, 1
+        d.x, d.w, d.scales, d.sizes, d.expert_ids, d.y = 64, 64, 64, 64, 64, 64
+        d.G, d.N, d.K, d.E, d.M = 1, 8, 64, 1, 1
+        for k, v in kw.items():
+            setattr(d, k, v)
+        return d
+
+    def call(d):
+        return lib.gnf4_grouped_gemm_ex(ctypes.byref(d), 64, 1 << 20, None)
+
+    assert call(desc(struct_bytes=8)) == 1                       # wrong struct size
+    assert call(desc(format=2)) == 1                             # unknown format
+    assert call(desc(scale_dtype=gnf4.GNF4_SCALE_E8M0)) == 1     # NF4 with e8m0 scales
+    assert call(desc(format=gnf4.GNF4_FMT_MXFP4)) == 1           # MXFP4 with fp32 scales
+    assert call(desc(epilogue=3)) == 1
+    assert call(desc(epilogue=2, swiglu_limit=0.0)) == 1         # the clamp needs a limit
+    assert call(desc(epilogue=2, N=7)) == 3                      # odd N with SwiGLU
+    assert call(desc(hidden=64)) == 1                            # x and hidden both given
+    assert call(desc(x=None)) == 1                               # neither
+    assert call(desc(x=None, hidden=64, sorted_idx=64, top_k=0)) == 1
+    assert call(desc(K=96)) == 3                                 # K % 64
+    assert call(desc(M=0)) == 0                                  # nothing to do
+    assert call(desc()) == 2                                     # fake pointers: not device memory
+    assert lib.gnf4_grouped_gemm_ex(None, 64, 1 << 20, None) == 1

@@ -386,14 +386,29 @@ def test_prefill_gemm_full_size_mixtral(gi):
     check_gemm(x, packed, absmax, sizes, experts, mode=gnf4.GNF4_MODE_AUTO, rows=rows)
 
 
-def test_prefill_refuses_fused_swiglu():
-    rng = np.random.default_rng(3)
-    x = synth.activations_bf16(300, 64, seed=3)
-    packed = rng.integers(0, 256, size=(1, 64, 32), dtype=np.uint8)
-    absmax = rng.uniform(0.01, 0.1, size=(1, 64, 1)).astype(np.float32)
-    with pytest.raises(gnf4.Gnf4Error) as ei:
-        run_gemm(x, packed, absmax, [300], [0], swiglu=True, mode=gnf4.GNF4_MODE_PREFILL)
-    assert ei.value.status == 3
-    # AUTO keeps a fused SwiGLU on the decode kernel
-    check_gemm(x, packed, absmax, [300], [0], swiglu=True, mode=gnf4.GNF4_MODE_AUTO,
-               rows=np.array([0, 150, 299]))
+@pytest.mark.parametrize("E,N,K,sizes,experts", [
+    (3, 520, 192, [300, 0, 513, 7], [2, 0, 1, 1]),     # ragged groups, N/2 = 260 not /128
+    (2, 512, 2048, [256, 255, 257], [1, 0, 1]),        # token-tile edges
+    (2, 200, 128, [300, 40], [1, 0]),                  # rows of y (N/2 = 100) not /16 bytes
+])
+def test_prefill_gemm_fused_swiglu(E, N, K, sizes, experts):
+    # The tensor-core kernel pairs gate row j and up row N/2 + j in the same
+    # warp's TMEM lanes and combines them in the epilogue.
+    rng = np.random.default_rng(E * 17 + N + K)
+    M = int(sum(sizes))
+    x = synth.activations_bf16(M, K, seed=E + N)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    check_gemm(x, packed, absmax, sizes, experts, swiglu=True, mode=gnf4.GNF4_MODE_PREFILL)
+
+
+def test_prefill_gemm_full_size_mixtral_swiglu_through_auto():
+    # Mixtral-8x22B-shaped gate_up with the fused SwiGLU: AUTO now takes the
+    # tensor-core kernel (8192 rows over 8 experts); stratified rows.
+    w = synth.WORKLOADS["mixtral_8x22b"]
+    g = w.gemms[0]
+    _, sizes, experts, ng = groups_from_routing(w)
+    packed, absmax = synth.random_packed_stack(w.E, g.N, g.K, seed=0, which=g.name)
+    x = synth.activations_bf16(w.M, g.K, seed=0, which=g.name)
+    rows = tile_strata(sizes[:ng], seed=9)
+    check_gemm(x, packed, absmax, sizes, experts, swiglu=True, mode=gnf4.GNF4_MODE_AUTO, rows=rows)

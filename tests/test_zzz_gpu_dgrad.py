@@ -23,6 +23,8 @@ pytestmark = pytest.mark.gpu
     (3, 200, 192, [0, 1, 7, 8, 9, 17, 0], [2, 0, 1, 2, 0, 1, 1]),   # ragged, empty groups
     (4, 2048, 1024, [2, 3, 0, 3], [3, 1, 0, 0]),             # OLMoE-like down shapes
     (2, 96, 2880, [5, 4], [1, 1]),                           # K = 2880 (not a multiple of 256)
+    (3, 1024, 2048, [1, 1, 1, 1, 1, 1, 1, 1], [0, 1, 2, 0, 1, 2, 0, 1]),  # 8 one-row groups: a starved grid
+    (2, 5760, 2880, [37, 3], [1, 0]),                        # GPT-OSS-like gate_up rows, > 8 rows a group
     (8, 64, 320, [1] * 8, list(range(8))[::-1]),
 ])
 def test_grouped_dgrad_parity(E, N, K, sizes, experts):
@@ -51,7 +53,7 @@ def test_grouped_dgrad_bad_metadata_sets_error_and_writes_nothing():
     absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
     for sizes, experts, bit in [([2, 2], [0, 1], "sizes"), ([3, 3], [0, 3], "expert"),
                                 ([7, -1], [0, 1], "sizes")]:
-        ws = gnf4.make_workspace(256)
+        ws = gnf4.make_workspace(gnf4.gnf4_workspace_bytes(gnf4.GNF4_OP_GROUPED_DGRAD, 6, N, K, E, 2))
         dx = torch.full((6, K), 7.0, dtype=torch.bfloat16, device="cuda")
         gnf4.gnf4_grouped_dgrad(bf16_to_dev(dy), dev(packed), dev(absmax),
                                 dev(np.asarray(sizes, np.int32)),
