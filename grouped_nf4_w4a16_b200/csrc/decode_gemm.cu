@@ -96,8 +96,9 @@ constexpr int kRowOffOff = kXsOff + kStages * kXsStage;       // int32 [kMaxG + 
 constexpr int kBarOff = (kRowOffOff + (kMaxG + 1) * 4 + 7) / 8 * 8;   // mbarriers, see kNumBars
 // full[kStages] (copies landed), empty[kStages] (consumers done), xready
 // [kStages] (activations converted), then per unit pair: xfull (the three
-// partial sums written), xempty (the block-0 warp done reading them)
-constexpr int kNumBars = 3 * kStages + kTileUnits;
+// partial sums written), xempty (the block-0 warp done reading them), and
+// `never`, which nothing arrives at (the wait-limit test hook)
+constexpr int kNumBars = 3 * kStages + kTileUnits + 1;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;              // int [8]
 // table: 256-byte row per packed byte b: lane l's hi pair at l * 4, its
 // remainder pair at 128 + l * 4
@@ -154,7 +155,7 @@ struct Tile {
 // Tile t: batch t / tpb, the (t % tpb)-th run of up to 8 units of it.
 __device__ __forceinline__ Tile make_tile(int64_t t, const Problem &p, const int *batch_start,
                                           const int *row_off, const uint16_t *gexp) {
-  const int64_t bt = t / p.tpb;
+  const int64_t bt = div_fast(t, p.tpb);
   const int32_t jt = static_cast<int32_t>(t - bt * p.tpb);
   int lo = 0, hi = p.G;   // invariant: batch_start[lo] <= bt < batch_start[hi]
   while (hi - lo > 1) {
@@ -176,7 +177,7 @@ __device__ __forceinline__ Tile make_tile(int64_t t, const Problem &p, const int
 // one of the two for every CTA that holds a piece of it).
 __device__ __forceinline__ int64_t piece_slot(int64_t W, int64_t P, int64_t KC, int64_t t,
                                               int64_t c) {
-  return c * 2 + (range_lo(W, P, c) / KC == t ? 0 : 1);
+  return c * 2 + (div_fast(range_lo(W, P, c), KC) == t ? 0 : 1);
 }
 
 // Packed-weight tensor maps: boxes of 8, 16, 32, 64 and 128 rows x 128 bytes
@@ -320,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *xready = empty + kStages;
   uint64_t *xfull = xready + kStages;          // [kPairs]
   uint64_t *xempty = xfull + kPairs;           // [kPairs]
+  uint64_t *never = xempty + kPairs;
   int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort
   volatile int *abort_flag = &misc[1];
   __shared__ int s_tot;       // total batches (written by warp 0 with the group table)
@@ -347,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&xfull[i], 3);
       mbar_init(&xempty[i], 1);
     }
+    mbar_init(never, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int i = 0; i < kNumWMaps; ++i) prefetch_tensormap(&wmaps.m[i]);
     if (a.epi == 2)
@@ -373,8 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
-  // bounded waits give up after the header's limit when it sets one
-  const uint64_t limit_ns = hdr->reserved[0] ? static_cast<uint64_t>(hdr->reserved[0]) : kTimeoutNs;
+  // Test hook: a non-zero word 2 of the header shortens every bounded wait to
+  // that many nanoseconds, and the consumers then start with a wait on a
+  // barrier that nothing arrives at, so the timeout path runs for certain.
+  const uint32_t hook_ns = hdr->reserved[0];
+  const uint64_t limit_ns = hook_ns ? static_cast<uint64_t>(hook_ns) : kTimeoutNs;
 
   // ---- group table from (sizes, expert_ids), validated on the device: built
   //      by warp 0 alone (its lanes' loads in flight together, one warp scan),
@@ -452,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = lane >> 3, r = lane & 7;
     uint32_t it = 0;
     for (int64_t s = s_lo; s < s_hi;) {
-      const int64_t t = s / KC;
+      const int64_t t = div_fast(s, KC);
       const int k0 = static_cast<int>(s - t * KC);
       const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
       const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int64_t s = s_lo; s < s_hi && ok;) {
-      const int64_t t = s / KC;
+      const int64_t t = div_fast(s, KC);
       const int k0 = static_cast<int>(s - t * KC);
       const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
       const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
@@ -670,9 +676,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto xchg_at = [&](int b, int uu) -> float4 * {
     return reinterpret_cast<float4 *>(smem + kXchgOff) + ((up * 3 + (b - 1)) * 2 + uu) * 32 + lane;
   };
+  if (hook_ns != 0 && !warp_wait_all(never, 0, abort_flag, hdr, limit_ns)) return;
   uint32_t it = 0, ep = 0;
   for (int64_t s = s_lo; s < s_hi;) {
-    const int64_t t = s / KC;
+    const int64_t t = div_fast(s, KC);
     const int k0 = static_cast<int>(s - t * KC);
     const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
     const Tile tl = make_tile(t, p, batch_start, row_off, gexp);

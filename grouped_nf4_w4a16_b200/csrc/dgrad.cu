@@ -18,9 +18,9 @@
 //   each of its 4 rows and decodes each byte through the per-lane replicated
 //   byte -> (fp16 code value of even k, odd k) table; byte permutes then pair
 //   the values of two rows for one k (the MMA's A register pairs run along
-//   the contraction). Weight values carry two fp16 parts (hi and the
-//   remainder times 2^13), within 1e-7 relative of NF4[code], as the decode
-//   GEMM does with a fused SwiGLU.
+//   the contraction). Weight values enter as their fp16 rounding (relative
+//   error at most 2^-12, as the decode GEMM without SwiGLU; kDgParts = 2
+//   adds the remainder times 2^13, within 1e-7 relative of NF4[code]).
 //   B: absmax varies with n, so it joins dy: dy'[m][n] = dy[m][n] *
 //   absmax[n][block of the tile], exact in fp32, then scaled by a power of
 //   two per (row m, 16 n of a warp) into [2^14, 2^15) and split into two
@@ -58,6 +58,9 @@ constexpr int kDgAStage = kDgRows * 4;       // absmax of the stage's rows
 constexpr int kDgMaxG = GNF4_MAX_EXPERTS;
 constexpr int kRedFloats = 16;               // per lane: 4 m-tiles x 4 accumulators
 constexpr float kWLoInv = 1.0f / 8192.0f;    // weight remainders carried times 2^13
+// fp16 parts per code value: one, the rounding of NF4[code] (relative error at
+// most 2^-12, as the decode GEMM without SwiGLU), or two (within 1e-7)
+constexpr int kDgParts = 1;
 constexpr float kYLoInv = 1.0f / 2048.0f;    // dy' remainders carried times 2^11
 
 // Shared memory, absolute shared-window addresses (the table at a multiple
@@ -154,10 +157,12 @@ __global__ void __launch_bounds__(kDgThreads, 1)
   for (int i = tid; i < 256 * 8; i += kDgThreads) {
     const int b = i >> 3, part = i & 7;
     const uint32_t hp = code_hi(b >> 4) | (code_hi(b & 15) << 16);
-    const uint32_t lp = code_lo(b >> 4) | (code_lo(b & 15) << 16);
     uint4 *dst = reinterpret_cast<uint4 *>(smem + kDgLutOff + b * 256);
     dst[part] = make_uint4(hp, hp, hp, hp);
-    dst[8 + part] = make_uint4(lp, lp, lp, lp);
+    if (kDgParts == 2) {
+      const uint32_t lp = code_lo(b >> 4) | (code_lo(b & 15) << 16);
+      dst[8 + part] = make_uint4(lp, lp, lp, lp);
+    }
   }
 
   pdl_wait();
@@ -218,7 +223,7 @@ __global__ void __launch_bounds__(kDgThreads, 1)
 
   // batch of tile t: first row, valid rows, expert
   auto tile_batch = [&](int64_t t, int64_t *row0, int *mrows, int *e) {
-    const int64_t bt = t / KB;
+    const int64_t bt = div_fast(t, KB);
     int lo = 0, hi = G;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -236,13 +241,13 @@ __global__ void __launch_bounds__(kDgThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int64_t s = s_lo; s < s_hi && ok;) {
-      const int64_t t = s / KC;
+      const int64_t t = div_fast(s, KC);
       const int k0 = static_cast<int>(s - t * KC);
       const int k1 = static_cast<int>(min(static_cast<int64_t>(KC), k0 + (s_hi - s)));
       int64_t row0;
       int mrows, e;
       tile_batch(t, &row0, &mrows, &e);
-      const int kb = static_cast<int>(t % KB);
+      const int kb = static_cast<int>(t - div_fast(t, KB) * KB);
       const int64_t ebase = static_cast<int64_t>(e) * N;
       for (int kc = k0; kc < k1; ++kc, ++it) {
         const int st = static_cast<int>(it % kDgStages);
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kDgThreads, 1)
   float *red = reinterpret_cast<float *>(smem + kDgRedOff);
   uint32_t it = 0, ep = 0;
   for (int64_t s = s_lo; s < s_hi;) {
-    const int64_t t = s / KC;
+    const int64_t t = div_fast(s, KC);
     const int k0 = static_cast<int>(s - t * KC);
     const int k1 = static_cast<int>(min(static_cast<int64_t>(KC), k0 + (s_hi - s)));
     // D fragments of the 4 m-tiles: [t][0] k = 2 (4 g + t), row 2q; [1] same
@@ -358,26 +363,31 @@ __global__ void __launch_bounds__(kDgThreads, 1)
       const uint32_t wc = *reinterpret_cast<const uint32_t *>(wst + woff + 8 * 32);
       const uint32_t wd = *reinterpret_cast<const uint32_t *>(wst + woff + 12 * 32);
       uint32_t ha[4], la[4], hb[4], lb[4], hc[4], lc[4], hd[4], ld[4];
-      decode_word<2>(lutlane, wa, ha, la);
-      decode_word<2>(lutlane, wb, hb, lb);
-      decode_word<2>(lutlane, wc, hc, lc);
-      decode_word<2>(lutlane, wd, hd, ld);
+      decode_word<kDgParts>(lutlane, wa, ha, la);
+      decode_word<kDgParts>(lutlane, wb, hb, lb);
+      decode_word<kDgParts>(lutlane, wc, hc, lc);
+      decode_word<kDgParts>(lutlane, wd, hd, ld);
 #pragma unroll
       for (int t4 = 0; t4 < 4; ++t4) {
         // pair two rows' values of one k: a0/a2 even k (MMA row g), a1/a3 odd
         const uint32_t a0 = prmt(ha[t4], hb[t4], 0x5410u), a1 = prmt(ha[t4], hb[t4], 0x7632u);
         const uint32_t a2 = prmt(hc[t4], hd[t4], 0x5410u), a3 = prmt(hc[t4], hd[t4], 0x7632u);
-        const uint32_t r0 = prmt(la[t4], lb[t4], 0x5410u), r1 = prmt(la[t4], lb[t4], 0x7632u);
-        const uint32_t r2 = prmt(lc[t4], ld[t4], 0x5410u), r3 = prmt(lc[t4], ld[t4], 0x7632u);
-        float chh[4], chl[4], clh[4];
-        mma_f16_z(chh, a0, a1, a2, a3, bh[0], bh[1]);   // hi weights x hi dy'
-        mma_f16_z(chl, a0, a1, a2, a3, bl[0], bl[1]);   // hi weights x dy' remainders
-        mma_f16_z(clh, r0, r1, r2, r3, bh[0], bh[1]);   // weight remainders x hi dy'
+        float chh[4], chl[4];
+        mma_f16_z(chh, a0, a1, a2, a3, bh[0], bh[1]);   // weights x hi dy'
+        mma_f16_z(chl, a0, a1, a2, a3, bl[0], bl[1]);   // weights x dy' remainders
+        float sum[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float sum = fmaf(clh[i], kWLoInv, fmaf(chl[i], kYLoInv, chh[i]));
-          acc[t4][i] = fmaf(sum, (i & 1) ? inv1 : inv0, acc[t4][i]);
+        for (int i = 0; i < 4; ++i) sum[i] = fmaf(chl[i], kYLoInv, chh[i]);
+        if (kDgParts == 2) {
+          const uint32_t r0 = prmt(la[t4], lb[t4], 0x5410u), r1 = prmt(la[t4], lb[t4], 0x7632u);
+          const uint32_t r2 = prmt(lc[t4], ld[t4], 0x5410u), r3 = prmt(lc[t4], ld[t4], 0x7632u);
+          float clh[4];
+          mma_f16_z(clh, r0, r1, r2, r3, bh[0], bh[1]);   // weight remainders x hi dy'
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sum[i] = fmaf(clh[i], kWLoInv, sum[i]);
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[t4][i] = fmaf(sum[i], (i & 1) ? inv1 : inv0, acc[t4][i]);
       }
       __syncwarp();
       mbar_arrive_elect(&empty[st]);
@@ -403,7 +413,7 @@ __global__ void __launch_bounds__(kDgThreads, 1)
     int mrows, e;
     tile_batch(t, &row0, &mrows, &e);
     const int t4 = warp >> 2, i = warp & 3;
-    const int kk = static_cast<int>(t % KB) * 64 + 2 * (4 * g + t4) + (i >> 1);
+    const int kk = static_cast<int>(t - div_fast(t, KB) * KB) * 64 + 2 * (4 * g + t4) + (i >> 1);
     const int m = 2 * q + (i & 1);
     const int64_t b_first = cta_of(W, P, t * KC), b_last = cta_of(W, P, t * KC + KC - 1);
     if (b_first != b_last) {
@@ -411,7 +421,7 @@ __global__ void __launch_bounds__(kDgThreads, 1)
       // CTA's slot (first or last tile of its range), count it; the piece
       // that counts last adds all pieces in order and stores
       auto slot = [&](int64_t c) -> float * {
-        const int64_t which = range_lo(W, P, c) / KC == t ? 0 : 1;
+        const int64_t which = div_fast(range_lo(W, P, c), KC) == t ? 0 : 1;
         return partials + ((c * 2 + which) * kRedFloats + warp) * 32;
       };
       slot(blockIdx.x)[lane] = val;

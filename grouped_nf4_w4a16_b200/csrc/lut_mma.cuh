@@ -120,20 +120,24 @@ __device__ __forceinline__ uint32_t code_lo(int c) {
   return half_bits((nf4_value(c) - __half2float(h)) * 8192.0f);
 }
 
+// a / b and a % b for non-negative a, b > 0: 32-bit when both fit (a
+// uniform branch; the 64-bit division is a long software sequence).
+__device__ __forceinline__ int64_t div_fast(int64_t a, int64_t b) {
+  if (((a | b) >> 32) == 0)
+    return static_cast<int64_t>(static_cast<uint32_t>(a) / static_cast<uint32_t>(b));
+  return a / b;
+}
+
 // Stream-K range arithmetic over W tile-stages and P CTAs: CTA b owns
 // [range_lo(b), range_lo(b + 1)); cta_of(s) is the CTA that owns stage s.
 // (64-bit products while W * P stays below 2^62, which covers every shape
 // the host accepts by a wide margin; 128-bit otherwise)
 __device__ __forceinline__ int64_t range_lo(int64_t W, int64_t P, int64_t b) {
-  if (W < (int64_t{1} << 54))
-    return static_cast<int64_t>(static_cast<uint64_t>(W) * static_cast<uint64_t>(b) /
-                                static_cast<uint64_t>(P));
+  if (W < (int64_t{1} << 54)) return div_fast(W * b, P);
   return static_cast<int64_t>((static_cast<unsigned __int128>(W) * b) / P);
 }
 __device__ __forceinline__ int64_t cta_of(int64_t W, int64_t P, int64_t s) {
-  if (W < (int64_t{1} << 54))
-    return static_cast<int64_t>((static_cast<uint64_t>(s + 1) * static_cast<uint64_t>(P) - 1) /
-                                static_cast<uint64_t>(W));
+  if (W < (int64_t{1} << 54)) return div_fast((s + 1) * P - 1, W);
   return static_cast<int64_t>((static_cast<unsigned __int128>(s + 1) * P - 1) / W);
 }
 

@@ -363,16 +363,25 @@ __device__ __forceinline__ int64_t weight_row(const PrefillParams &p, int n0, ui
   return 2 * j + (l & 1);
 }
 
-// One scale value (block scale times nothing else) as fp32: element idx of
-// the stack's scale array; for e8m0 the larger of the pair at 2-byte element
-// idx (row maxima only need the larger).
-__device__ __forceinline__ float scale_max_at(const PrefillParams &p, int64_t idx) {
-  if (p.scale_kind == kScaleF32) return fabsf(__ldg(static_cast<const float *>(p.scales) + idx));
-  const uint32_t v = __ldg(static_cast<const unsigned short *>(p.scales) + idx);
-  if (p.scale_kind == kScaleBf16) return fabsf(__uint_as_float(v << 16));
-  const uint32_t m = max(v & 0xFFu, v >> 8);
+// A row maximum of the block scales is gathered from raw loads: the raw bits
+// of element idx of the scale array (fp32, bf16, or an e8m0 pair at 2-byte
+// element idx), and their magnitude as fp32 (for e8m0 the larger of the
+// pair). The two are split so that a load issued ahead is only consumed
+// where its value is needed.
+__device__ __forceinline__ uint32_t scale_raw_at(const PrefillParams &p, int64_t idx) {
+  if (p.scale_kind == kScaleF32)
+    return __float_as_uint(__ldg(static_cast<const float *>(p.scales) + idx));
+  return __ldg(static_cast<const unsigned short *>(p.scales) + idx);
+}
+__device__ __forceinline__ float scale_mag(const PrefillParams &p, uint32_t raw) {
+  if (p.scale_kind == kScaleF32) return fabsf(__uint_as_float(raw));
+  if (p.scale_kind == kScaleBf16) return fabsf(__uint_as_float(raw << 16));
+  const uint32_t m = max(raw & 0xFFu, raw >> 8);
   return m == 255u ? __uint_as_float(0x7FC00000u)
                    : (m == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(m << 23));
+}
+__device__ __forceinline__ float scale_max_at(const PrefillParams &p, int64_t idx) {
+  return scale_mag(p, scale_raw_at(p, idx));
 }
 
 // Warp-uniform bounded wait with cluster-scope acquire: lane 0 waits, every
@@ -737,9 +746,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, G, tile_start, row_off, gsize, gexp, ncols_tile);
         const int64_t ap_next = row_scales(t + npairs);
         float mx_next = 0.0f;
-        float nxq[4];   // next tile's block scales, folded 4 K-steps after their load
+        uint32_t nxq[4];   // next tile's raw block scales, folded 4 K-steps after their load
 #pragma unroll
-        for (int j = 0; j < 4; ++j) nxq[j] = 0.0f;
+        for (int j = 0; j < 4; ++j) nxq[j] = 0u;
         bool rok;
         const int64_t n = weight_row(p, ti.n0, rank, rl, &rok);
         // scale-array element index of this row's blocks (for the 2-byte
@@ -787,8 +796,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             am *= rscale;
             // next tile's block scales, first used 4 K-steps after their load (no wait here)
-            mx_next = fmaxf(mx_next, nxq[sub]);
-            nxq[sub] = ap_next >= 0 ? scale_max_at(p, ap_next + kb) : 0.0f;
+            mx_next = fmaxf(mx_next, scale_mag(p, nxq[sub]));
+            nxq[sub] = ap_next >= 0 ? scale_raw_at(p, ap_next + kb) : 0u;
             const int s = g % kAStages;
             const uint32_t ph = (g / kAStages) & 1u;
             // hi[i]: bf16 pair of k = 32 half + 2i, 2i+1; lo[i]: e4m3 of k = 32 half + 4i .. +3
@@ -841,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, nxq[j]);
+        for (int j = 0; j < 4; ++j) mx_next = fmaxf(mx_next, scale_mag(p, nxq[j]));
         mx = mx_next;
         // ---- epilogue: accumulator -> bf16 y (this CTA's 128 weight rows).
         // Chunks of 32 tokens: scaled and rounded into a shared-memory box
