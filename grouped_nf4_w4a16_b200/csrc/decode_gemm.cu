@@ -65,9 +65,20 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kTmaWarp = kConsumerWarps;          // issues the tensor copies
-constexpr int kScaleWarp = kConsumerWarps + 1;    // copies scales (and gathered activations)
-constexpr int kXWarp = kConsumerWarps + 2;        // converts the staged activations to fp16
-constexpr int kThreads = (kConsumerWarps + 3) * 32;
+// The three other warps copy scales (and gathered activations) or convert
+// the staged activations to fp16. With one 16-byte scale copy per row one
+// copy warp keeps up and two convert; with 4-byte copies two copy and one
+// converts. 20 warps keep 96 registers per thread (each SM sub-partition
+// holds 5 of them); a copy warp that also issued the tensor copies delayed
+// them behind its own copies.
+constexpr int kThreads = (kConsumerWarps + 4) * 32;
+template <bool WIDE>
+struct WarpRoles {
+  static constexpr int kScaleWarps = WIDE ? 1 : 2;
+  static constexpr int kXWarps = 3 - kScaleWarps;
+  static constexpr int kScaleWarp0 = kTmaWarp + 1;
+  static constexpr int kXWarp0 = kScaleWarp0 + kScaleWarps;
+};
 constexpr int kTileUnits = 8;                 // units per tile (2 row groups each)
 constexpr int kStages = 6;
 constexpr int kBatch = 8;                     // activation rows per batch (MMA N)
@@ -279,12 +290,19 @@ __device__ __forceinline__ void store_outputs(uint16_t *y, float alpha, float li
 
 // PARTS: fp16 parts per NF4 code value (1 or 2). SK: the scale encoding
 // (kScaleF32, kScaleBf16, or kScaleE8m0 for MXFP4, which is one part).
-template <int PARTS, int SK>
+// WIDE: fp32 scales whose 4 blocks of a stage are one 16-byte aligned run in
+// every row (K % 256 == 0, scales 16-byte aligned), copied 16 bytes at a time.
+template <int PARTS, int SK, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gemm_kernel(const __grid_constant__ WeightMaps wmaps,
                        const __grid_constant__ CUtensorMap xmap,
                        const __grid_constant__ DecodeParams a) {
   constexpr bool MX = SK == kScaleE8m0;
+  static_assert(!WIDE || SK == kScaleF32, "16-byte scale copies are for fp32 scales");
+  constexpr int kScaleWarps = WarpRoles<WIDE>::kScaleWarps;
+  constexpr int kXWarps = WarpRoles<WIDE>::kXWarps;
+  constexpr int kScaleWarp0 = WarpRoles<WIDE>::kScaleWarp0;
+  constexpr int kXWarp0 = WarpRoles<WIDE>::kXWarp0;
   extern __shared__ __align__(1024) char smem_raw[];
   // The parameters the loops use, as locals: the parameter block's address
   // is never taken, so every use is a constant-bank operand, not a load that
@@ -341,9 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     misc[0] = 0;
     misc[1] = 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 32 + 1);            // 32 cp.async arrivals + the byte-count arrival
+      // one cp.async arrival per scale-warp lane + the byte-count arrival
+      mbar_init(&full[s], 32 * kScaleWarps + 1);
       mbar_init(&empty[s], kConsumerWarps);
-      mbar_init(&xready[s], 1);
+      mbar_init(&xready[s], kXWarps);
     }
     for (int i = 0; i < kPairs; ++i) {
       mbar_init(&xfull[i], 3);
@@ -448,40 +467,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (static_cast<int64_t>(blockIdx.x) >= P) return;
   const int64_t s_lo = range_lo(W, P, blockIdx.x), s_hi = range_lo(W, P, blockIdx.x + 1);
 
-  if (warp == kXWarp) {
+  if (warp >= kXWarp0) {
     // ------------------------------------------------ activation conversion
-    // Per stage, lane (block b = lane / 8, row r = lane % 8) rewrites its 64
-    // staged bf16 activations in place as fp16 x * 2^S, S putting the
-    // largest magnitude of those 64 in [2^14, 2^15) (0 for all zeros, Inf or
-    // NaN): exact for every value above 2^-28 of that maximum. 2^-S goes to
-    // the stage's scale table for the consumers' block sums.
-    const int b = lane >> 3, r = lane & 7;
+    // Per stage, each (block b, row r) of the staged bf16 activations is
+    // rewritten in place as fp16 x * 2^S, S putting the largest magnitude of
+    // its 64 values in [2^14, 2^15) (0 for all zeros, Inf or NaN): exact for
+    // every value above 2^-28 of that maximum. 2^-S goes to the stage's
+    // scale table for the consumers' block sums. The kXWarps lanes of one
+    // (block, row) take 8 / kXWarps of its 16-byte chunks each.
+    constexpr int kChunks = 8 / kXWarps;
+    const int xi = (warp - kXWarp0) * 32 + lane;
+    const int h = xi % kXWarps, b = (xi / kXWarps) >> 3, r = (xi / kXWarps) & 7;
     uint32_t it = 0;
     for (int64_t s = s_lo; s < s_hi;) {
       const int64_t t = div_fast(s, KC);
       const int k0 = static_cast<int>(s - t * KC);
       const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
       const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
+      // rows past the batch feed only outputs that are never stored: skipped
+      const bool live = r < tl.mrows;
+      const uint32_t pair_mask = __ballot_sync(0xffffffffu, live);
       for (int kc = k0; kc < k1; ++kc, ++it) {
         const int st = static_cast<int>(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
         if (!warp_wait_one(&full[st], ph, abort_flag, hdr, limit_ns)) return;
-        // rows past the batch feed only outputs that are never stored: skipped
-        if (r < tl.mrows) {
+        if (live) {
           char *row = smem + kXOff + st * kXStage + b * kBoxBytes + r * 128;
-          uint4 v[8];
-          // bf16 magnitudes compare as integers, two per word; four
-          // independent chains keep the reduction short
+          uint4 v[kChunks];
+          // bf16 magnitudes compare as integers, two per word
           uint32_t m4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            v[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ r) << 4));
+          for (int c = 0; c < kChunks; ++c) {
+            v[c] = *reinterpret_cast<const uint4 *>(row + (((kChunks * h + c) ^ r) << 4));
             m4[0] = __vmaxu2(m4[0], v[c].x & 0x7FFF7FFFu);
             m4[1] = __vmaxu2(m4[1], v[c].y & 0x7FFF7FFFu);
             m4[2] = __vmaxu2(m4[2], v[c].z & 0x7FFF7FFFu);
             m4[3] = __vmaxu2(m4[3], v[c].w & 0x7FFF7FFFu);
           }
-          const uint32_t mx2 = __vmaxu2(__vmaxu2(m4[0], m4[1]), __vmaxu2(m4[2], m4[3]));
+          uint32_t mx2 = __vmaxu2(__vmaxu2(m4[0], m4[1]), __vmaxu2(m4[2], m4[3]));
+          if (kXWarps == 2) mx2 = __vmaxu2(mx2, __shfl_xor_sync(pair_mask, mx2, 1));
           const uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
           const int eb = static_cast<int>(mx >> 7);   // biased exponent of the largest magnitude
           int S = 0;
@@ -489,19 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           S = S > 126 ? 126 : S;
           const float sc = __uint_as_float(static_cast<uint32_t>(S + 127) << 23);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kChunks; ++c) {
             const uint32_t in[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
             uint32_t out[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16) * sc,
-                                                  __uint_as_float(in[j] & 0xFFFF0000u) * sc);
-              out[j] = *reinterpret_cast<const uint32_t *>(&h);
+              const __half2 hv = __floats2half2_rn(__uint_as_float(in[j] << 16) * sc,
+                                                   __uint_as_float(in[j] & 0xFFFF0000u) * sc);
+              out[j] = *reinterpret_cast<const uint32_t *>(&hv);
             }
-            *reinterpret_cast<uint4 *>(row + ((c ^ r) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<uint4 *>(row + (((kChunks * h + c) ^ r) << 4)) =
+                make_uint4(out[0], out[1], out[2], out[3]);
           }
-          reinterpret_cast<float *>(smem + kXsOff + st * kXsStage)[lane] =
-              __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
+          if (h == 0)
+            reinterpret_cast<float *>(smem + kXsOff + st * kXsStage)[b * 8 + r] =
+                __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&xready[st]);
@@ -511,20 +537,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  if (warp >= kTmaWarp) {
+  if (warp >= kConsumerWarps) {
     // ------------------------------------------------------------ producers
-    // Two warps fill each stage: the copy warp issues the tensor copies (one
-    // byte-count arrival), the scale warp the 4-byte scale copies and, with a
-    // gather, the activation rows as 16-byte copies (one arrival per lane
-    // when its copies land). Split so that neither issue stream waits behind
-    // the other.
-    const bool scale_warp = warp == kScaleWarp;
-    const int r = lane >> 2, blk = lane & 3;
+    // Lane 0 of the copy warp issues the tensor copies (one byte-count
+    // arrival); the lanes of the scale warps copy scales and, with a gather,
+    // activation rows as 16-byte copies (one arrival per lane when its
+    // copies land). Scale warp sw takes the units i with i % kScaleWarps ==
+    // sw.
+    const bool scale_warp = warp >= kScaleWarp0;
+    const int sw = warp - kScaleWarp0;
+    const bool tma_lane = warp == kTmaWarp && lane == 0;
+    // WIDE: one copy per (unit, row group, row); else one 4-byte copy per
+    // (unit, row group, row, block)
+    constexpr bool wide = WIDE;
+    // wide: lane copies row r of row group wrg of units wu + 2 kScaleWarps jj;
+    // narrow: lane copies block blk of row r of its units
+    const int r = wide ? (lane & 7) : (lane >> 2);
+    const int blk = wide ? 0 : (lane & 3);
+    const int wrg = (lane >> 3) & 1, wu = sw + kScaleWarps * (lane >> 4);
     const int64_t total_rows = static_cast<int64_t>(p.E) * p.N;
     // scale bytes of the whole stack (2-byte encodings: the last word read
     // must stay inside it)
     const int64_t scale_bytes = total_rows * p.KB * 2;
-    // gathered activations: lane copies row gr = lane % 8 of block gb = lane / 8
+    // gathered activations: lane copies chunks sw * kGChunks + cc of row
+    // gr = lane % 8 of block gb = lane / 8
+    constexpr int kGChunks = 8 / kScaleWarps;
     const int gr = lane & 7, gb = lane >> 3;
     uint32_t it = 0;
     bool ok = true;
@@ -548,64 +585,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t e00 = wrow(0, 0, r) * p.KB + blk;
       const int64_t du = (wrow(1, 0, r) - wrow(0, 0, r)) * p.KB;
       const int64_t dg = (wrow(0, 1, r) - wrow(0, 0, r)) * p.KB;
-      if (scale_warp) {
-        for (int i = 0; i < tl.nunits; ++i)
+      for (int i = 0; i < tl.nunits; ++i)
 #pragma unroll
-          for (int rgi = 0; rgi < 2; ++rgi)
-            if (wrow(i, rgi, r) < ebase + p.N) vmask |= 1u << (2 * i + rgi);
-        if (gather && gr < tl.mrows) {
-          const int32_t slot = sorted_idx[tl.row0 + gr];   // checked in range up front
-          hrow = hidden + static_cast<int64_t>(slot / top_k) * p.K;
-        }
+        for (int rgi = 0; rgi < 2; ++rgi)
+          if (wrow(i, rgi, r) < ebase + p.N) vmask |= 1u << (2 * i + rgi);
+      if (scale_warp && gather && gr < tl.mrows) {
+        const int32_t slot = sorted_idx[tl.row0 + gr];   // checked in range up front
+        hrow = hidden + static_cast<int64_t>(slot / top_k) * p.K;
       }
       for (int kc = k0; kc < k1; ++kc, ++it) {
         const int st = static_cast<int>(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
         if (!warp_wait_one(&empty[st], ph ^ 1u, abort_flag, hdr, limit_ns)) { ok = false; break; }
-        if (scale_warp) {
-          // stage layout [unit][block][row][row group], one 4-byte word each:
-          // a consumer lane reads both row groups of its row in one 8-byte load
-          const uint32_t as = smem_u32(smem + kAOff + st * kAStage + (blk * 8 + r) * 8);
-          const bool kok = kc * kStageBlocks + blk < p.KB;
-          const int64_t ek = e00 + kc * kStageBlocks;   // element of unit 0, row group 0
-          if (scale_kind == kScaleF32) {
-            const float *fk = static_cast<const float *>(scales) + ek;
-            for (int i = 0; i < tl.nunits; ++i) {
-#pragma unroll
-              for (int rgi = 0; rgi < 2; ++rgi) {
-                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
-                cp_async4(as + i * 256 + rgi * 4, v ? fk + i * du + rgi * dg : scales, v ? 4u : 0u);
-              }
-            }
-          } else {
-            // the 4-byte word that holds the (row, block)'s 2 bytes (the last
-            // word of the stack is read only as far as the stack goes)
-            const char *cb = static_cast<const char *>(scales);
-            for (int i = 0; i < tl.nunits; ++i) {
-#pragma unroll
-              for (int rgi = 0; rgi < 2; ++rgi) {
-                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
-                const int64_t wb = ((ek + i * du + rgi * dg) * 2) & ~int64_t{3};
-                cp_async4(as + i * 256 + rgi * 4, v ? cb + wb : scales,
-                          v ? (wb + 4 <= scale_bytes ? 4u : 2u) : 0u);
-              }
-            }
-          }
-          if (gather) {
-            // the batch's rows of x for this stage's 4 blocks, through
-            // sorted_idx, into the layout the tensor copy gives (128-byte
-            // swizzle: chunk c of row r at chunk c ^ r); rows past the batch
-            // and blocks past K are zero-filled
-            const int kbx = kc * kStageBlocks + gb;
-            const bool v = hrow != nullptr && kbx < p.KB;
-            const uint32_t dst = smem_u32(smem + kXOff + st * kXStage + gb * kBoxBytes + gr * 128);
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              cp_async16(dst + ((c ^ gr) << 4), v ? hrow + kbx * 64 + c * 8 : hidden,
-                         v ? 16u : 0u);
-          }
-          cp_async_arrive_noinc(&full[st]);
-        } else if (lane == 0) {
+        if (tma_lane) {
           mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(tl.nunits * 16 * 128 +
                                                                  (gather ? 0 : kXStage)));
           char *ws = smem + kWOff + st * kWStage;
@@ -627,12 +619,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(smem + kXOff + st * kXStage, &xmap, 0, static_cast<int>(tl.row0),
                         kc * kStageBlocks, &full[st]);
         }
+        if (scale_warp) {
+          // stage layout [unit][row group][row][block], one 4-byte word
+          // each: the consumer lane of row g reads word g * 4 + blk of the
+          // unit's two row groups
+          const uint32_t as = smem_u32(smem + kAOff + st * kAStage + r * 16 + blk * 4);
+          const int64_t ek = e00 + kc * kStageBlocks;   // element of unit 0, row group 0
+          if (wide) {
+            const float *fk = static_cast<const float *>(scales) + ek;
+#pragma unroll
+            for (int jj = 0; jj < 4 / kScaleWarps; ++jj) {
+              const int i = wu + 2 * kScaleWarps * jj;
+              const bool v = (vmask >> (2 * i + wrg)) & 1u;
+              cp_async16(as + i * 256 + wrg * 128, v ? fk + i * du + wrg * dg : scales,
+                         v ? 16u : 0u);
+            }
+          } else if (scale_kind == kScaleF32) {
+            const bool kok = kc * kStageBlocks + blk < p.KB;
+            const float *fk = static_cast<const float *>(scales) + ek;
+            for (int i = sw; i < tl.nunits; i += kScaleWarps) {
+#pragma unroll
+              for (int rgi = 0; rgi < 2; ++rgi) {
+                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
+                cp_async4(as + i * 256 + rgi * 128, v ? fk + i * du + rgi * dg : scales,
+                          v ? 4u : 0u);
+              }
+            }
+          } else {
+            // the 4-byte word that holds the (row, block)'s 2 bytes (the last
+            // word of the stack is read only as far as the stack goes)
+            const bool kok = kc * kStageBlocks + blk < p.KB;
+            const char *cb = static_cast<const char *>(scales);
+            for (int i = sw; i < tl.nunits; i += kScaleWarps) {
+#pragma unroll
+              for (int rgi = 0; rgi < 2; ++rgi) {
+                const bool v = kok && ((vmask >> (2 * i + rgi)) & 1u);
+                const int64_t wb = ((ek + i * du + rgi * dg) * 2) & ~int64_t{3};
+                cp_async4(as + i * 256 + rgi * 128, v ? cb + wb : scales,
+                          v ? (wb + 4 <= scale_bytes ? 4u : 2u) : 0u);
+              }
+            }
+          }
+          if (gather) {
+            // the batch's rows of x for this stage's 4 blocks, through
+            // sorted_idx, into the layout the tensor copy gives (128-byte
+            // swizzle: chunk c of row r at chunk c ^ r); rows past the batch
+            // and blocks past K are zero-filled
+            const int kbx = kc * kStageBlocks + gb;
+            const bool v = hrow != nullptr && kbx < p.KB;
+            const uint32_t dst = smem_u32(smem + kXOff + st * kXStage + gb * kBoxBytes + gr * 128);
+#pragma unroll
+            for (int cc = 0; cc < kGChunks; ++cc) {
+              const int c = kGChunks * sw + cc;
+              cp_async16(dst + ((c ^ gr) << 4), v ? hrow + kbx * 64 + c * 8 : hidden,
+                         v ? 16u : 0u);
+            }
+          }
+          cp_async_arrive_noinc(&full[st]);
+        }
       }
       s += k1 - k0;
     }
-    if (scale_warp) {
-      cp_async_wait_all();
-    } else if (lane == 0) {
+    if (scale_warp) cp_async_wait_all();
+    if (tma_lane) {
       // the copies of the last stages must land before the CTA exits
       const uint32_t n = it < static_cast<uint32_t>(kStages) ? it : static_cast<uint32_t>(kStages);
       for (uint32_t d = 0; d < n; ++d) {
@@ -700,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const char *wst = smem + kWOff + st * kWStage;
         // 2^-S of activation rows 2q and 2q + 1 in this block
         const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + st * kXsStage)[blk * 4 + q];
-        const char *ast = smem + kAOff + st * kAStage + (blk * 8 + g) * 8;
+        const char *ast = smem + kAOff + st * kAStage + g * 16 + blk * 4;
         // (rows past the batch feed only outputs that are never stored)
         const char *xst = smem + kXOff + st * kXStage;
         const uint4 xf = *reinterpret_cast<const uint4 *>(xst + xoffF);
@@ -719,10 +768,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t wb0 = *reinterpret_cast<const uint32_t *>(r0 + offB);
           const uint32_t wa1 = *reinterpret_cast<const uint32_t *>(r1 + offA);
           const uint32_t wb1 = *reinterpret_cast<const uint32_t *>(r1 + offB);
-          const uint2 sw = *reinterpret_cast<const uint2 *>(ast + ui * 256);   // rows g, g + 8
+          // scale words of rows g and g + 8 (row groups 0 and 1)
+          uint32_t s0 = *reinterpret_cast<const uint32_t *>(ast + ui * 256);
+          uint32_t s1 = *reinterpret_cast<const uint32_t *>(ast + ui * 256 + 128);
           // the 2 scale bytes of (row, block) sit in the low or the high half
           // of the copied 4-byte word, as the element index is even or odd
-          uint32_t s0 = sw.x, s1 = sw.y;
           if (two_byte) {
             const int64_t j = tl.j0 + ui;
             const int64_t w0 = p.epi == 0 ? ebase + 16 * j + g
@@ -929,13 +979,19 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   d.partials = reinterpret_cast<float4 *>(ws + decode_zero_prefix_bytes(a.M, a.N, a.G, a.swiglu));
 
   const bool bf = !mx && a.scale_dtype == GNF4_SCALE_BF16;
-  auto kernel = mx ? decode_gemm_kernel<1, kScaleE8m0>
-                   : (parts == 2 ? (bf ? decode_gemm_kernel<2, kScaleBf16>
-                                       : decode_gemm_kernel<2, kScaleF32>)
-                                 : (bf ? decode_gemm_kernel<1, kScaleBf16>
-                                       : decode_gemm_kernel<1, kScaleF32>));
-  const int ki = mx ? 4 : (parts - 1) * 2 + (bf ? 1 : 0);
-  static bool configured[64][5] = {};
+  // 16-byte scale copies: fp32 scales, the 4 blocks of a stage one aligned
+  // run in every row
+  const bool wide = !mx && !bf && (a.K / 64) % kStageBlocks == 0 &&
+                    reinterpret_cast<uintptr_t>(a.scales) % 16 == 0;
+  auto kernel = mx ? decode_gemm_kernel<1, kScaleE8m0, false>
+                : bf ? (parts == 2 ? decode_gemm_kernel<2, kScaleBf16, false>
+                                   : decode_gemm_kernel<1, kScaleBf16, false>)
+                : wide ? (parts == 2 ? decode_gemm_kernel<2, kScaleF32, true>
+                                     : decode_gemm_kernel<1, kScaleF32, true>)
+                       : (parts == 2 ? decode_gemm_kernel<2, kScaleF32, false>
+                                     : decode_gemm_kernel<1, kScaleF32, false>);
+  const int ki = mx ? 6 : bf ? 3 + parts : (parts - 1) * 2 + (wide ? 1 : 0);
+  static bool configured[64][7] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev][ki]) {

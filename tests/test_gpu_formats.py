@@ -135,6 +135,31 @@ def test_bf16_absmax_odd_row_lengths():
         _check(y, oracle.grouped_gemm_bf16_absmax_f64(x, packed, ab, sizes, experts), "bf16 absmax")
 
 
+# ------------------------------------------ fp32 absmax copy paths
+@pytest.mark.parametrize("epi", [gnf4.GNF4_EPI_NONE, gnf4.GNF4_EPI_SWIGLU])
+def test_fp32_absmax_unaligned_base_matches_aligned(epi):
+    # K % 256 == 0 with a 16-byte aligned absmax takes one 16-byte scale copy
+    # per row and stage; the same absmax 4 bytes past a 16-byte boundary
+    # takes 4-byte copies. Same values, same arithmetic: bit-identical output.
+    E, N, K = 3, 272, 1024
+    rng = np.random.default_rng(77 + epi)
+    packed = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
+    absmax = rng.uniform(0.01, 0.1, size=(E, N, K // 64)).astype(np.float32)
+    sizes, experts = [5, 0, 8, 3], [2, 0, 1, 0]
+    x = synth.activations_bf16(int(sum(sizes)), K, seed=78)
+    aligned = dev(absmax)
+    assert aligned.data_ptr() % 16 == 0
+    buf = torch.zeros(absmax.size + 4, dtype=torch.float32, device="cuda")
+    shifted = buf[1:1 + absmax.size].view(absmax.shape)
+    shifted.copy_(aligned)
+    assert shifted.data_ptr() % 16 == 4
+    ys = [_ex(packed, a, sizes, experts, x=bf16_to_dev(x), epilogue=epi, mode=gnf4.GNF4_MODE_DECODE)
+          for a in (aligned, shifted)]
+    assert torch.equal(ys[0], ys[1])
+    _check(ys[1], _epi_ref(oracle.grouped_gemm_f64(x, packed, absmax, sizes, experts), epi),
+           "fp32 absmax, 4-byte copies")
+
+
 # ------------------------------------------ interleaved clamped SwiGLU
 @pytest.mark.parametrize("E,N,K,sizes,experts", [
     (4, 520, 2880, [3, 0, 12], [3, 1, 0]),
