@@ -288,6 +288,162 @@ __device__ __forceinline__ void store_outputs(uint16_t *y, float alpha, float li
   }
 }
 
+__device__ __forceinline__ Problem make_problem(const DecodeParams &a) {
+  Problem p;
+  p.N = a.N; p.K = a.K; p.E = a.E; p.G = a.G; p.epi = a.epi;
+  p.KB = a.K / 64;
+  p.KC = (p.KB + kStageBlocks - 1) / kStageBlocks;
+  p.upb = a.epi ? (a.N / 2 + 7) / 8 : (a.N + 15) / 16;
+  p.tpb = (p.upb + kTileUnits - 1) / kTileUnits;
+  return p;
+}
+
+// Generic pointer of shared-window address `off`.
+__device__ __forceinline__ char *shared_ptr(uint32_t off) {
+  return static_cast<char *>(__cvta_shared_to_generic(off));
+}
+
+// The suspending part of a bounded wait on the mbarrier at shared address
+// `bar`: the time limit (shortened by a non-zero header word 2, the test
+// hook) and the CTA's abort flag are read here, out of the stage loop.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, WsHeader *hdr) {
+  const uint32_t hook = hdr->reserved[0];
+  const uint64_t limit_ns = hook ? static_cast<uint64_t>(hook) : kTimeoutNs;
+  const uint32_t hint = limit_ns < kWaitHintNs ? static_cast<uint32_t>(limit_ns) : kWaitHintNs;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(shared_ptr(kMiscOff)) + 1;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint)
+        : "memory");
+    if (ok) return true;
+    if (*abort_flag) return false;
+    if (global_timer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      report_error(hdr, GNF4_DEVERR_TIMEOUT, blockIdx.x);
+      return false;
+    }
+  }
+}
+
+// Bounded wait of the whole warp (warp-uniform answer) on the mbarrier at
+// shared address `bar`: one non-suspending try, else the loop above.
+__device__ __forceinline__ bool warp_wait_sa(uint32_t bar, uint32_t parity, WsHeader *hdr) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  if (!ok) ok = wait_slow(bar, parity, hdr) ? 1u : 0u;
+  return __all_sync(0xffffffffu, ok != 0);
+}
+
+// One arrival on the mbarrier at shared address `bar` for the whole
+// (converged) warp, by an elected lane.
+__device__ __forceinline__ void arrive_elect_sa(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+// The end of one tile piece for the calling consumer warp (unit pair up =
+// warp % 4, block blk = warp / 4) with its sums acc0 (unit 2 up) and acc1
+// (unit 2 up + 1) after the ep-th piece of tile t (tl; whole: the piece is
+// the whole tile): block warps 1..3 hand their sums to the pair's block-0
+// warp, which stores the outputs, or, for a piece of a cut tile, leaves its
+// partial sums and counts the piece; the piece that counts last adds all
+// pieces in order and stores. Out of line, with the values it needs
+// recomputed here from shared memory and the parameters, so that they do
+// not stay live across the stage loop. False if a wait gave up.
+__device__ __noinline__ bool finish_piece(const DecodeParams &a, float4 acc0, float4 acc1,
+                                          int64_t t, Tile tl, bool whole, uint32_t ep) {
+  char *smem = shared_ptr(0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int up = warp & 3, blk = warp >> 2, g = lane >> 2, q = lane & 3;
+  const Problem p = make_problem(a);
+  const uint32_t xfull = kBarOff + (3 * kStages + up) * 8;
+  const uint32_t xempty = kBarOff + (3 * kStages + kPairs + up) * 8;
+  float4 *xchg = reinterpret_cast<float4 *>(smem + kXchgOff) + up * 3 * 2 * 32 + lane;
+  float acc[2][4] = {{acc0.x, acc0.y, acc0.z, acc0.w}, {acc1.x, acc1.y, acc1.z, acc1.w}};
+  const bool act1 = 2 * up + 1 < tl.nunits;
+  if (blk != 0) {
+    // hand the partial sums to the pair's block-0 warp
+    if (ep > 0 && !warp_wait_sa(xempty, (ep - 1) & 1u, a.hdr)) return false;
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu)
+      xchg[((blk - 1) * 2 + uu) * 32] = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(reinterpret_cast<uint64_t *>(smem + xfull));
+    return true;
+  }
+  if (!warp_wait_sa(xfull, ep & 1u, a.hdr)) return false;
+#pragma unroll
+  for (int b = 1; b < 4; ++b) {
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu) {
+      const float4 v = xchg[((b - 1) * 2 + uu) * 32];
+      acc[uu][0] += v.x;
+      acc[uu][1] += v.y;
+      acc[uu][2] += v.z;
+      acc[uu][3] += v.w;
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(reinterpret_cast<uint64_t *>(smem + xempty));
+  if (whole) {
+    store_outputs(a.y, a.alpha, a.limit, p, tl, up, g, q, acc, act1);
+    return true;
+  }
+  const int64_t KC = p.KC;
+  const int64_t W = static_cast<int64_t>(reinterpret_cast<const int *>(smem + kMiscOff)[2]) * p.tpb * KC;
+  const int64_t P = min(static_cast<int64_t>(gridDim.x), W);
+  const int64_t b_first = cta_of(W, P, t * KC), b_last = cta_of(W, P, t * KC + KC - 1);
+  // a piece of a cut tile: leave the partial sums, count the piece; the
+  // piece that counts last adds all pieces in order and stores
+  float4 *mine = a.partials + (piece_slot(W, P, KC, t, blockIdx.x) * kPairs + up) * kPartialSlot;
+#pragma unroll
+  for (int uu = 0; uu < 2; ++uu)
+    mine[uu * 32 + lane] = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
+  __syncwarp();
+  uint32_t old = 0;
+  uint32_t *cnt = a.counters + b_first * kPairs + up;
+  if (lane == 0) {
+    __threadfence();
+    old = atomic_add_acq_rel(cnt, 1u);
+  }
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old == static_cast<uint32_t>(b_last - b_first)) {
+    __syncwarp();
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[uu][i] = 0.0f;
+    for (int64_t c = b_first; c <= b_last; ++c) {
+      const float4 *pc = a.partials + (piece_slot(W, P, KC, t, c) * kPairs + up) * kPartialSlot;
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu) {
+        const float4 v = __ldcg(pc + uu * 32 + lane);
+        acc[uu][0] += v.x;
+        acc[uu][1] += v.y;
+        acc[uu][2] += v.z;
+        acc[uu][3] += v.w;
+      }
+    }
+    store_outputs(a.y, a.alpha, a.limit, p, tl, up, g, q, acc, act1);
+    if (lane == 0) *cnt = 0u;   // reusable by the next launch
+  }
+  return true;
+}
+
 // PARTS: fp16 parts per NF4 code value (1 or 2). SK: the scale encoding
 // (kScaleF32, kScaleBf16, or kScaleE8m0 for MXFP4, which is one part).
 // WIDE: fp32 scales whose 4 blocks of a stage are one 16-byte aligned run in
@@ -313,10 +469,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint16_t *const hidden = a.hidden;
   const int32_t *const sorted_idx = a.sorted_idx;
   const int32_t top_k = a.top_k;
-  uint16_t *const yout = a.y;
-  const float alpha = a.alpha, limit = a.limit;
-  float4 *const partials = a.partials;
-  uint32_t *const counters = a.counters;
   // generic pointer of shared-window address 0: smem + kXxxOff is region kXxx
   const uint32_t dyn0 = smem_u32(smem_raw);
   char *smem = smem_raw - dyn0;
@@ -340,19 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *xfull = xready + kStages;          // [kPairs]
   uint64_t *xempty = xfull + kPairs;           // [kPairs]
   uint64_t *never = xempty + kPairs;
-  int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort
+  int *misc = reinterpret_cast<int *>(smem + kMiscOff);   // [0] error bits, [1] abort, [2] batches
   volatile int *abort_flag = &misc[1];
-  __shared__ int s_tot;       // total batches (written by warp 0 with the group table)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();
 
-  Problem p;
-  p.N = a.N; p.K = a.K; p.E = a.E; p.G = a.G; p.epi = a.epi;
-  p.KB = a.K / 64;
-  p.KC = (p.KB + kStageBlocks - 1) / kStageBlocks;
-  p.upb = a.epi ? (a.N / 2 + 7) / 8 : (a.N + 15) / 16;
-  p.tpb = (p.upb + kTileUnits - 1) / kTileUnits;
+  const Problem p = make_problem(a);
   const bool gather = hidden != nullptr;
 
   if (tid == 0) {
@@ -448,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       batch_start[p.G] = static_cast<int>(tot_b);
       row_off[p.G] = static_cast<int>(tot_r);
       if (tot_r != a.M) bad |= GNF4_DEVERR_SIZES;
-      s_tot = static_cast<int>(tot_b);
+      misc[2] = static_cast<int>(tot_b);
       misc[0] = bad;
     }
   }
@@ -458,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && tid == 0) report_error(hdr, static_cast<uint32_t>(errbits), 0);
     return;
   }
-  const int64_t T = static_cast<int64_t>(s_tot) * p.tpb;   // tiles
+  const int64_t T = static_cast<int64_t>(misc[2]) * p.tpb;   // tiles
   const int64_t KC = p.KC;
   const int64_t W = T * KC;                                 // tile-stages
   // CTAs beyond the tile-stage count take nothing, so every range is non-empty
@@ -721,10 +867,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool xswap = MX && (q & 1) != 0;
   const uint32_t lutlane = static_cast<uint32_t>(kLutOff) | (static_cast<uint32_t>(lane) * 4u);
   constexpr bool two_byte = SK != kScaleF32;
-  // partial sums of block warp b (1..3) for unit uu of the pair
-  auto xchg_at = [&](int b, int uu) -> float4 * {
-    return reinterpret_cast<float4 *>(smem + kXchgOff) + ((up * 3 + (b - 1)) * 2 + uu) * 32 + lane;
-  };
   if (hook_ns != 0 && !warp_wait_all(never, 0, abort_flag, hdr, limit_ns)) return;
   uint32_t it = 0, ep = 0;
   for (int64_t s = s_lo; s < s_hi;) {
@@ -733,55 +875,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k1 = static_cast<int>(min(KC, k0 + (s_hi - s)));
     const Tile tl = make_tile(t, p, batch_start, row_off, gexp);
     const bool act0 = 2 * up < tl.nunits, act1 = 2 * up + 1 < tl.nunits;
-    const int64_t ebase = static_cast<int64_t>(tl.e) * p.N;
+    // Two-byte scales: bit 2 uu + r is set if row group r of unit uu finds
+    // its 2 bytes in the high half of the copied word (odd element index;
+    // the element index of (row, block kc * 4 + blk) has the parity of
+    // row * KB + blk).
+    uint32_t hsel = 0;
+    if (two_byte) {
+      const int64_t ebase = static_cast<int64_t>(tl.e) * p.N;
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu) {
+        const int64_t j = tl.j0 + 2 * up + uu;
+        const int64_t w0 = p.epi == 0 ? ebase + 16 * j + g
+                           : (p.epi == 1 ? ebase + 8 * j + g : ebase + 2 * (8 * j + g));
+        const int64_t w1 = p.epi == 0 ? w0 + 8 : (p.epi == 1 ? w0 + p.N / 2 : w0 + 1);
+        hsel |= static_cast<uint32_t>((w0 * p.KB + blk) & 1) << (2 * uu);
+        hsel |= static_cast<uint32_t>((w1 * p.KB + blk) & 1) << (2 * uu + 1);
+      }
+    }
     // C fragment: [0] weight row g, activation row 2q; [1] row g, 2q + 1;
     // [2] row g + 8 (SwiGLU: the matching up row), 2q; [3] row g + 8, 2q + 1
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     for (int kc = k0; kc < k1; ++kc, ++it) {
       const int st = static_cast<int>(it % kStages);
       const uint32_t ph = (it / kStages) & 1u;
-      // the activation warp arrives on xready only after it has observed
+      // the activation warps arrive on xready only after they have observed
       // this stage's copies complete (full), so this one wait also orders
       // the copied weights and scales before the reads below
-      if (!warp_wait_all(&xready[st], ph, abort_flag, hdr, limit_ns)) return;
+      if (!warp_wait_sa(kBarOff + (2 * kStages + st) * 8, ph, a.hdr)) return;
       if (act0) {
         // A block past K reads zero-filled activations and scales: it adds 0.
-        const char *wst = smem + kWOff + st * kWStage;
+        // (Shared-window addresses: region kXxx starts at address kXxx.)
+        const uint32_t wst = kWOff + st * kWStage;
         // 2^-S of activation rows 2q and 2q + 1 in this block
-        const float2 xs = reinterpret_cast<const float2 *>(smem + kXsOff + st * kXsStage)[blk * 4 + q];
-        const char *ast = smem + kAOff + st * kAStage + g * 16 + blk * 4;
+        const float2 xs = lds_f2(kXsOff + st * kXsStage + (blk * 4 + q) * 8);
+        const uint32_t ast = kAOff + st * kAStage + g * 16 + blk * 4;
         // (rows past the batch feed only outputs that are never stored)
-        const char *xst = smem + kXOff + st * kXStage;
-        const uint4 xf = *reinterpret_cast<const uint4 *>(xst + xoffF);
-        const uint4 xg = *reinterpret_cast<const uint4 *>(xst + xoffG);
+        const uint32_t xst = kXOff + st * kXStage;
+        const uint4 xf = lds_u4(xst + xoffF);
+        const uint4 xg = lds_u4(xst + xoffG);
         const uint4 xa = xswap ? xg : xf;   // chunk cA
         const uint4 xb = xswap ? xf : xg;   // chunk cB
-        const int kb = kc * kStageBlocks + blk;
 #pragma unroll
         for (int uu = 0; uu < 2; ++uu) {
           if (uu == 1 && !act1) break;
           const int ui = 2 * up + uu;
           // weight rows g and g + 8 of the unit (1 KB boxes of 8 rows)
-          const char *r0 = wst + (p.epi ? ui : 2 * ui) * kBoxBytes;
-          const char *r1 = wst + (p.epi ? kTileUnits + ui : 2 * ui + 1) * kBoxBytes;
-          const uint32_t wa0 = *reinterpret_cast<const uint32_t *>(r0 + offA);
-          const uint32_t wb0 = *reinterpret_cast<const uint32_t *>(r0 + offB);
-          const uint32_t wa1 = *reinterpret_cast<const uint32_t *>(r1 + offA);
-          const uint32_t wb1 = *reinterpret_cast<const uint32_t *>(r1 + offB);
+          const uint32_t r0 = wst + (p.epi ? ui : 2 * ui) * kBoxBytes;
+          const uint32_t r1 = wst + (p.epi ? kTileUnits + ui : 2 * ui + 1) * kBoxBytes;
+          const uint32_t wa0 = lds_u32(r0 + offA);
+          const uint32_t wb0 = lds_u32(r0 + offB);
+          const uint32_t wa1 = lds_u32(r1 + offA);
+          const uint32_t wb1 = lds_u32(r1 + offB);
           // scale words of rows g and g + 8 (row groups 0 and 1)
-          uint32_t s0 = *reinterpret_cast<const uint32_t *>(ast + ui * 256);
-          uint32_t s1 = *reinterpret_cast<const uint32_t *>(ast + ui * 256 + 128);
+          uint32_t s0 = lds_u32(ast + ui * 256);
+          uint32_t s1 = lds_u32(ast + ui * 256 + 128);
           // the 2 scale bytes of (row, block) sit in the low or the high half
           // of the copied 4-byte word, as the element index is even or odd
           if (two_byte) {
-            const int64_t j = tl.j0 + ui;
-            const int64_t w0 = p.epi == 0 ? ebase + 16 * j + g
-                               : (p.epi == 1 ? ebase + 8 * j + g : ebase + 2 * (8 * j + g));
-            const int64_t w1 = p.epi == 0 ? w0 + 8 : (p.epi == 1 ? w0 + p.N / 2 : w0 + 1);
-            const uint32_t h0 = static_cast<uint32_t>((w0 * p.KB + kb) & 1);
-            const uint32_t h1 = static_cast<uint32_t>((w1 * p.KB + kb) & 1);
-            s0 = (s0 >> (16 * h0)) & 0xFFFFu;
-            s1 = (s1 >> (16 * h1)) & 0xFFFFu;
+            s0 = (s0 >> (16 * ((hsel >> (2 * uu)) & 1u))) & 0xFFFFu;
+            s1 = (s1 >> (16 * ((hsel >> (2 * uu + 1)) & 1u))) & 0xFFFFu;
           }
           // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
           // then (2, 3) of each word; activation registers in the same order.
@@ -831,72 +983,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      mbar_arrive_elect(&empty[st]);
+      arrive_elect_sa(kBarOff + (kStages + st) * 8);
     }
     if (act0) {
-      if (blk != 0) {
-        // hand the partial sums to the pair's block-0 warp
-        if (ep > 0 && !warp_wait_one(&xempty[up], (ep - 1) & 1u, abort_flag, hdr, limit_ns)) return;
-#pragma unroll
-        for (int uu = 0; uu < 2; ++uu)
-          *xchg_at(blk, uu) = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xfull[up]);
-      } else {
-        if (!warp_wait_one(&xfull[up], ep & 1u, abort_flag, hdr, limit_ns)) return;
-#pragma unroll
-        for (int b = 1; b < 4; ++b) {
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu) {
-            const float4 v = *xchg_at(b, uu);
-            acc[uu][0] += v.x;
-            acc[uu][1] += v.y;
-            acc[uu][2] += v.z;
-            acc[uu][3] += v.w;
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xempty[up]);
-        const int64_t b_first = cta_of(W, P, t * KC), b_last = cta_of(W, P, t * KC + KC - 1);
-        if (b_first == b_last) {
-          store_outputs(yout, alpha, limit, p, tl, up, g, q, acc, act1);
-        } else {
-          // a piece of a cut tile: leave the partial sums, count the piece;
-          // the piece that counts last adds all pieces in order and stores
-          float4 *mine = partials + (piece_slot(W, P, KC, t, blockIdx.x) * kPairs + up) * kPartialSlot;
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu)
-            mine[uu * 32 + lane] = make_float4(acc[uu][0], acc[uu][1], acc[uu][2], acc[uu][3]);
-          __syncwarp();
-          uint32_t old = 0;
-          uint32_t *cnt = counters + b_first * kPairs + up;
-          if (lane == 0) {
-            __threadfence();
-            old = atomic_add_acq_rel(cnt, 1u);
-          }
-          old = __shfl_sync(0xffffffffu, old, 0);
-          if (old == static_cast<uint32_t>(b_last - b_first)) {
-            __syncwarp();
-#pragma unroll
-            for (int uu = 0; uu < 2; ++uu)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) acc[uu][i] = 0.0f;
-            for (int64_t c = b_first; c <= b_last; ++c) {
-              const float4 *pc = partials + (piece_slot(W, P, KC, t, c) * kPairs + up) * kPartialSlot;
-#pragma unroll
-              for (int uu = 0; uu < 2; ++uu) {
-                const float4 v = __ldcg(pc + uu * 32 + lane);
-                acc[uu][0] += v.x;
-                acc[uu][1] += v.y;
-                acc[uu][2] += v.z;
-                acc[uu][3] += v.w;
-              }
-            }
-            store_outputs(yout, alpha, limit, p, tl, up, g, q, acc, act1);
-            if (lane == 0) *cnt = 0u;   // reusable by the next launch
-          }
-        }
-      }
+      if (!finish_piece(a, make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]),
+                        make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]), t, tl,
+                        k0 == 0 && k1 == KC, ep))
+        return;
       ++ep;
     }
     s += k1 - k0;
