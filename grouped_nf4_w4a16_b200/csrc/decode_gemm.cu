@@ -288,6 +288,14 @@ __device__ __forceinline__ void store_outputs(uint16_t *y, float alpha, float li
   }
 }
 
+// The next stage slot of the ring; its phase parity flips when the slot wraps.
+__device__ __forceinline__ void next_stage(int &st, uint32_t &ph) {
+  if (++st == kStages) {
+    st = 0;
+    ph ^= 1u;
+  }
+}
+
 __device__ __forceinline__ Problem make_problem(const DecodeParams &a) {
   Problem p;
   p.N = a.N; p.K = a.K; p.E = a.E; p.G = a.G; p.epi = a.epi;
@@ -624,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kChunks = 8 / kXWarps;
     const int xi = (warp - kXWarp0) * 32 + lane;
     const int h = xi % kXWarps, b = (xi / kXWarps) >> 3, r = (xi / kXWarps) & 7;
-    uint32_t it = 0;
+    int st = 0;          // stage slot and its phase parity, advanced per stage
+    uint32_t ph = 0;
     for (int64_t s = s_lo; s < s_hi;) {
       const int64_t t = div_fast(s, KC);
       const int k0 = static_cast<int>(s - t * KC);
@@ -633,9 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // rows past the batch feed only outputs that are never stored: skipped
       const bool live = r < tl.mrows;
       const uint32_t pair_mask = __ballot_sync(0xffffffffu, live);
-      for (int kc = k0; kc < k1; ++kc, ++it) {
-        const int st = static_cast<int>(it % kStages);
-        const uint32_t ph = (it / kStages) & 1u;
+      for (int kc = k0; kc < k1; ++kc, next_stage(st, ph)) {
         if (!warp_wait_one(&full[st], ph, abort_flag, hdr, limit_ns)) return;
         if (live) {
           char *row = smem + kXOff + st * kXStage + b * kBoxBytes + r * 128;
@@ -731,10 +738,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t e00 = wrow(0, 0, r) * p.KB + blk;
       const int64_t du = (wrow(1, 0, r) - wrow(0, 0, r)) * p.KB;
       const int64_t dg = (wrow(0, 1, r) - wrow(0, 0, r)) * p.KB;
-      for (int i = 0; i < tl.nunits; ++i)
+      if (scale_warp)
+        for (int i = 0; i < tl.nunits; ++i)
 #pragma unroll
-        for (int rgi = 0; rgi < 2; ++rgi)
-          if (wrow(i, rgi, r) < ebase + p.N) vmask |= 1u << (2 * i + rgi);
+          for (int rgi = 0; rgi < 2; ++rgi)
+            if (wrow(i, rgi, r) < ebase + p.N) vmask |= 1u << (2 * i + rgi);
       if (scale_warp && gather && gr < tl.mrows) {
         const int32_t slot = sorted_idx[tl.row0 + gr];   // checked in range up front
         hrow = hidden + static_cast<int64_t>(slot / top_k) * p.K;
@@ -868,7 +876,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lutlane = static_cast<uint32_t>(kLutOff) | (static_cast<uint32_t>(lane) * 4u);
   constexpr bool two_byte = SK != kScaleF32;
   if (hook_ns != 0 && !warp_wait_all(never, 0, abort_flag, hdr, limit_ns)) return;
-  uint32_t it = 0, ep = 0;
+  int st = 0;            // stage slot and its phase parity, advanced per stage
+  uint32_t ph = 0, ep = 0;
   for (int64_t s = s_lo; s < s_hi;) {
     const int64_t t = div_fast(s, KC);
     const int k0 = static_cast<int>(s - t * KC);
@@ -895,9 +904,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // C fragment: [0] weight row g, activation row 2q; [1] row g, 2q + 1;
     // [2] row g + 8 (SwiGLU: the matching up row), 2q; [3] row g + 8, 2q + 1
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    for (int kc = k0; kc < k1; ++kc, ++it) {
-      const int st = static_cast<int>(it % kStages);
-      const uint32_t ph = (it / kStages) & 1u;
+    for (int kc = k0; kc < k1; ++kc, next_stage(st, ph)) {
       // the activation warps arrive on xready only after they have observed
       // this stage's copies complete (full), so this one wait also orders
       // the copied weights and scales before the reads below
