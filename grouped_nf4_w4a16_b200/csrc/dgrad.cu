@@ -467,13 +467,17 @@ cudaError_t launch_grouped_dgrad(const uint16_t *dy, const uint8_t *w, const flo
                                  int64_t M, int32_t N, int32_t K, int32_t E, uint16_t *dx,
                                  WsHeader *hdr, cudaStream_t stream) {
   if (N % 8 != 0 || static_cast<int64_t>(E) * N + kDgRows >= INT_MAX) return cudaErrorNotSupported;
-  // packed weights as [E*N rows][K/2 bytes], boxes of 256 rows x 32 bytes
+  // packed weights as [E*N rows][K/2 bytes], boxes of 256 rows x 32 bytes.
+  // Each 32-byte row piece is fetched into L2 as 64 bytes: the neighbouring
+  // 64-element block is the next tile's, read a tile (KC stages) later,
+  // while 256-byte fetches were mostly evicted before their other 7 blocks
+  // were used (5x the weight bytes from DRAM).
   CUtensorMap wmap;
   if (!encode_tensor_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, w,
                             static_cast<uint64_t>(K / 2),
                             static_cast<uint64_t>(E) * static_cast<uint64_t>(N),
                             static_cast<uint64_t>(K / 2), 32, kDgRows,
-                            CU_TENSOR_MAP_SWIZZLE_NONE))
+                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_64B))
     return cudaErrorInvalidValue;
   DgradParams prm;
   prm.dy = dy;

@@ -149,20 +149,24 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 
 // ------------------------------------------------------------ host side
 // Encodes a tiled tensor map of rank 2 to 5: dims[0] is the contiguous
-// dimension, pitches[i] the byte stride of dims[i + 1]. Returns false if the
-// driver refuses it.
+// dimension, pitches[i] the byte stride of dims[i + 1]. `promotion` is the
+// L2 fetch size of each access (256 bytes unless a narrow box's neighbours
+// would be evicted before they are used). Returns false if the driver
+// refuses it.
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,
                        const uint64_t *dims, const uint64_t *pitches, const uint32_t *box,
-                       CUtensorMapSwizzle swizzle);
+                       CUtensorMapSwizzle swizzle,
+                       CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 
 // 2-D row-major tensor [rows][cols] (row pitch in bytes).
-inline bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
-                                 uint64_t cols, uint64_t rows, uint64_t row_pitch_bytes,
-                                 uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+inline bool encode_tensor_map_2d(
+    CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t cols, uint64_t rows,
+    uint64_t row_pitch_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle,
+    CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
   const uint64_t dims[2] = {cols, rows};
   const uint64_t pitches[1] = {row_pitch_bytes};
   const uint32_t box[2] = {box_cols, box_rows};
-  return encode_tensor_map(map, dtype, 2, base, dims, pitches, box, swizzle);
+  return encode_tensor_map(map, dtype, 2, base, dims, pitches, box, swizzle, promotion);
 }
 
 }  // namespace gnf4

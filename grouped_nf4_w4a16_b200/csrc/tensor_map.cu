@@ -22,7 +22,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,
                        const uint64_t *dims, const uint64_t *pitches, const uint32_t *box,
-                       CUtensorMapSwizzle swizzle) {
+                       CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promotion) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (encode == nullptr || rank < 2 || rank > 5) return false;
   cuuint64_t d[5], st[4];
@@ -34,8 +34,8 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, co
   }
   for (int i = 0; i + 1 < rank; ++i) st[i] = static_cast<cuuint64_t>(pitches[i]);
   const CUresult r = encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d,
-                            st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                            st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promotion,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
