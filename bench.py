@@ -517,40 +517,68 @@ def time_glue(prob, stream, reps=50):
 
 
 def run_e2e(prob, stream, steps):
+    """The step through the public entry points with host inputs and
+    outputs: every step copies its inputs in from pinned host memory and its
+    results out to pinned host memory. Pipelined as a serving loop runs it:
+    step i's inputs are copied in (one copy stream) and step i-1's results
+    copied out (another) while step i-1 / i computes, over two sets of device
+    buffers; the timed region runs from the first copy in to the last copy
+    out."""
     gnf4 = prob.gnf4
     dev = prob.topk.device
     h_topk = torch.from_numpy(prob.topk_np).pin_memory()
     h_x = [torch.from_numpy(d["x_np"].view(np.int16)).pin_memory() for d in prob.gemms]
     h_y = [torch.empty(d["y"].shape, dtype=torch.int16).pin_memory() for d in prob.gemms]
-    d_topk = torch.empty_like(prob.topk)
-    d_x = [torch.empty(d["x"].shape, dtype=torch.int16, device=dev) for d in prob.gemms]
+    nbuf = 2
+    d_topk = [torch.empty_like(prob.topk) for _ in range(nbuf)]
+    d_x = [[torch.empty(d["x"].shape, dtype=torch.int16, device=dev) for d in prob.gemms]
+           for _ in range(nbuf)]
+    d_y = [[torch.empty_like(d["y"]) for d in prob.gemms] for _ in range(nbuf)]
     h2d = h_topk.numel() * 4 + sum(t.numel() * 2 for t in h_x)
     d2h = sum(t.numel() * 2 for t in h_y)
+    copy_in = torch.cuda.Stream(device=dev)
+    copy_out = torch.cuda.Stream(device=dev)
+    in_ready = [torch.cuda.Event() for _ in range(nbuf)]
+    computed = [torch.cuda.Event() for _ in range(nbuf)]
+    out_done = [torch.cuda.Event() for _ in range(nbuf)]
 
-    def one(r):
-        d_topk.copy_(h_topk, non_blocking=True)
-        for a, b in zip(d_x, h_x):
-            a.copy_(b, non_blocking=True)
-        gnf4.gnf4_moe_align(d_topk, prob.w.E, sorted_idx=prob.sorted_idx, sizes=prob.sizes,
-                            expert_ids=prob.expert_ids, num_groups=prob.num_groups,
-                            workspace=prob.ws_align)
-        for i, d in enumerate(prob.gemms):
-            gnf4.gnf4_grouped_gemm(d_x[i].view(torch.bfloat16), d["W"][r], d["A"][r], prob.sizes,
-                                   prob.expert_ids, epilogue=d["epi"], y=d["y"],
-                                   workspace=d["ws"])
-            h_y[i].copy_(d["y"].view(torch.int16), non_blocking=True)
+    def one(i, r):
+        j = i % nbuf
+        with torch.cuda.stream(copy_in):
+            if i >= nbuf:
+                copy_in.wait_event(computed[j])     # buffer j's inputs read by step i - 2
+            d_topk[j].copy_(h_topk, non_blocking=True)
+            for a, b in zip(d_x[j], h_x):
+                a.copy_(b, non_blocking=True)
+            in_ready[j].record(copy_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(in_ready[j])
+            if i >= nbuf:
+                stream.wait_event(out_done[j])      # buffer j's results copied out by step i - 2
+            gnf4.gnf4_moe_align(d_topk[j], prob.w.E, sorted_idx=prob.sorted_idx,
+                                sizes=prob.sizes, expert_ids=prob.expert_ids,
+                                num_groups=prob.num_groups, workspace=prob.ws_align)
+            for k, d in enumerate(prob.gemms):
+                gnf4.gnf4_grouped_gemm(d_x[j][k].view(torch.bfloat16), d["W"][r], d["A"][r],
+                                       prob.sizes, prob.expert_ids, epilogue=d["epi"],
+                                       y=d_y[j][k], workspace=d["ws"])
+            computed[j].record(stream)
+        with torch.cuda.stream(copy_out):
+            copy_out.wait_event(computed[j])
+            for k in range(len(prob.gemms)):
+                h_y[k].copy_(d_y[j][k].view(torch.int16), non_blocking=True)
+            out_done[j].record(copy_out)
 
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            one(i % prob.R)
-    stream.synchronize()
+    for i in range(3):
+        one(i, i % prob.R)
+    torch.cuda.synchronize(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    with torch.cuda.stream(stream):
-        for i in range(steps):
-            one(i % prob.R)
-    b.record(stream)
+    a.record(copy_in)
+    for i in range(steps):
+        one(i, i % prob.R)
+    b.record(copy_out)
     b.synchronize()
+    torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / steps
     return ms, h2d, d2h, steps
 
@@ -737,7 +765,10 @@ def main():
         "glue": glue,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "how": "eager C-ABI calls; pinned host inputs copied in and results copied out every step"},
+                "how": ("eager C-ABI calls; every step copies its inputs in from pinned host memory and "
+                        "its results out to pinned host memory, pipelined: copies in and out on two "
+                        "copy streams overlap the previous / next step's compute over two sets of "
+                        "device buffers")},
         "gpu_launches": kpl * args.steps if kpl is not None else None,
         "step_kernels": res["step_kernels"],
         "timing": ("each step is one CUDA graph of the C-ABI calls (moe_align, then each GEMM); "
