@@ -32,19 +32,22 @@
 //
 // Formats and numerics (per stage, each consumer lane decodes packed bytes
 // through a byte-indexed table replicated per lane, so no lookup conflicts)
-//   NF4:   code value NF4[c] carried as its fp16 rounding hi; with a fused
-//          SwiGLU also the fp16 of the remainder times 2^13 (two MMAs), which
-//          together are within 1e-7 relative of the fp32 value (SwiGLU
-//          multiplies a gate error by the up value, so the gate_up GEMM of a
-//          SwiGLU layer keeps both parts). The scale is the fp32 (or bf16)
-//          absmax of the 64-element block, applied to the block's fp32 sum.
+//   NF4:   code value NF4[c] carried as hi = fp16(NF4[c] * kTableScale), one
+//          MMA per 16 K-elements; the block sum is multiplied by
+//          1 / kTableScale (see kTableScale). With a fused SwiGLU the up rows
+//          also carry the remainder (NF4[c] * kTableScale - hi) * 2^13 as fp16
+//          in a second MMA (gate rows 0 there): SwiGLU multiplies an up error
+//          by silu(gate), which a near-zero up value leaves unbounded by the
+//          relative tolerance, while a one-part gate stays well inside it.
+//          The scale is the fp32 (or bf16) absmax of the 64-element block,
+//          applied to the block's fp32 sum.
 //   MXFP4: e2m1 code values are exact in fp16 (one MMA); the e8m0 scale of
 //          each 32-element half-block is applied to its fp32 sum.
 //   Activations are staged as bf16 and rewritten in place as fp16 times a
 //   power of two per (row, 64-element block), which the block sum divides out.
 //
-// Inside a CTA (warp 16 = tensor copies, warp 17 = scale copies and, when the
-// activations are gathered, their row copies, warp 18 = activation conversion,
+// Inside a CTA (warp 16 = tensor copies; warps 17-19 = scale copies and, when
+// the activations are gathered, their row copies, or activation conversion;
 // warps 0-15 = consumers)
 //   Consumer warp w takes 64-element block w / 4 of every stage for the two
 //   units 2 (w % 4), 2 (w % 4) + 1; when a tile piece ends, the four block
@@ -89,7 +92,6 @@ constexpr int kXStage = kStageBlocks * kBoxBytes;                // 4 KB
 constexpr int kXsStage = kStageBlocks * kBatch * 4;              // 128 B: 2^-S per (block, row)
 constexpr int kAStage = kTileUnits * 2 * 8 * kStageBlocks * 4;   // 2 KB of scale words
 constexpr int kMaxG = GNF4_MAX_EXPERTS;
-constexpr float kLoInv = 1.0f / 8192.0f;      // remainders are carried times 2^13
 constexpr int kPairs = kTileUnits / 2;        // unit pairs per tile
 constexpr int kPartialSlot = 2 * 32;          // float4 per (pair) partial: 2 units x 32 lanes
 
@@ -126,6 +128,15 @@ constexpr int kSmemBytes = kSmemEnd - kMinDyn;
 static_assert(kMiscOff + 8 * 4 <= kLutOff, "low region overlaps the table");
 static_assert(kBarOff % 8 == 0 && kXOff % 1024 == 0 && kLutOff % 65536 == 0, "alignment");
 static_assert(kSmemBytes + kDynBase - kMinDyn <= 227 * 1024, "fits one CTA per SM");
+
+// NF4 code values enter the MMAs as fp16(NF4[c] * kTableScale). Of the
+// scales in [1, 2) (searched on a 5e-7 grid) this one gives the smallest
+// largest rounding error over the 16 values: 6.0e-5 of the code range,
+// against 1.9e-4 for the plain fp16 rounding. The consumers' per-block
+// factor 2^-S carries the 1 / kTableScale back.
+constexpr float kTableScale = 1.6776540f;
+constexpr float kTableInv = 1.0f / kTableScale;
+constexpr float kLoInv = 1.0f / 8192.0f;      // up-row remainders are carried times 2^13
 
 // Scale encodings of the stack (GemmArgs::scale_kind).
 constexpr int kScaleF32 = 0;    // NF4 absmax, fp32
@@ -452,11 +463,11 @@ __device__ __noinline__ bool finish_piece(const DecodeParams &a, float4 acc0, fl
   return true;
 }
 
-// PARTS: fp16 parts per NF4 code value (1 or 2). SK: the scale encoding
-// (kScaleF32, kScaleBf16, or kScaleE8m0 for MXFP4, which is one part).
+// SK: the scale encoding (kScaleF32, kScaleBf16, or kScaleE8m0 for MXFP4).
+// UPLO: the up rows of a SwiGLU unit also carry the code remainders (NF4).
 // WIDE: fp32 scales whose 4 blocks of a stage are one 16-byte aligned run in
 // every row (K % 256 == 0, scales 16-byte aligned), copied 16 bytes at a time.
-template <int PARTS, int SK, bool WIDE>
+template <int SK, bool WIDE, bool UPLO>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gemm_kernel(const __grid_constant__ WeightMaps wmaps,
                        const __grid_constant__ CUtensorMap xmap,
@@ -531,21 +542,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- decode table: row b, lane slot l: the fp16 pair of byte b's two code
-  //      values (low half = even k) at l * 4 and (NF4 with two parts) the pair
-  //      of remainders at 128 + l * 4. NF4 puts even k in the high nibble,
-  //      MXFP4 in the low nibble.
+  //      values (low half = even k) at l * 4 and (UPLO) the pair of their
+  //      remainders at 128 + l * 4. NF4 puts even k in the high nibble, MXFP4
+  //      in the low nibble.
   for (int i = tid; i < 256 * 8; i += kThreads) {
     const int b = i >> 3, part = i & 7;
-    uint32_t hp, lp = 0u;
-    if (MX) {
-      hp = half_bits(e2m1_value(b & 15)) | (half_bits(e2m1_value(b >> 4)) << 16);
-    } else {
-      hp = code_hi(b >> 4) | (code_hi(b & 15) << 16);
-      if (PARTS == 2) lp = code_lo(b >> 4) | (code_lo(b & 15) << 16);
+    const uint32_t hp =
+        MX ? half_bits(e2m1_value(b & 15)) | (half_bits(e2m1_value(b >> 4)) << 16)
+           : half_bits(nf4_value(b >> 4) * kTableScale) |
+                 (half_bits(nf4_value(b & 15) * kTableScale) << 16);
+    uint4 *row = reinterpret_cast<uint4 *>(smem + kLutOff + b * 256);
+    row[part] = make_uint4(hp, hp, hp, hp);
+    if (UPLO) {
+      // remainder of the scaled value: exact in fp32, at most 2^-11 of it
+      const float v0 = nf4_value(b >> 4) * kTableScale, v1 = nf4_value(b & 15) * kTableScale;
+      const uint32_t lp = half_bits((v0 - __half2float(__ushort_as_half(hp & 0xFFFFu))) * 8192.0f) |
+                          (half_bits((v1 - __half2float(__ushort_as_half(hp >> 16))) * 8192.0f) << 16);
+      row[8 + part] = make_uint4(lp, lp, lp, lp);
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(smem + kLutOff + b * 256);
-    dst[part] = make_uint4(hp, hp, hp, hp);
-    if (PARTS == 2) dst[8 + part] = make_uint4(lp, lp, lp, lp);
   }
 
   pdl_wait();   // inputs may come from the previous kernel on the stream
@@ -626,8 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Per stage, each (block b, row r) of the staged bf16 activations is
     // rewritten in place as fp16 x * 2^S, S putting the largest magnitude of
     // its 64 values in [2^14, 2^15) (0 for all zeros, Inf or NaN): exact for
-    // every value above 2^-28 of that maximum. 2^-S goes to the stage's
-    // scale table for the consumers' block sums. The kXWarps lanes of one
+    // every value above 2^-28 of that maximum. 2^-S (NF4: times
+    // 1 / kTableScale, one fp32 rounding) goes to the stage's scale table for
+    // the consumers' block sums. The kXWarps lanes of one
     // (block, row) take 8 / kXWarps of its 16-byte chunks each.
     constexpr int kChunks = 8 / kXWarps;
     const int xi = (warp - kXWarp0) * 32 + lane;
@@ -680,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (h == 0)
             reinterpret_cast<float *>(smem + kXsOff + st * kXsStage)[b * 8 + r] =
-                __uint_as_float(static_cast<uint32_t>(127 - S) << 23);
+                __uint_as_float(static_cast<uint32_t>(127 - S) << 23) * (MX ? 1.0f : kTableInv);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&xready[st]);
@@ -944,11 +959,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // MMA k pairs (2q, 2q+1) and (2q+8, 2q+9) <- packed bytes (0, 1)
           // then (2, 3) of each word; activation registers in the same order.
+          // (UPLO: rows g + 8, the up rows, with their remainders)
           uint32_t ha0[4], la0[4], ha1[4], la1[4], hb0[4], lb0[4], hb1[4], lb1[4];
-          decode_word<PARTS>(lutlane, wa0, ha0, la0);
-          decode_word<PARTS>(lutlane, wa1, ha1, la1);
-          decode_word<PARTS>(lutlane, wb0, hb0, lb0);
-          decode_word<PARTS>(lutlane, wb1, hb1, lb1);
+          decode_word<1>(lutlane, wa0, ha0, la0);
+          decode_word<UPLO ? 2 : 1>(lutlane, wa1, ha1, la1);
+          decode_word<1>(lutlane, wb0, hb0, lb0);
+          decode_word<UPLO ? 2 : 1>(lutlane, wb1, hb1, lb1);
           if (MX) {
             // the two 32-element halves separately, each times its e8m0
             // scale (byte 0 of the pair: first half, byte 1: second half)
@@ -969,14 +985,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16(ch, ha0[2], ha1[2], ha0[3], ha1[3], xa.z, xa.w);
             mma_f16(ch, hb0[0], hb1[0], hb0[1], hb1[1], xb.x, xb.y);
             mma_f16(ch, hb0[2], hb1[2], hb0[3], hb1[3], xb.z, xb.w);
-            if (PARTS == 2) {
+            if (UPLO) {   // the up rows' remainders (gate rows' operands 0)
               float cl[4];
-              mma_f16_z(cl, la0[0], la1[0], la0[1], la1[1], xa.x, xa.y);
-              mma_f16(cl, la0[2], la1[2], la0[3], la1[3], xa.z, xa.w);
-              mma_f16(cl, lb0[0], lb1[0], lb0[1], lb1[1], xb.x, xb.y);
-              mma_f16(cl, lb0[2], lb1[2], lb0[3], lb1[3], xb.z, xb.w);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) ch[i] = fmaf(cl[i], kLoInv, ch[i]);
+              mma_f16_z(cl, 0u, la1[0], 0u, la1[1], xa.x, xa.y);
+              mma_f16(cl, 0u, la1[2], 0u, la1[3], xa.z, xa.w);
+              mma_f16(cl, 0u, lb1[0], 0u, lb1[1], xb.x, xb.y);
+              mma_f16(cl, 0u, lb1[2], 0u, lb1[3], xb.z, xb.w);
+              ch[2] = fmaf(cl[2], kLoInv, ch[2]);
+              ch[3] = fmaf(cl[3], kLoInv, ch[3]);
             }
             // absmax of rows g and g + 8 (fp32, or bf16 widened exactly)
             const float am0 = __uint_as_float(two_byte ? s0 << 16 : s0);
@@ -1021,7 +1037,6 @@ size_t decode_zero_prefix_bytes(int64_t M, int32_t N, int32_t G, int32_t swiglu)
 cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   if (static_cast<int64_t>(a.E) * a.N + a.N + 256 >= INT_MAX) return cudaErrorNotSupported;
   const bool mx = a.fmt == GNF4_FMT_MXFP4;
-  const int parts = (!mx && a.epi != GNF4_EPI_NONE) ? 2 : 1;
   WeightMaps wm;
   std::memset(&wm, 0, sizeof(wm));
   // packed weights as [E*N rows][K/2 bytes], boxes of (8 << i) rows x 128 bytes
@@ -1083,14 +1098,16 @@ cudaError_t launch_decode_gemm(const GemmArgs &a, cudaStream_t stream) {
   // run in every row
   const bool wide = !mx && !bf && (a.K / 64) % kStageBlocks == 0 &&
                     reinterpret_cast<uintptr_t>(a.scales) % 16 == 0;
-  auto kernel = mx ? decode_gemm_kernel<1, kScaleE8m0, false>
-                : bf ? (parts == 2 ? decode_gemm_kernel<2, kScaleBf16, false>
-                                   : decode_gemm_kernel<1, kScaleBf16, false>)
-                : wide ? (parts == 2 ? decode_gemm_kernel<2, kScaleF32, true>
-                                     : decode_gemm_kernel<1, kScaleF32, true>)
-                       : (parts == 2 ? decode_gemm_kernel<2, kScaleF32, false>
-                                     : decode_gemm_kernel<1, kScaleF32, false>);
-  const int ki = mx ? 6 : bf ? 3 + parts : (parts - 1) * 2 + (wide ? 1 : 0);
+  // SwiGLU (NF4): the up rows carry their code remainders
+  const bool uplo = !mx && a.epi != GNF4_EPI_NONE;
+  auto kernel = mx     ? decode_gemm_kernel<kScaleE8m0, false, false>
+                : bf   ? (uplo ? decode_gemm_kernel<kScaleBf16, false, true>
+                               : decode_gemm_kernel<kScaleBf16, false, false>)
+                : wide ? (uplo ? decode_gemm_kernel<kScaleF32, true, true>
+                               : decode_gemm_kernel<kScaleF32, true, false>)
+                       : (uplo ? decode_gemm_kernel<kScaleF32, false, true>
+                               : decode_gemm_kernel<kScaleF32, false, false>);
+  const int ki = mx ? 6 : (bf ? 4 : wide ? 2 : 0) + (uplo ? 1 : 0);
   static bool configured[64][7] = {};
   int dev = 0;
   cudaGetDevice(&dev);
