@@ -193,14 +193,15 @@ GNF4_API gnf4_status gnf4_moe_align(const int32_t *topk_ids, int64_t T, int32_t 
  *               again before reusing it. Two calls that may run
  *               concurrently need separate workspaces.
  * Numerics: every product enters an fp32 accumulator. DECODE carries each
- *   code value as its fp16 rounding (relative error at most 2^-12; the
- *   elementwise tolerance above holds with margin on the shapes in scope)
- *   and, with a fused SwiGLU (which multiplies a gate error by the up
- *   value), also the fp16 of the remainder (scaled by 2^13), together
- *   within 1e-7 relative of the fp32 table value; x per row and 64-element
- *   block is scaled by a power of two into fp16 (exact for every element
- *   above 2^-28 of that block's largest magnitude); each block sum is
- *   scaled by absmax and the power of two in fp32. DECODE's stream-K split
+ *   NF4 code value as hi = fp16(NF4[code] * 1.677654), a scale that keeps
+ *   the rounding error of every value within 6.0e-5 (the elementwise
+ *   tolerance above holds with margin on the shapes in scope); with a
+ *   fused SwiGLU (which multiplies an up error by silu(gate)) the up rows
+ *   also carry the fp16 of the remainder (scaled by 2^13), together within
+ *   2^-21 relative of the scaled value; x per row and 64-element block is
+ *   scaled by a power of two into fp16 (exact for every element above
+ *   2^-28 of that block's largest magnitude); each block sum is scaled by
+ *   absmax, the power of two and 1 / 1.677654 in fp32. DECODE's stream-K split
  *   adds the fp32 partial sums of a cut tile in a fixed order: results are
  *   deterministic for a given GPU (SM count).
  *   PREFILL scales each weight row and each row of x by a power of two,
@@ -335,8 +336,8 @@ GNF4_API gnf4_status gnf4_dequant_debug(const uint8_t *w, const float *absmax, i
  *               counters at zero).
  * One launch of a tensor-core kernel (mma.sync, fp32 accumulation) over
  * batches of up to 8 rows and 64-element blocks of k, split over the SMs by
- * tile-stages of 256 weight rows. Numerics: the weight carried as two fp16
- * parts (within 1e-7 relative of NF4[code]); dy * absmax, exact in fp32,
+ * tile-stages of 256 weight rows. Numerics: the weight carried as its fp16
+ * rounding (relative error at most 2^-12); dy * absmax, exact in fp32,
  * scaled by a power of two per (row, 16 weight rows) and carried as two fp16
  * parts; fp32 sums, a fixed summation order (deterministic for a given GPU).
  * Alignment: dy and w 16-byte aligned, absmax 4, dx 2, workspace 16.
