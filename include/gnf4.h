@@ -442,13 +442,13 @@ GNF4_API gnf4_status gnf4_read_device_status(void *workspace, int32_t clear, uin
  * GNF4_NOALLOC_SCRATCH_BYTES bytes, reserved on every GPU that loads the
  * library for as long as the process runs. Nothing is allocated or freed.
  *  - The first call on a device looks up that array's device address (one
- *    runtime query, once per device, with that device current). Make that
- *    first call before starting any stream capture on the device.
+ *    runtime query, once per device, with that device current).
  *  - Problems whose decode-kernel workspace exceeds
  *    GNF4_NOALLOC_SCRATCH_BYTES are refused with GNF4_ERR_SCRATCH_LIMIT
- *    before anything is launched (the current decode kernel needs only the
- *    256-byte status header, so no problem size reaches the limit; callers
- *    should still handle the code).
+ *    before anything is launched (the decode kernel's workspace is the
+ *    status header plus its stream-K counters and partial sums, about
+ *    1.2 MB on a 148-SM GPU whatever the problem size, so the limit is not
+ *    reached there; callers should still handle the code).
  *  - All calls share the one array and it keeps the previous call's
  *    contents; each call first clears the part that must start at zero (an
  *    asynchronous memset on `stream`). Calls whose GPU work can overlap (on
