@@ -924,8 +924,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this stage's copies complete (full), so this one wait also orders
       // the copied weights and scales before the reads below
       if (!warp_wait_sa(kBarOff + (2 * kStages + st) * 8, ph, a.hdr)) return;
-      if (act0) {
-        // A block past K reads zero-filled activations and scales: it adds 0.
+      // a block past K (the last stage of a row whose K / 64 is not a
+      // multiple of 4) would only add the zeros its copies filled in
+      if (act0 && kc * kStageBlocks + blk < p.KB) {
         // (Shared-window addresses: region kXxx starts at address kXxx.)
         const uint32_t wst = kWOff + st * kWStage;
         // 2^-S of activation rows 2q and 2q + 1 in this block
